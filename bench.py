@@ -1,0 +1,440 @@
+#!/usr/bin/env python3
+"""Throughput of the W4A4 + low-rank linear layer on B200.
+
+Workload (one GPU): the Llama-3-8B attention projection in the decode
+regime, K = N = 4096, rank 32, Hadamard block 128, M = 16 tokens (other M via
+--m).  One "step" is one pass of the hot path -- tq_quantize_act (rotation,
+per-token INT4 codes, X L1) then tq_w4a4_lr_gemm (INT4 GEMM, INT32
+accumulation, bf16 low-rank branch, epilogue) -- over 16 distinct layers, so
+the 16 x 8.9 MB of packed weights (143 MB) exceed the 126 MB L2 and every
+layer streams its weights from HBM.  The offline weight packing is not part
+of a step.  A step is replayed as one CUDA graph.
+
+Metric: algorithmic GB/s of the layer (X + L1^T + Wq + s_w + L2^T + Y bytes
+per layer), the decode roofline quantity; TOPS (2 M N K) is reported beside it.
+
+--impl reference times the CPU oracle (fp64 C, the parity reference) on a
+bounded sample of the same workload.
+
+Multi-GPU (torchrun): every rank runs its own independent batch of layers
+(weak scaling, no data-path collective); rank 0 prints max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+low-rank linear TOPS and GB/s at Llama-3 shapes; % of INT8/HBM roofline"
+K_DIM = N_DIM = 4096
+RANK = 32
+HAD = 128
+LAYERS = 16
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--m", type=int, default=16, help="tokens per layer")
+    ap.add_argument("--layers", type=int, default=LAYERS)
+    ap.add_argument("--no-sweep", action="store_true", help="skip the M=1/128 side measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def layer_bytes(M, K, N, r):
+    """Algorithmic bytes of one layer: X + L1^T + Wq + s_w + L2^T + Y."""
+    return 2 * M * K + 2 * r * K + K * N // 2 + 4 * N + 2 * N * r + 2 * M * N
+
+
+def gemm_bytes(M, K, N, r):
+    """Compulsory bytes of the GEMM kernel: Xq + s_x + XL1 + Wq + s_w + L2^T + Y."""
+    return M * K // 2 + 4 * M + 4 * M * r + K * N // 2 + 4 * N + 2 * N * r + 2 * M * N
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
+    except Exception:
+        return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def profiled_traffic(kernel_src: str, profile: str):
+    """DRAM bytes per launch recorded in a committed ncu summary, or None when
+    the summary is missing or was taken on a different kernel source."""
+    try:
+        txt = open(os.path.join(ROOT, "profiles", profile)).read()
+        src = open(os.path.join(ROOT, kernel_src), "rb").read()
+    except OSError:
+        return None
+    m_h = re.search(r"source_sha256:\s*([0-9a-f]{64})", txt)
+    m_t = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", txt)
+    if not m_h or not m_t or m_h.group(1) != hashlib.sha256(src).hexdigest():
+        return None
+    return float(m_t.group(1))
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons through NVML while running."""
+
+    def __init__(self, index: int, period: float = 0.02):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        names = {
+            "hw_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwSlowdown", 0x8),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonHwThermalSlowdown", 0x40),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksThrottleReasonSwThermalSlowdown", 0x20),
+            "sw_power_cap": getattr(nv, "nvmlClocksThrottleReasonSwPowerCap", 0x4),
+        }
+        while True:
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            if self._stop.wait(self.period):
+                break
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        s = sorted(self.samples)
+        return {"sm_mhz": s[len(s) // 2] if s else None, "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(s)}
+
+
+# ----------------------------------------------------------------- GPU arm
+
+def build_layers(tq, torch, M, L, seed0, device):
+    import synth
+    sh = synth.CONFIGS["decode"].with_(M=M)
+    layers = []
+    for i in range(L):
+        w = synth.make_weights(sh, seed=seed0 + 10 * i, device="cuda")
+        Rt = w["Rt"].to(device)
+        Wq, s_w = tq.tq_pack_weight(Rt, HAD)
+        del Rt
+        lay = {
+            "X": synth.make_activations(sh, seed=seed0 + 10 * i).to(device),
+            "L1t": w["L1t"].to(device), "L2t": w["L2t"].to(device), "Wq": Wq, "s_w": s_w,
+            "Xq": torch.empty(M, K_DIM // 2, dtype=torch.uint8, device=device),
+            "s_x": torch.empty(M, dtype=torch.float32, device=device),
+            "XL1": torch.empty(M, RANK, dtype=torch.float32, device=device),
+            "Y": torch.empty(M, N_DIM, dtype=torch.bfloat16, device=device),
+            "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N_DIM, K_DIM, RANK),
+                              dtype=torch.uint8, device=device),
+        }
+        layers.append(lay)
+    torch.cuda.synchronize()
+    return layers
+
+
+def layer_call(tq, lay, ev=None):
+    tq.tq_quantize_act(lay["X"], HAD, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
+    if ev is not None:
+        ev[0].record()
+    tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"], lay["L2t"],
+                       Y=lay["Y"], workspace=lay["ws"])
+    if ev is not None:
+        ev[1].record()
+
+
+def capture(torch, fn):
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()  # one eager pass (function attributes, tensor maps) before capture
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s):
+            fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(torch, g, steps, warmup, dist=None):
+    for _ in range(warmup):
+        g.replay()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    return e0.elapsed_time(e1) / steps  # ms per step
+
+
+def run_tq(args, rank, world, local_rank, dist):
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M, L = args.m, args.layers
+    layers = build_layers(tq, torch, M, L, seed0=1000 * rank, device=dev)
+
+    def step():
+        for lay in layers:
+            layer_call(tq, lay)
+
+    g = capture(torch, step)
+
+    with ClockSampler(local_rank) as clk:
+        ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
+    clocks = clk.summary()
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # per-kernel durations of the same step, events captured in the graph
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in layers]
+
+    def step_ev():
+        for lay, ev in zip(layers, evs):
+            layer_call(tq, lay, ev)
+
+    g_ev = capture(torch, step_ev)
+    reps = max(1, min(args.steps, 50))
+    gemm_ms = []
+    for _ in range(max(3, args.warmup)):
+        g_ev.replay()
+    for _ in range(reps):
+        g_ev.replay()
+        torch.cuda.synchronize()
+        gemm_ms.extend(a.elapsed_time(b) for a, b in evs)
+    gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
+
+    # end to end: pinned host X in, host Y out, every step
+    hx = [lay["X"].cpu().pin_memory() for lay in layers]
+    hy = [torch.empty_like(lay["Y"], device="cpu").pin_memory() for lay in layers]
+
+    def step_e2e():
+        for lay, x, y in zip(layers, hx, hy):
+            lay["X"].copy_(x, non_blocking=True)
+            layer_call(tq, lay)
+            y.copy_(lay["Y"], non_blocking=True)
+
+    g_e2e = capture(torch, step_e2e)
+    ms_e2e = time_graph(torch, g_e2e, args.steps, args.warmup, dist if world > 1 else None)
+    if world > 1:
+        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    sweep = {}
+    if not args.no_sweep and world == 1:
+        for m2 in (1, 128):
+            if m2 == M:
+                continue
+            ls = build_layers(tq, torch, m2, L, seed0=7, device=dev)
+
+            def st(ls=ls):
+                for lay in ls:
+                    layer_call(tq, lay)
+
+            g2 = capture(torch, st)
+            ms2 = time_graph(torch, g2, args.steps, args.warmup)
+            b2 = L * layer_bytes(m2, K_DIM, N_DIM, RANK)
+            sweep[f"M={m2}"] = {"GB/s": round(b2 / ms2 / 1e6, 1), "us_per_layer": round(ms2 * 1e3 / L, 3),
+                                "TOPS": round(L * 2 * m2 * N_DIM * K_DIM / ms2 / 1e9, 3)}
+            del ls, g2
+
+    bytes_step = L * layer_bytes(M, K_DIM, N_DIM, RANK)
+    value = world * bytes_step / ms / 1e6          # GB/s, all ranks
+    e2e = world * bytes_step / ms_e2e / 1e6
+    peak, peak_src = measured_peaks()
+    gb = gemm_bytes(M, K_DIM, N_DIM, RANK)
+    achieved = gb / (gemm_ms_avg * 1e-3) / 1e9
+    traffic = profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm.cu",
+                               "w4a4_lr_gemm_decode_m16.md") if M == 16 else None
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic (seeded N(0,1) activations with 1% x30 outlier channels; "
+                "W = U diag(i^-1/2) V^T at std 0.02, random-init, no checkpoint)",
+        "config": {
+            "workload": f"Llama-3-8B attention projection, decode: M={M} tokens, K=N=4096, "
+                        f"rank {RANK}, Hadamard block {HAD}; {L} distinct layers per step",
+            "M": M, "K": K_DIM, "N": N_DIM, "r": RANK, "had_block": HAD,
+            "layers_per_step": L,
+            "l2": f"inputs larger than L2: {L} layers x {gb / 1e6:.1f} MB of GEMM operands",
+            "parallelism": f"{world} independent replica(s), no data-path collective",
+            "graph": "one CUDA graph per step; GEMM launched with programmatic dependent launch",
+        },
+        "TOPS": round(world * L * 2 * M * N_DIM * K_DIM / ms / 1e9, 3),
+        "us_per_layer": round(ms * 1e3 / L, 3),
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": "w4a4_lr_gemm_kernel (decode tiling, split-K)",
+            "gemm_us": round(gemm_ms_avg * 1e3, 3),
+            "algorithmic_bytes_per_launch": gb, "peak_source": peak_src,
+        },
+        "e2e": {"value": round(e2e, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hx),
+                "d2h_bytes_per_step": sum(y.numel() * y.element_size() for y in hy),
+                "ms_per_step": round(ms_e2e, 5)},
+        "gpu_launches": 2 * L * args.steps,
+        "clocks": clocks,
+    }
+    if sweep:
+        out["sweep"] = sweep
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(M, budget_s=12.0)
+    return out
+
+
+# ------------------------------------------------------------ oracle (CPU)
+
+def cpu_baseline(M, budget_s=12.0):
+    """The fp64 C oracle, as it stands, on a bounded sample of the workload:
+    repeated evaluations of one decode layer (rotation + codes + X L1,
+    integer GEMM, low-rank branch, epilogue; weights packed beforehand)."""
+    import numpy as np
+
+    import oracle
+    import synth
+
+    sh = synth.CONFIGS["decode"].with_(M=M)
+    L = synth.make_layer(sh, seed=0)
+    w = oracle.pack_weight(L["Rt"], HAD)          # offline, untimed
+    X, L1t, L2t = L["X"], L["L1t"], L["L2t"]
+    n, t0 = 0, time.perf_counter()
+    while True:
+        a = oracle.quantize_act(X, HAD)
+        acc = oracle.int_gemm(a["qx"], w["qw"])
+        _, lr = oracle.lowrank(X, L1t, L2t)
+        oracle.epilogue(a["s_x"], w["s_w"], acc, lr)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = (time.perf_counter() - t0) / n
+    val = layer_bytes(M, K_DIM, N_DIM, RANK) / dt / 1e9
+    return {"value": round(val, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n} evaluations of one decode layer (M={M}, K=N=4096, r=32), "
+                      f"{dt:.2f} s each; weights packed outside the timing",
+            "s_per_layer": round(dt, 3)}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step a bounded sample (one layer
+    of the same workload), timed on the host cores."""
+    import oracle
+    import synth
+
+    M = args.m
+    sh = synth.CONFIGS["decode"].with_(M=M)
+    L = synth.make_layer(sh, seed=0)
+    w = oracle.pack_weight(L["Rt"], HAD)
+    X, L1t, L2t = L["X"], L["L1t"], L["L2t"]
+
+    def one():
+        a = oracle.quantize_act(X, HAD)
+        acc = oracle.int_gemm(a["qx"], w["qw"])
+        _, lr = oracle.lowrank(X, L1t, L2t)
+        oracle.epilogue(a["s_x"], w["s_w"], acc, lr)
+
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    val = layer_bytes(M, K_DIM, N_DIM, RANK) / dt / 1e9
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"Llama-3-8B attention projection, decode: M={M} tokens, "
+                               f"K=N=4096, rank {RANK}, Hadamard block {HAD}; each step one layer",
+                   "M": M, "K": K_DIM, "N": N_DIM, "r": RANK, "had_block": HAD},
+        "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": "one decode layer per step (rotation, codes, X L1, integer "
+                                   "GEMM, low-rank branch, epilogue); weights packed untimed"},
+        "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args)))
+        return 0
+    dist = None
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    out = run_tq(args, rank, world, local_rank, dist)
+    if rank == 0:
+        print(json.dumps(out))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,157 @@
+/*
+ * tq.h -- C ABI of the B200 (sm_100a) W4A4 + low-rank linear layer.
+ *
+ *   Y = dequant( Q4(X H) . Q4(H^T R) ) + (X L1) L2
+ *
+ * H is the block-diagonal Sylvester Hadamard matrix (block b along K,
+ * normalised by 1/sqrt(b)); Q4 is the symmetric 4-bit quantizer of CoQuant
+ * Eq. (1) (zero-point 0, s = max|.| / 7, RoundClip to [-7, 7]), applied per
+ * token to the rotated activations and per output channel to the rotated
+ * residual; the integer product accumulates in INT32 (TwinQuant notes,
+ * section 04.C, Figure 4); the bf16 low-rank branch (X L1) L2 is the U V term
+ * of the SVDQuant-style split (TwinQuant notes, section 02.A) and both
+ * branches meet in one epilogue (TwinQuant, "single epilogue" of the fused
+ * dual-component kernel).  The rotation rests on CoQuant Eq. (3):
+ * (X H)(H^T W) = X W for orthogonal H.
+ *
+ * Conventions shared by every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller; the library
+ *    allocates nothing on these paths.  Calls are asynchronous on `stream`
+ *    (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *  - Matrices are row-major with K (the reduction / in-feature dimension)
+ *    contiguous, the nn.Linear [out][in] convention: X [M][K], R^T [N][K],
+ *    L1^T [r][K], L2^T [N][r], Y [M][N].  bf16 data is passed as uint16_t
+ *    bit patterns.
+ *  - Packed int4 codes ("Xq", "Wq") are [rows][K/2] bytes.  Within every
+ *    group of 32 consecutive codes (16 bytes) byte i holds code i in the low
+ *    nibble and code i+16 in the high nibble, each a 4-bit two's complement
+ *    number in [-7, 7] (-8 is never produced).
+ *  - Scales are fp32: s_x[m] = max_k |(X H)[m,k]| / 7, s_w[n] likewise over
+ *    row n of R^T H.  A row that is all zero gets scale 0 and all codes 0.
+ *  - Shape limits: M >= 1; 128 <= K <= 32768 with K % 128 == 0;
+ *    had_block in {1, 2, 4, ..., 256} (1 = no rotation) dividing K;
+ *    N >= 8 with N % 8 == 0; r = 0 or a multiple of 16 up to 512.
+ *    Every pointer must be 16-byte aligned.
+ *  - Inputs must be finite.  Rounding is round-half-to-even everywhere.
+ *  - Errors are returned synchronously before anything is launched
+ *    (TQ_ERR_INVALID_VALUE, TQ_ERR_UNSUPPORTED_SHAPE, TQ_ERR_MISALIGNED,
+ *    TQ_ERR_WORKSPACE, TQ_ERR_NO_DEVICE); a failed launch returns
+ *    TQ_ERR_CUDA.  Kernel-side watchdog timeouts (a pipeline wait that never
+ *    completes) are recorded in the GEMM workspace and reported by
+ *    tq_query_device_status.  No call aborts the process.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TQ_API __attribute__((visibility("default")))
+#else
+#define TQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_VALUE = 1,     /* null pointer, non-positive size          */
+  TQ_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the limits above           */
+  TQ_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned         */
+  TQ_ERR_CUDA = 4,              /* CUDA launch or runtime error             */
+  TQ_ERR_TIMEOUT = 5,           /* a kernel's bounded wait gave up          */
+  TQ_ERR_WORKSPACE = 6,         /* workspace missing or too small           */
+  TQ_ERR_NO_DEVICE = 7          /* current device is not an sm_100 GPU      */
+} tq_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+TQ_API const char* tq_status_string(int status);
+
+/* ABI version of this library (major * 100 + minor). */
+TQ_API int tq_version(void);
+
+/*
+ * tq_pack_weight -- offline rotation + per-output-channel INT4 quantization
+ * of the residual (CoQuant Eq. (3): the weight side of (X H)(H^T W); Eq. (1)
+ * per channel; CoQuant's protocol uses per-channel symmetric weights).
+ *
+ *   Rt   [N][K] fp32  in : R^T, the residual in nn.Linear layout
+ *   Wq   [N][K/2] u8 out : packed int4 codes of row n of R^T H
+ *   s_w  [N] fp32    out : per-channel scales
+ * Not on the per-token path: run once per layer.
+ */
+TQ_API int tq_pack_weight(const float* Rt, int N, int K, int had_block,
+                   uint8_t* Wq, float* s_w, void* stream);
+
+/*
+ * tq_quantize_act -- online rotation X H (one 128-wide or had_block-wide
+ * fast Walsh-Hadamard transform per block), symmetric per-token INT4
+ * quantization (CoQuant Eq. (1); TwinQuant notes section 02) and the
+ * low-rank down-projection X L1 (TwinQuant notes section 02.A), all from one
+ * read of X.
+ *
+ *   X    [M][K] bf16    in : activations
+ *   L1t  [r][K] bf16    in : L1^T (down-projection weight); NULL iff r == 0
+ *   Xq   [M][K/2] u8   out : packed codes of X H
+ *   s_x  [M] fp32      out : per-token scales
+ *   XL1  [M][r] fp32   out : X L1 (unrotated, unquantized X); NULL iff r == 0
+ */
+TQ_API int tq_quantize_act(const uint16_t* X, int M, int K, int had_block,
+                    const uint16_t* L1t, int r,
+                    uint8_t* Xq, float* s_x, float* XL1, void* stream);
+
+/*
+ * Bytes of device workspace tq_w4a4_lr_gemm needs for this shape (always at
+ * least 256).  The workspace must be zero-filled once before its first use;
+ * every call leaves its counters zero again, so it can be reused by later
+ * calls on the same stream (not by concurrent calls).
+ */
+TQ_API size_t tq_gemm_workspace_bytes(int M, int N, int K, int r);
+
+/*
+ * tq_w4a4_lr_gemm -- the layer's main kernel (TwinQuant's fused
+ * dual-component kernel, bf16 low-rank form):
+ *
+ *   Y[m][n] = bf16( s_x[m] s_w[n] sum_k qx[m][k] qw[n][k]
+ *                   + sum_j bf16(XL1[m][j]) L2t[n][j] )
+ *
+ * the integer sum exact in INT32, the low-rank sum in fp32.
+ *   Xq, s_x, XL1   : outputs of tq_quantize_act (XL1 NULL iff r == 0)
+ *   Wq, s_w        : outputs of tq_pack_weight
+ *   L2t [N][r] bf16: L2^T (up-projection weight); NULL iff r == 0
+ *   Y   [M][N] bf16: output
+ *   workspace      : >= tq_gemm_workspace_bytes(M, N, K, r) bytes, zeroed
+ *                    before first use (see above)
+ */
+TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
+                    const uint8_t* Wq, const float* s_w,
+                    const float* XL1, const uint16_t* L2t,
+                    int M, int N, int K, int r, uint16_t* Y,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * tq_debug_w4a4_gemm_acc -- test hook: the same GEMM kernel with the
+ * low-rank branch off, writing the raw INT32 accumulators
+ * acc[m][n] = sum_k qx[m][k] qw[n][k] to `acc` [M][N] (int32) instead of Y.
+ * Lets a caller check the integer path bit-exactly on codes of its choice.
+ */
+TQ_API int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq,
+                           int M, int N, int K, int32_t* acc,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * tq_query_device_status -- synchronises `stream`, then reads the status word
+ * kernels record in `workspace` (a GEMM workspace) and clears it.  Returns
+ * TQ_OK, TQ_ERR_TIMEOUT if a bounded in-kernel wait gave up since the last
+ * query, or TQ_ERR_CUDA.
+ */
+TQ_API int tq_query_device_status(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H_ */

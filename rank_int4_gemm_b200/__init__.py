@@ -1,0 +1,12 @@
+"""B200 (sm_100a) W4A4 + low-rank linear layer.
+
+The compute lives in libtq.so (hand-written CUDA for sm_100a behind the C ABI
+of include/tq.h); this package only marshals torch tensors into that ABI.
+There is no CPU fallback: importing the binding without the built library
+raises.
+"""
+from .tq import (  # noqa: F401
+    TQError, lib_path, tq_status_string, tq_version, tq_pack_weight, tq_quantize_act,
+    tq_gemm_workspace_bytes, tq_w4a4_lr_gemm, tq_debug_w4a4_gemm_acc,
+    tq_query_device_status, Workspace, layer_forward,
+)

@@ -1,0 +1,477 @@
+// tq_act.cu -- rotation + symmetric INT4 quantization kernels.
+//
+//  * quantize_act_kernel: the per-token activation stage.  One thread-block
+//    cluster owns 16 tokens; its C CTAs split K.  Each warp owns one token,
+//    holds its slice of X in registers, applies the Sylvester fast
+//    Walsh-Hadamard transform per block (in-register butterflies, then
+//    shuffles), and the cluster combines the per-slice absmax through
+//    distributed shared memory before every CTA writes its packed codes.  The
+//    same read of X feeds the X.L1 down-projection on tensor cores
+//    (mma.sync bf16, fp32 accumulation), reduced across the cluster in a fixed
+//    order, so results are deterministic.
+//  * pack_weight_kernel: the offline per-output-channel weight stage (one CTA
+//    per row of R^T, transform in shared memory).
+//
+// Quantizer: CoQuant Eq. (1), symmetric, s = max|x| / 7, RoundClip to
+// [-7, 7]; rotation: CoQuant Eq. (3) with a Hadamard U.  The transform is
+// computed unnormalised; the 1/sqrt(b) factor cancels in the codes and is
+// folded into the stored scale.
+#include <cuda_bf16.h>
+
+#include "tq_internal.h"
+#include "tq_ptx.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kActRows = 16;       // tokens per cluster (one warp each)
+constexpr int kActThreads = 512;   // 16 warps
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+  return v;
+}
+
+// Unnormalised Sylvester transform over blocks of b consecutive values; a lane
+// holds E consecutive values, so a block spans b/E lanes when b > E.
+template <int E>
+__device__ __forceinline__ void fwht_warp(float (&v)[E], int b) {
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+    if (h < b) {
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        if ((i & h) == 0) {
+          const float a = v[i], c = v[i + h];
+          v[i] = a + c;
+          v[i + h] = a - c;
+        }
+      }
+    }
+  }
+  const uint32_t lane = threadIdx.x & 31u;
+  for (int s = 1; s * E < b; s <<= 1) {
+    const bool upper = (lane & (uint32_t)s) != 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float o = __shfl_xor_sync(kFull, v[i], s);
+      v[i] = upper ? (o - v[i]) : (v[i] + o);
+    }
+  }
+}
+
+// RoundClip(v * inv) with ties to even.
+__device__ __forceinline__ int quant_code(float v, float inv) {
+  float t = rintf(v * inv);
+  t = fminf(fmaxf(t, -7.f), 7.f);
+  return (int)t;
+}
+
+// Writes the E codes of this lane into the packed layout: inside a 32-code
+// group byte i = code i | code (i+16) << 4.  The lanes holding codes i and
+// i+16 of a group exchange nibbles and each writes half of their bytes.
+// `row_bytes` points at the byte of the row where this warp pass starts.
+template <int E>
+__device__ __forceinline__ void store_packed(const int (&q)[E], uint8_t* row_bytes) {
+  constexpr int G = 32 / E;  // lanes per 32-code group
+  constexpr int H = G / 2;   // lanes holding the low nibbles
+  uint64_t mine = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) mine |= (uint64_t)(q[i] & 0xF) << (4 * i);
+  const int lane = (int)(threadIdx.x & 31u);
+  const uint64_t other = __shfl_xor_sync(kFull, mine, H);
+  const int a = lane % G;
+  const bool low_side = a < H;
+  const uint64_t lo = low_side ? mine : other;
+  const uint64_t hi = low_side ? other : mine;
+  const int nib0 = low_side ? 0 : E / 2;
+  uint64_t out = 0;
+#pragma unroll
+  for (int i = 0; i < E / 2; ++i) {
+    const uint64_t l = (lo >> (4 * (nib0 + i))) & 0xFull;
+    const uint64_t h = (hi >> (4 * (nib0 + i))) & 0xFull;
+    out |= (l | (h << 4)) << (8 * i);
+  }
+  uint8_t* dst = row_bytes + (lane / G) * 16 + (a % H) * E + nib0;
+  if constexpr (E == 16) {
+    *reinterpret_cast<uint64_t*>(dst) = out;
+  } else if constexpr (E == 8) {
+    *reinterpret_cast<uint32_t*>(dst) = (uint32_t)out;
+  } else {
+    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)out;
+  }
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x2(uint32_t (&r)[2], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
+                                          const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+struct ActParams {
+  const __nv_bfloat16* X;
+  const __nv_bfloat16* L1t;
+  uint8_t* Xq;
+  float* s_x;
+  float* XL1;
+  int M, K, b, r;
+  int passes_per_cta;  // P
+  int total_passes;    // K / W
+  int kc;              // L1 k-chunk (columns) staged per step
+  float scale_mul;     // 1 / (7 sqrt(b))
+};
+
+// Shared-memory carve-up of quantize_act_kernel.
+template <int E>
+struct ActSmem {
+  static constexpr int W = 32 * E;
+  int xs_stride;   // bf16 elements per X row (slice + 8 pad)
+  int l1_stride;   // bf16 elements per staged L1^T row (kc + 8 pad)
+  size_t off_l1, off_part, off_amax, total;
+  __host__ __device__ ActSmem(int P, int r, int kc) {
+    xs_stride = P * W + 8;
+    l1_stride = kc + 8;
+    size_t xs_bytes = (size_t)kActRows * xs_stride * 2;
+    off_l1 = (xs_bytes + 127) & ~size_t(127);
+    size_t l1_bytes = (size_t)2 * r * l1_stride * 2;
+    off_part = (off_l1 + l1_bytes + 127) & ~size_t(127);
+    size_t part_bytes = (size_t)kActRows * r * 4;
+    off_amax = (off_part + part_bytes + 127) & ~size_t(127);
+    total = off_amax + 2 * kActRows * 4;
+  }
+};
+
+template <int E>
+__global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActParams p) {
+  constexpr int W = 32 * E;
+  constexpr int PMAX = 64 / E;  // register budget: PMAX * E values per lane
+  extern __shared__ __align__(128) uint8_t smem[];
+
+  pdl_launch_dependents();  // let the GEMM start streaming its weights
+  pdl_wait();
+
+  const int P = p.passes_per_cta;
+  const ActSmem<E> L(P, p.r, p.kc);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* l1s = reinterpret_cast<__nv_bfloat16*>(smem + L.off_l1);
+  float* part = reinterpret_cast<float*>(smem + L.off_part);
+  float* amax_part = reinterpret_cast<float*>(smem + L.off_amax);
+  float* amax_row = amax_part + kActRows;
+
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const int pass0 = (int)crank * P;
+  const int np = min(P, p.total_passes - pass0);
+  const int slice = np * W;
+  const int kbase = pass0 * W;
+  const int row0 = blockIdx.y * kActRows;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+
+  // ---- stage X[row0:row0+16][kbase:kbase+slice] (zero rows past M)
+  {
+    const int chunks_per_row = slice / 8;  // 16-byte chunks
+    for (int c = tid; c < kActRows * chunks_per_row; c += kActThreads) {
+      const int rr = c / chunks_per_row, cc = c % chunks_per_row;
+      const int gm = row0 + rr;
+      const bool ok = gm < p.M;
+      const __nv_bfloat16* src = p.X + (size_t)(ok ? gm : 0) * p.K + kbase + cc * 8;
+      cp_async16(xs + (size_t)rr * L.xs_stride + cc * 8, src, ok);
+    }
+    cp_async_commit();
+  }
+  // ---- first L1^T chunk
+  const int nchunks = (p.r > 0) ? slice / p.kc : 0;
+  auto stage_l1 = [&](int ci, int buf) {
+    const int cpr = p.kc / 8;
+    __nv_bfloat16* dst = l1s + (size_t)buf * p.r * L.l1_stride;
+    for (int c = tid; c < p.r * cpr; c += kActThreads) {
+      const int j = c / cpr, cc = c % cpr;
+      const __nv_bfloat16* src = p.L1t + (size_t)j * p.K + kbase + ci * p.kc + cc * 8;
+      cp_async16(dst + (size_t)j * L.l1_stride + cc * 8, src, true);
+    }
+    cp_async_commit();
+  };
+  if (nchunks > 0) stage_l1(0, 0);
+
+  cp_async_wait<1>();  // X landed (the L1 chunk may still be in flight)
+  if (nchunks == 0) cp_async_wait<0>();
+  __syncthreads();
+
+  // ---- rotation of this warp's token: PMAX passes of W columns
+  float v[PMAX][E];
+  float amax = 0.f;
+  const int my_row = row0 + warp;
+#pragma unroll
+  for (int ps = 0; ps < PMAX; ++ps) {
+    if (ps < np) {
+      const __nv_bfloat16* src = xs + (size_t)warp * L.xs_stride + ps * W + lane * E;
+      if constexpr (E >= 8) {
+#pragma unroll
+        for (int i = 0; i < E; i += 8) {  // 16-byte aligned: lane * E * 2 bytes
+          const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(h2[j]);
+            v[ps][i + 2 * j] = f.x;
+            v[ps][i + 2 * j + 1] = f.y;
+          }
+        }
+      } else {  // E == 4: one 8-byte load
+        const uint2 u = *reinterpret_cast<const uint2*>(src);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float2 f = __bfloat1622float2(h2[j]);
+          v[ps][2 * j] = f.x;
+          v[ps][2 * j + 1] = f.y;
+        }
+      }
+      fwht_warp<E>(v[ps], p.b);
+#pragma unroll
+      for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[ps][i]));
+    }
+  }
+  amax = warp_max(amax);
+  if (lane == 0) amax_part[warp] = amax;
+
+  // ---- X L1 partial over this CTA's slice: warps own 8-column tiles of r
+  if (nchunks > 0) {
+    const int ntiles = p.r / 8;
+    constexpr int kMaxTilesPerWarp = 4;  // r <= 512
+    float acc[kMaxTilesPerWarp][4];
+#pragma unroll
+    for (int t = 0; t < kMaxTilesPerWarp; ++t)
+      acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+    const uint32_t xs_base = smem_u32(xs);
+    for (int ci = 0; ci < nchunks; ++ci) {
+      if (ci + 1 < nchunks) {
+        stage_l1(ci + 1, (ci + 1) & 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      __syncthreads();
+      const uint32_t l1_base = smem_u32(l1s + (size_t)(ci & 1) * p.r * L.l1_stride);
+      for (int kk = 0; kk < p.kc; kk += 16) {
+        uint32_t a[4];
+        {
+          const int mat = lane >> 3, rin = lane & 7;
+          const int rr = rin + (mat & 1) * 8;
+          const int cc = ci * p.kc + kk + (mat >> 1) * 8;
+          ldmatrix_x4(a, xs_base + (uint32_t)((rr * L.xs_stride + cc) * 2));
+        }
+#pragma unroll
+        for (int t = 0; t < kMaxTilesPerWarp; ++t) {
+          const int tile = warp + 16 * t;
+          if (tile < ntiles) {
+            uint32_t bb[2];
+            const int l = lane & 15;
+            const int jr = tile * 8 + (l & 7);
+            const int cc = kk + (l >> 3) * 8;
+            ldmatrix_x2(bb, l1_base + (uint32_t)((jr * L.l1_stride + cc) * 2));
+            mma_16816(acc[t], a, bb);
+          }
+        }
+      }
+      __syncthreads();  // buffer (ci & 1) is refilled two chunks later
+    }
+    // C fragment: rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
+#pragma unroll
+    for (int t = 0; t < kMaxTilesPerWarp; ++t) {
+      const int tile = warp + 16 * t;
+      if (tile < ntiles) {
+        const int rr = lane >> 2, cc = tile * 8 + 2 * (lane & 3);
+        part[rr * p.r + cc] = acc[t][0];
+        part[rr * p.r + cc + 1] = acc[t][1];
+        part[(rr + 8) * p.r + cc] = acc[t][2];
+        part[(rr + 8) * p.r + cc + 1] = acc[t][3];
+      }
+    }
+  }
+
+  cluster_sync();  // partial absmax and X L1 of every CTA are visible
+
+  if (tid < kActRows) {
+    const uint32_t a_addr = smem_u32(&amax_part[tid]);
+    float m = 0.f;
+    for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, dsmem_ld_f32(dsmem_map(a_addr, c)));
+    amax_row[tid] = m;
+  }
+  __syncthreads();
+
+  // ---- codes of this CTA's slice
+  if (my_row < p.M) {
+    const float am = amax_row[warp];
+    const float inv = am > 0.f ? 7.f / am : 0.f;
+    uint8_t* xrow = p.Xq + (size_t)my_row * (p.K / 2);
+#pragma unroll
+    for (int ps = 0; ps < PMAX; ++ps) {
+      if (ps < np) {
+        int q[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) q[i] = quant_code(v[ps][i], inv);
+        store_packed<E>(q, xrow + (kbase + ps * W) / 2);
+      }
+    }
+    if (crank == 0 && lane == 0) p.s_x[my_row] = am * p.scale_mul;
+  }
+
+  // ---- leader: X L1 = sum over the cluster's CTAs, in rank order
+  if (crank == 0 && p.r > 0) {
+    const uint32_t part_addr = smem_u32(part);
+    for (int idx = tid; idx < kActRows * p.r; idx += kActThreads) {
+      const int rr = idx / p.r;
+      if (row0 + rr >= p.M) continue;
+      float s = 0.f;
+      for (uint32_t c = 0; c < csize; ++c)
+        s += dsmem_ld_f32(dsmem_map(part_addr + (uint32_t)idx * 4u, c));
+      p.XL1[(size_t)(row0 + rr) * p.r + (idx % p.r)] = s;
+    }
+  }
+
+  cluster_sync();  // keep shared memory alive until every peer has read it
+}
+
+// ------------------------------------------------------------ weight pack
+
+constexpr int kPackThreads = 256;
+
+__global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const float* __restrict__ Rt,
+                                                                   int K, int b, float scale_mul,
+                                                                   uint8_t* __restrict__ Wq,
+                                                                   float* __restrict__ s_w) {
+  extern __shared__ __align__(16) float row[];
+  __shared__ float red[kPackThreads / 32];
+  const int n = blockIdx.x;
+  const float* src = Rt + (size_t)n * K;
+  for (int k = threadIdx.x * 4; k < K; k += kPackThreads * 4)
+    *reinterpret_cast<float4*>(row + k) = *reinterpret_cast<const float4*>(src + k);
+  __syncthreads();
+  // in-place Sylvester butterflies, level by level (pairs never cross blocks)
+  for (int h = 1; h < b; h <<= 1) {
+    for (int t = threadIdx.x; t < K / 2; t += kPackThreads) {
+      const int i = (t / h) * 2 * h + (t % h);
+      const float a = row[i], c = row[i + h];
+      row[i] = a + c;
+      row[i + h] = a - c;
+    }
+    __syncthreads();
+  }
+  float m = 0.f;
+  for (int k = threadIdx.x; k < K; k += kPackThreads) m = fmaxf(m, fabsf(row[k]));
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float mm = threadIdx.x < kPackThreads / 32 ? red[threadIdx.x] : 0.f;
+    mm = warp_max(mm);
+    if (threadIdx.x == 0) red[0] = mm;
+  }
+  __syncthreads();
+  const float amax = red[0];
+  const float inv = amax > 0.f ? 7.f / amax : 0.f;
+  uint8_t* dst = Wq + (size_t)n * (K / 2);
+  for (int byte = threadIdx.x; byte < K / 2; byte += kPackThreads) {
+    const int g = byte / 16, i = byte % 16;
+    const int lo = quant_code(row[g * 32 + i], inv);
+    const int hi = quant_code(row[g * 32 + 16 + i], inv);
+    dst[byte] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+  }
+  if (threadIdx.x == 0) s_w[n] = amax * scale_mul;
+}
+
+template <int E>
+cudaError_t launch_act_e(const ActParams& prm_in, cudaStream_t stream) {
+  constexpr int W = 32 * E;
+  constexpr int PMAX = 64 / E;
+  ActParams prm = prm_in;
+  const int tp = prm.K / W;
+  int P = (tp + 7) / 8;          // portable clusters (<= 8 CTAs) when possible
+  if (P > PMAX) P = (tp + 15) / 16;
+  if (P > PMAX) return cudaErrorInvalidValue;
+  const int C = (tp + P - 1) / P;
+  prm.passes_per_cta = P;
+  prm.total_passes = tp;
+  prm.kc = prm.r > 256 ? 32 : (prm.r > 128 ? 64 : 128);
+  const ActSmem<E> L(P, prm.r, prm.kc);
+  auto kern = quantize_act_kernel<E>;
+  static uint64_t attr_set = 0;  // one bit per device
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_set >> dev & 1u)) {
+    // the largest carve-up any supported shape needs (P * W <= 2048, r <= 512)
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)ActSmem<E>(PMAX, 512, 32).total);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, (prm.M + kActRows - 1) / kActRows, 1);
+  cfg.blockDim = dim3(kActThreads, 1, 1);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
+                                const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
+                                cudaStream_t stream) {
+  ActParams prm{};
+  prm.X = reinterpret_cast<const __nv_bfloat16*>(X);
+  prm.L1t = reinterpret_cast<const __nv_bfloat16*>(L1t);
+  prm.Xq = Xq;
+  prm.s_x = s_x;
+  prm.XL1 = XL1;
+  prm.M = M;
+  prm.K = K;
+  prm.b = had_block;
+  prm.r = r;
+  prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  if (K % 512 == 0 && had_block <= 512) return launch_act_e<16>(prm, stream);
+  if (K % 256 == 0 && had_block <= 256) return launch_act_e<8>(prm, stream);
+  if (had_block <= 128) return launch_act_e<4>(prm, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
+                               float* s_w, cudaStream_t stream) {
+  const size_t smem = (size_t)K * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  pack_weight_kernel<<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -1,0 +1,160 @@
+// tq_api.cu -- the C ABI declared in include/tq.h: argument validation, then
+// one launch per call on the caller's stream.  No allocation, no host sync
+// (except tq_query_device_status, which exists to synchronise).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "../../include/tq.h"
+#include "tq_internal.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool pow2_block(int b) { return b >= 1 && b <= 256 && (b & (b - 1)) == 0; }
+
+int check_device() {
+  static int cached = -1;
+  if (cached < 0) {
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return TQ_ERR_NO_DEVICE;
+    }
+    cached = (major == 10) ? TQ_OK : TQ_ERR_NO_DEVICE;
+  }
+  return cached;
+}
+
+int check_k(int K, int had_block) {
+  if (K < 128 || K > 32768 || K % 128 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if (!pow2_block(had_block) || K % had_block != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  return TQ_OK;
+}
+
+int check_r(int r) {
+  if (r < 0) return TQ_ERR_INVALID_VALUE;
+  if (r % 16 != 0 || r > 512) return TQ_ERR_UNSUPPORTED_SHAPE;
+  return TQ_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char* tq_status_string(int status) {
+  switch (status) {
+    case TQ_OK: return "TQ_OK";
+    case TQ_ERR_INVALID_VALUE: return "TQ_ERR_INVALID_VALUE";
+    case TQ_ERR_UNSUPPORTED_SHAPE: return "TQ_ERR_UNSUPPORTED_SHAPE";
+    case TQ_ERR_MISALIGNED: return "TQ_ERR_MISALIGNED";
+    case TQ_ERR_CUDA: return "TQ_ERR_CUDA";
+    case TQ_ERR_TIMEOUT: return "TQ_ERR_TIMEOUT";
+    case TQ_ERR_WORKSPACE: return "TQ_ERR_WORKSPACE";
+    case TQ_ERR_NO_DEVICE: return "TQ_ERR_NO_DEVICE";
+    default: return "TQ_ERR_UNKNOWN";
+  }
+}
+
+int tq_version(void) { return 100; }
+
+int tq_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq, float* s_w,
+                   void* stream) {
+  if (!Rt || !Wq || !s_w || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (!aligned16(Rt) || !aligned16(Wq) || !aligned16(s_w)) return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_pack_weight(Rt, N, K, had_block, Wq, s_w,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int tq_quantize_act(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t, int r,
+                    uint8_t* Xq, float* s_x, float* XL1, void* stream) {
+  if (!X || !Xq || !s_x || M <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1 != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(s_x) || (r > 0 && !aligned16(L1t)) ||
+      (r > 0 && !aligned16(XL1)))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x, XL1,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t tq_gemm_workspace_bytes(int M, int N, int K, int r) {
+  if (M <= 0 || N <= 0 || K <= 0) return 256;
+  return tq::gemm_workspace_bytes(M, N, K, r);
+}
+
+static int gemm_common(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w,
+                       const float* XL1, const uint16_t* L2t, int M, int N, int K, int r,
+                       uint16_t* Y, int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
+  if (!Xq || !Wq || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (!Y && !acc) return TQ_ERR_INVALID_VALUE;
+  if (Y && (!s_x || !s_w)) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (XL1 != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Xq) || !aligned16(Wq) || (s_x && !aligned16(s_x)) ||
+      (s_w && !aligned16(s_w)) || (XL1 && !aligned16(XL1)) || (L2t && !aligned16(L2t)) ||
+      (Y && !aligned16(Y)) || (acc && !aligned16(acc)) || (ws && !aligned16(ws)))
+    return TQ_ERR_MISALIGNED;
+  if (!ws || ws_bytes < tq::gemm_workspace_bytes(M, N, K, r)) return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  tq::GemmArgs a{};
+  a.Xq = Xq;
+  a.s_x = s_x;
+  a.Wq = Wq;
+  a.s_w = s_w;
+  a.XL1 = XL1;
+  a.L2t = L2t;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.Y = Y;
+  a.acc_out = acc;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return from_cuda(tq::launch_gemm(a, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w,
+                    const float* XL1, const uint16_t* L2t, int M, int N, int K, int r,
+                    uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Y) return TQ_ERR_INVALID_VALUE;
+  return gemm_common(Xq, s_x, Wq, s_w, XL1, L2t, M, N, K, r, Y, nullptr, workspace,
+                     workspace_bytes, stream);
+}
+
+int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq, int M, int N, int K,
+                           int32_t* acc, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!acc) return TQ_ERR_INVALID_VALUE;
+  return gemm_common(Xq, nullptr, Wq, nullptr, nullptr, nullptr, M, N, K, 0, nullptr, acc,
+                     workspace, workspace_bytes, stream);
+}
+
+int tq_query_device_status(void* workspace, void* stream) {
+  if (!workspace) return TQ_ERR_INVALID_VALUE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, workspace, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return TQ_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyAsync(workspace, &zero, 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    return TQ_ERR_TIMEOUT;
+  }
+  return TQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,40 @@
+// tq_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace tq {
+
+// Host-side knobs for experiments (0 = automatic choice).
+struct Tuning {
+  int split_k = 0;        // decode GEMM: number of K splits
+  int pdl = 1;            // launch the GEMM with programmatic dependent launch
+};
+Tuning& tuning();
+
+cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
+                               float* s_w, cudaStream_t stream);
+
+cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
+                                const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
+                                float* XL1, cudaStream_t stream);
+
+struct GemmArgs {
+  const uint8_t* Xq;
+  const float* s_x;
+  const uint8_t* Wq;
+  const float* s_w;
+  const float* XL1;
+  const uint16_t* L2t;
+  int M, N, K, r;
+  uint16_t* Y;          // bf16 output (null in accumulator-debug mode)
+  int32_t* acc_out;     // raw accumulators (debug mode only)
+  void* ws;
+  size_t ws_bytes;
+};
+
+size_t gemm_workspace_bytes(int M, int N, int K, int r);
+cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream);
+
+}  // namespace tq

@@ -1,0 +1,185 @@
+"""ctypes binding of libtq.so: argument marshalling only.
+
+Every function has the name of the C entry point it calls and forwards torch
+tensors as raw device pointers plus the current CUDA stream.  Outputs that the
+caller does not pass are allocated with torch (plumbing); nothing is computed
+here.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(
+        f"{_LIB_PATH} is missing: build it with `python -m rank_int4_gemm_b200.build_lib` "
+        "(there is no fallback implementation)")
+
+_lib = ctypes.CDLL(_LIB_PATH)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+_lib.tq_status_string.restype = ctypes.c_char_p
+_lib.tq_status_string.argtypes = [_I]
+_lib.tq_version.restype = _I
+_lib.tq_pack_weight.restype = _I
+_lib.tq_pack_weight.argtypes = [_P, _I, _I, _I, _P, _P, _P]
+_lib.tq_quantize_act.restype = _I
+_lib.tq_quantize_act.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]
+_lib.tq_gemm_workspace_bytes.restype = ctypes.c_size_t
+_lib.tq_gemm_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.tq_w4a4_lr_gemm.restype = _I
+_lib.tq_w4a4_lr_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
+                                  ctypes.c_size_t, _P]
+_lib.tq_debug_w4a4_gemm_acc.restype = _I
+_lib.tq_debug_w4a4_gemm_acc.argtypes = [_P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
+_lib.tq_query_device_status.restype = _I
+_lib.tq_query_device_status.argtypes = [_P, _P]
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {tq_status_string(status)} ({status})")
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def raw() -> ctypes.CDLL:
+    """The loaded C library (for callers passing raw pointers)."""
+    return _lib
+
+
+def tq_status_string(status: int) -> str:
+    return _lib.tq_status_string(int(status)).decode()
+
+
+def tq_version() -> int:
+    return int(_lib.tq_version())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise TQError(st, where)
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name}: expected contiguous CUDA {dtype} {tuple(shape)}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def tq_pack_weight(Rt: torch.Tensor, had_block: int, Wq=None, s_w=None, stream=None):
+    """R^T [N][K] fp32 -> (Wq [N][K/2] uint8, s_w [N] fp32)."""
+    N, K = Rt.shape
+    _need(Rt, torch.float32, (N, K), "Rt")
+    if Wq is None:
+        Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=Rt.device)
+    if s_w is None:
+        s_w = torch.empty(N, dtype=torch.float32, device=Rt.device)
+    _check(_lib.tq_pack_weight(_ptr(Rt), N, K, int(had_block), _ptr(Wq), _ptr(s_w),
+                               _stream(stream)), "tq_pack_weight")
+    return Wq, s_w
+
+
+def tq_quantize_act(X: torch.Tensor, had_block: int, L1t=None, Xq=None, s_x=None, XL1=None,
+                    stream=None):
+    """X [M][K] bf16 (+ L1^T [r][K] bf16) -> (Xq [M][K/2] u8, s_x [M] f32, XL1 [M][r] f32)."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, (M, K), "X")
+    r = 0 if L1t is None else L1t.shape[0]
+    if r:
+        _need(L1t, torch.bfloat16, (r, K), "L1t")
+    dev = X.device
+    if Xq is None:
+        Xq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    if r and XL1 is None:
+        XL1 = torch.empty(M, r, dtype=torch.float32, device=dev)
+    _check(_lib.tq_quantize_act(_ptr(X), M, K, int(had_block), _ptr(L1t) if r else None, r,
+                                _ptr(Xq), _ptr(s_x), _ptr(XL1) if r else None, _stream(stream)),
+           "tq_quantize_act")
+    return Xq, s_x, (XL1 if r else None)
+
+
+def tq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return int(_lib.tq_gemm_workspace_bytes(M, N, K, r))
+
+
+class Workspace:
+    """A zero-filled device workspace that grows on demand (plumbing)."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, workspace=None,
+                    stream=None):
+    """Y [M][N] bf16 = s_x s_w (Xq . Wq) + bf16(XL1) L2^T."""
+    M, K2 = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * K2
+    r = 0 if XL1 is None else XL1.shape[1]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
+    if workspace is None:
+        workspace = Workspace(Xq.device)
+    need = tq_gemm_workspace_bytes(M, N, K, r)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_gemm(_ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(s_w),
+                                _ptr(XL1) if r else None, _ptr(L2t) if r else None,
+                                M, N, K, r, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
+           "tq_w4a4_lr_gemm")
+    return Y
+
+
+def tq_debug_w4a4_gemm_acc(Xq, Wq, acc=None, workspace=None, stream=None):
+    """Raw INT32 accumulators acc[m][n] = sum_k qx[m][k] qw[n][k]."""
+    M, K2 = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * K2
+    if acc is None:
+        acc = torch.empty(M, N, dtype=torch.int32, device=Xq.device)
+    if workspace is None:
+        workspace = Workspace(Xq.device)
+    ws = workspace.get(tq_gemm_workspace_bytes(M, N, K, 0)) if isinstance(workspace, Workspace) \
+        else workspace
+    _check(_lib.tq_debug_w4a4_gemm_acc(_ptr(Xq), _ptr(Wq), M, N, K, _ptr(acc), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "tq_debug_w4a4_gemm_acc")
+    return acc
+
+
+def tq_query_device_status(workspace, stream=None) -> int:
+    ws = workspace.buf if isinstance(workspace, Workspace) else workspace
+    return int(_lib.tq_query_device_status(_ptr(ws), _stream(stream)))
+
+
+def layer_forward(X, L1t, L2t, Wq, s_w, had_block, workspace=None, stream=None, out=None):
+    """One layer: tq_quantize_act then tq_w4a4_lr_gemm (two kernel launches)."""
+    Xq, s_x, XL1 = tq_quantize_act(X, had_block, L1t, stream=stream)
+    return tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w, XL1, L2t, Y=out, workspace=workspace,
+                           stream=stream)

@@ -120,6 +120,8 @@ def make_weights(shape: LayerShape, seed: int = 0, device: str = "cpu") -> dict:
     """
     K, N, r = shape.K, shape.N, shape.r
     p = min(K, N)
+    if r > p:
+        raise ValueError(f"rank {r} exceeds min(K, N) = {p}")
     U = _orthonormal(K, p, seed + 1, device)
     V = _orthonormal(N, p, seed + 2, device)
     sig = _spectrum(shape, p, device)
