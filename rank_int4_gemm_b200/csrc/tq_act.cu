@@ -134,6 +134,7 @@ struct ActParams {
   int passes_per_cta;  // P
   int total_passes;    // K / W
   int kc;              // L1 k-chunk (columns) staged per step
+  int l1_bufs;         // staged chunk buffers (all chunks, or 2)
   float scale_mul;     // 1 / (7 sqrt(b))
 };
 
@@ -144,18 +145,21 @@ struct ActSmem {
   int xs_stride;   // bf16 elements per X row (slice + 8 pad)
   int l1_stride;   // bf16 elements per staged L1^T row (kc + 8 pad)
   size_t off_l1, off_part, off_amax, total;
-  __host__ __device__ ActSmem(int P, int r, int kc) {
+  __host__ __device__ ActSmem(int P, int r, int kc, int nbuf) {
     xs_stride = P * W + 8;
     l1_stride = kc + 8;
     size_t xs_bytes = (size_t)kActRows * xs_stride * 2;
     off_l1 = (xs_bytes + 127) & ~size_t(127);
-    size_t l1_bytes = (size_t)2 * r * l1_stride * 2;
+    size_t l1_bytes = (size_t)nbuf * r * l1_stride * 2;
     off_part = (off_l1 + l1_bytes + 127) & ~size_t(127);
     size_t part_bytes = (size_t)kActRows * r * 4;
     off_amax = (off_part + part_bytes + 127) & ~size_t(127);
     total = off_amax + 2 * kActRows * 4;
   }
 };
+// Staged L1^T chunks: all of the slice at once when it fits in this budget
+// (one round trip to memory), else a double buffer.
+constexpr size_t kL1AllBudget = 81920;
 
 template <int E>
 __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActParams p) {
@@ -167,7 +171,7 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
   pdl_wait();
 
   const int P = p.passes_per_cta;
-  const ActSmem<E> L(P, p.r, p.kc);
+  const ActSmem<E> L(P, p.r, p.kc, p.l1_bufs);
   __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
   __nv_bfloat16* l1s = reinterpret_cast<__nv_bfloat16*>(smem + L.off_l1);
   float* part = reinterpret_cast<float*>(smem + L.off_part);
@@ -197,8 +201,10 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
     }
     cp_async_commit();
   }
-  // ---- first L1^T chunk
+  // ---- L1^T chunks of this slice: all of them up front when they fit,
+  //      otherwise the first of a double buffer
   const int nchunks = (p.r > 0) ? slice / p.kc : 0;
+  const bool all_l1 = nchunks > 0 && p.l1_bufs >= nchunks;
   auto stage_l1 = [&](int ci, int buf) {
     const int cpr = p.kc / 8;
     __nv_bfloat16* dst = l1s + (size_t)buf * p.r * L.l1_stride;
@@ -209,10 +215,20 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
     }
     cp_async_commit();
   };
-  if (nchunks > 0) stage_l1(0, 0);
-
-  cp_async_wait<1>();  // X landed (the L1 chunk may still be in flight)
+  if (all_l1) {
+    for (int ci = 0; ci < nchunks; ++ci) stage_l1(ci, ci);
+  } else if (nchunks > 0) {
+    stage_l1(0, 0);
+  }
+  // X is the oldest group; wait for it only (L1 chunks may still be in flight)
   if (nchunks == 0) cp_async_wait<0>();
+  else if (all_l1) {
+    // groups: X, chunk 0..nchunks-1 -> at most nchunks pending means X done;
+    // wait_group takes an immediate, so wait for everything when chunks are few
+    cp_async_wait<0>();
+  } else {
+    cp_async_wait<1>();
+  }
   __syncthreads();
 
   // ---- rotation of this warp's token: PMAX passes of W columns
@@ -263,14 +279,17 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
       acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
     const uint32_t xs_base = smem_u32(xs);
     for (int ci = 0; ci < nchunks; ++ci) {
-      if (ci + 1 < nchunks) {
-        stage_l1(ci + 1, (ci + 1) & 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
+      if (!all_l1) {
+        if (ci + 1 < nchunks) {
+          stage_l1(ci + 1, (ci + 1) & 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+        __syncthreads();
       }
-      __syncthreads();
-      const uint32_t l1_base = smem_u32(l1s + (size_t)(ci & 1) * p.r * L.l1_stride);
+      const int buf = all_l1 ? ci : (ci & 1);
+      const uint32_t l1_base = smem_u32(l1s + (size_t)buf * p.r * L.l1_stride);
       for (int kk = 0; kk < p.kc; kk += 16) {
         uint32_t a[4];
         {
@@ -292,7 +311,7 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
           }
         }
       }
-      __syncthreads();  // buffer (ci & 1) is refilled two chunks later
+      if (!all_l1) __syncthreads();  // buffer (ci & 1) is refilled two chunks later
     }
     // C fragment: rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
 #pragma unroll
@@ -400,19 +419,23 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const float* 
 }
 
 template <int E>
-cudaError_t launch_act_e(const ActParams& prm_in, cudaStream_t stream) {
+cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t stream) {
   constexpr int W = 32 * E;
   constexpr int PMAX = 64 / E;
   ActParams prm = prm_in;
   const int tp = prm.K / W;
-  int P = (tp + 7) / 8;          // portable clusters (<= 8 CTAs) when possible
+  int P = (tp + max_cluster - 1) / max_cluster;
   if (P > PMAX) P = (tp + 15) / 16;
   if (P > PMAX) return cudaErrorInvalidValue;
   const int C = (tp + P - 1) / P;
   prm.passes_per_cta = P;
   prm.total_passes = tp;
   prm.kc = prm.r > 256 ? 32 : (prm.r > 128 ? 64 : 128);
-  const ActSmem<E> L(P, prm.r, prm.kc);
+  if (prm.kc > P * W) prm.kc = P * W;
+  const int nchunks_max = (P * W) / prm.kc;
+  const size_t all_bytes = (size_t)nchunks_max * prm.r * (prm.kc + 8) * 2;
+  prm.l1_bufs = (all_bytes <= kL1AllBudget) ? nchunks_max : 2;
+  const ActSmem<E> L(P, prm.r, prm.kc, prm.l1_bufs);
   auto kern = quantize_act_kernel<E>;
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
@@ -420,12 +443,13 @@ cudaError_t launch_act_e(const ActParams& prm_in, cudaStream_t stream) {
   if (!(attr_set >> dev & 1u)) {
     // the largest carve-up any supported shape needs (P * W <= 2048, r <= 512)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ActSmem<E>(PMAX, 512, 32).total);
+                                         (int)ActSmem<E>(PMAX, 512, 32, 2).total);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
+  if (L.total > ActSmem<E>(PMAX, 512, 32, 2).total) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, (prm.M + kActRows - 1) / kActRows, 1);
   cfg.blockDim = dim3(kActThreads, 1, 1);
@@ -457,9 +481,12 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   prm.b = had_block;
   prm.r = r;
   prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  if (K % 512 == 0 && had_block <= 512) return launch_act_e<16>(prm, stream);
-  if (K % 256 == 0 && had_block <= 256) return launch_act_e<8>(prm, stream);
-  if (had_block <= 128) return launch_act_e<4>(prm, stream);
+  // Few token groups (decode): spread K over up to 16 CTAs of 256 columns.
+  const int groups = (M + kActRows - 1) / kActRows;
+  if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);
+  if (K % 512 == 0) return launch_act_e<16>(prm, 8, stream);
+  if (K % 256 == 0) return launch_act_e<8>(prm, 8, stream);
+  if (had_block <= 128) return launch_act_e<4>(prm, 8, stream);
   return cudaErrorInvalidValue;
 }
 
