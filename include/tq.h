@@ -143,6 +143,35 @@ TQ_API int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq,
                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * tq_w4a4_lr_gemm_noalloc -- tq_w4a4_lr_gemm for callers that cannot
+ * allocate device memory (a framework that owns the device allocator, a
+ * real-time path where an allocation could synchronise the device, a plugin
+ * that only ever receives pointers to its inputs and outputs).  Same inputs,
+ * output and result as tq_w4a4_lr_gemm, but no workspace argument: the
+ * kernel's scratch (its status word) lives in a fixed 256-byte array in the
+ * library's own device memory, which every GPU that loads the library keeps
+ * until the process exits.  Nothing is allocated on any call.
+ *
+ *  - Shapes needing more scratch than tq_gemm_workspace_bytes() = 256 bytes
+ *    are rejected with TQ_ERR_WORKSPACE before anything runs.
+ *  - The first call on a device looks up that array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - Every call clears the array on `stream` before its kernel and every call
+ *    shares it, so calls that overlap on the GPU (different streams with no
+ *    ordering between them) race on it.
+ *  - A watchdog timeout in this variant is recorded only in that shared
+ *    array and is not reported by tq_query_device_status.
+ * The pages have no counterpart of this entry point; it is an addition of
+ * this library.
+ */
+TQ_API int tq_w4a4_lr_gemm_noalloc(const uint8_t* Xq, const float* s_x,
+                                   const uint8_t* Wq, const float* s_w,
+                                   const float* XL1, const uint16_t* L2t,
+                                   int M, int N, int K, int r, uint16_t* Y,
+                                   void* stream);
+
+/*
  * tq_query_device_status -- synchronises `stream`, then reads the status word
  * kernels record in `workspace` (a GEMM workspace) and clears it.  Returns
  * TQ_OK, TQ_ERR_TIMEOUT if a bounded in-kernel wait gave up since the last

@@ -38,6 +38,8 @@ _lib.tq_w4a4_lr_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                   ctypes.c_size_t, _P]
 _lib.tq_debug_w4a4_gemm_acc.restype = _I
 _lib.tq_debug_w4a4_gemm_acc.argtypes = [_P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
+_lib.tq_w4a4_lr_gemm_noalloc.restype = _I
+_lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.tq_query_device_status.restype = _I
 _lib.tq_query_device_status.argtypes = [_P, _P]
 
@@ -154,6 +156,24 @@ def tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, workspace=None
                                 _ptr(XL1) if r else None, _ptr(L2t) if r else None,
                                 M, N, K, r, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
            "tq_w4a4_lr_gemm")
+    return Y
+
+
+def tq_w4a4_lr_gemm_noalloc(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, stream=None):
+    """tq_w4a4_lr_gemm without a workspace argument, for callers that cannot
+    allocate device memory: the kernel's scratch is a fixed array inside the
+    library (shared by all calls; overlapping calls race).  Y must be passed
+    by such callers; it is allocated here only as a convenience."""
+    M, K2 = Xq.shape
+    N = Wq.shape[0]
+    K = 2 * K2
+    r = 0 if XL1 is None else XL1.shape[1]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq.device)
+    _check(_lib.tq_w4a4_lr_gemm_noalloc(_ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(s_w),
+                                        _ptr(XL1) if r else None, _ptr(L2t) if r else None,
+                                        M, N, K, r, _ptr(Y), _stream(stream)),
+           "tq_w4a4_lr_gemm_noalloc")
     return Y
 
 
