@@ -51,6 +51,12 @@ def parse():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-sweep", action="store_true", help="skip the M=1/128 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill_gateup", "prefill_down", "large_gateup",
+                             "large_down", "sweep"],
+                    help="decode is the default workload; the others are the prefill "
+                         "shapes, scored in TOPS against the dense INT8 peak")
+    ap.add_argument("--rank", type=int, default=None, help="low-rank r override (sweep)")
     return ap.parse_args()
 
 
@@ -71,6 +77,18 @@ def measured_peaks():
         return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs)"
     except Exception:
         return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def int8_peak(sustained: bool):
+    """Dense INT8 tensor peak: the measured bf16 cuBLAS peak times the nominal
+    INT8/bf16 ratio of B200 (4.5 / 2.25 = 2)."""
+    key = "bf16_tflops_sustained" if sustained else "bf16_tflops"
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return 2.0 * float(d[key]), f"measured bf16 ({key}) x 2 nominal INT8/bf16 ratio"
+    except Exception:
+        return 2.0 * (1400.0 if sustained else 1590.0), "fallback bf16 x 2"
 
 
 def profiled_traffic(kernel_src: str, profile: str):
@@ -335,6 +353,95 @@ def run_tq(args, rank, world, local_rank, dist):
     return out
 
 
+# --------------------------------------------------------------- prefill arm
+
+def run_prefill(args, rank, world, local_rank, dist):
+    """One prefill layer per step (act + GEMM), over enough distinct layers
+    that the step's operands exceed L2; TOPS = 2 M N K per layer / time."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    sh = synth.CONFIGS[args.workload]
+    if args.rank is not None:
+        sh = sh.with_(r=args.rank)
+    M = args.m if args.m != 16 else sh.M
+    K, N, r, b = sh.K, sh.N, sh.r, sh.had_block
+    per_layer = 2 * M * K + K * N // 2 + 2 * M * N
+    L = max(1, min(args.layers, -(-200_000_000 // per_layer)))
+    layers = []
+    for i in range(L):
+        w = synth.make_weights(sh, seed=1000 * rank + 10 * i, device="cuda")
+        Rt = w["Rt"].to(dev)
+        Wq, s_w = tq.tq_pack_weight(Rt, b)
+        del Rt
+        layers.append({
+            "X": synth.make_activations(sh, seed=1000 * rank + 10 * i, M=M).to(dev),
+            "L1t": w["L1t"].to(dev) if r else None, "L2t": w["L2t"].to(dev) if r else None,
+            "Wq": Wq, "s_w": s_w,
+            "Xq": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            "s_x": torch.empty(M, dtype=torch.float32, device=dev),
+            "XL1": torch.empty(M, r, dtype=torch.float32, device=dev) if r else None,
+            "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+            "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev),
+        })
+    torch.cuda.synchronize()
+
+    def one(lay, ev=None):
+        tq.tq_quantize_act(lay["X"], b, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
+        if ev is not None:
+            ev[0].record()
+        tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"], lay["L2t"],
+                           Y=lay["Y"], workspace=lay["ws"])
+        if ev is not None:
+            ev[1].record()
+
+    g = capture(torch, lambda: [one(l) for l in layers])
+    with ClockSampler(local_rank) as clk:
+        ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    evs = [(torch.cuda.Event(enable_timing=True, external=True),
+            torch.cuda.Event(enable_timing=True, external=True)) for _ in layers]
+    g_ev = capture(torch, lambda: [one(l, e) for l, e in zip(layers, evs)])
+    gemm_ms = []
+    for _ in range(3):
+        g_ev.replay()
+    for _ in range(max(1, min(args.steps, 20))):
+        g_ev.replay()
+        torch.cuda.synchronize()
+        gemm_ms.extend(a.elapsed_time(bb) for a, bb in evs)
+    gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
+    ops = 2 * M * N * K
+    peak, src = int8_peak(sustained=False)
+    achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(world * L * ops / ms / 1e9, 2), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int4", "data": "synthetic",
+        "config": {"workload": f"{args.workload}: M={M}, K={K}, N={N}, rank {r}, Hadamard "
+                               f"block {b}; {L} distinct layer(s) per step",
+                   "M": M, "K": K, "N": N, "r": r, "had_block": b, "layers_per_step": L,
+                   "l2": "inputs larger than L2" if L * per_layer > 126e6 else "L2-resident"},
+        "GB/s": round(world * L * per_layer / ms / 1e6, 1),
+        "us_per_layer": round(ms * 1e3 / L, 3),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
+                     "unit": "TOPS", "frac": round(achieved / peak, 4), "traffic": None,
+                     "kernel": "w4a4_lr_gemm_kernel (prefill tiling)",
+                     "gemm_us": round(gemm_ms_avg * 1e3, 2), "peak_source": src,
+                     "lowrank_flops_per_launch": 2 * M * r * (K + N)},
+        "gpu_launches": 2 * L * args.steps,
+        "clocks": clk.summary(),
+    }
+    return out
+
+
 # ------------------------------------------------------------ oracle (CPU)
 
 def cpu_baseline(M, budget_s=12.0):
@@ -427,7 +534,10 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
-    out = run_tq(args, rank, world, local_rank, dist)
+    if args.workload == "decode":
+        out = run_tq(args, rank, world, local_rank, dist)
+    else:
+        out = run_prefill(args, rank, world, local_rank, dist)
     if rank == 0:
         print(json.dumps(out))
     if dist is not None:

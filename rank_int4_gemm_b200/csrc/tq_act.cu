@@ -18,6 +18,8 @@
 // folded into the stored scale.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "tq_internal.h"
 #include "tq_ptx.cuh"
 
@@ -124,6 +126,10 @@ __device__ __forceinline__ void mma_16816(float (&d)[4], const uint32_t (&a)[4],
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+__device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
 struct ActParams {
   const __nv_bfloat16* X;
   const __nv_bfloat16* L1t;
@@ -135,31 +141,43 @@ struct ActParams {
   int total_passes;    // K / W
   int kc;              // L1 k-chunk (columns) staged per step
   int l1_bufs;         // staged chunk buffers (all chunks, or 2)
+  int kparts;          // warps sharing one 8-column tile of r split its k steps
   float scale_mul;     // 1 / (7 sqrt(b))
 };
 
 // Shared-memory carve-up of quantize_act_kernel.
+//   xs     X tile [16][slice + 8] bf16
+//   l1s    staged L1^T chunks [nbuf][r][kc + 8] bf16
+//   partk  X L1 partials per k-part [KP][16][r] fp32
+//   recv   X L1 partials received from the cluster [C][16][ceil(r/C)] fp32
+//   amax   per-CTA absmax received from the cluster [C][16], row absmax [16]
 template <int E>
 struct ActSmem {
   static constexpr int W = 32 * E;
   int xs_stride;   // bf16 elements per X row (slice + 8 pad)
   int l1_stride;   // bf16 elements per staged L1^T row (kc + 8 pad)
-  size_t off_l1, off_part, off_amax, total;
-  __host__ __device__ ActSmem(int P, int r, int kc, int nbuf) {
+  int cols_max;    // X L1 columns owned per CTA in the cluster reduction
+  size_t off_l1, off_part, off_recv, off_amax, total;
+  __host__ __device__ ActSmem(int P, int r, int kc, int nbuf, int kp, int C) {
     xs_stride = P * W + 8;
     l1_stride = kc + 8;
+    cols_max = (r + C - 1) / C;
     size_t xs_bytes = (size_t)kActRows * xs_stride * 2;
     off_l1 = (xs_bytes + 127) & ~size_t(127);
     size_t l1_bytes = (size_t)nbuf * r * l1_stride * 2;
     off_part = (off_l1 + l1_bytes + 127) & ~size_t(127);
-    size_t part_bytes = (size_t)kActRows * r * 4;
-    off_amax = (off_part + part_bytes + 127) & ~size_t(127);
-    total = off_amax + 2 * kActRows * 4;
+    size_t part_bytes = (size_t)kp * kActRows * r * 4;
+    off_recv = (off_part + part_bytes + 127) & ~size_t(127);
+    size_t recv_bytes = (size_t)C * kActRows * cols_max * 4;
+    off_amax = (off_recv + recv_bytes + 127) & ~size_t(127);
+    total = off_amax + (size_t)(C + 1) * kActRows * 4;
   }
 };
 // Staged L1^T chunks: all of the slice at once when it fits in this budget
 // (one round trip to memory), else a double buffer.
 constexpr size_t kL1AllBudget = 81920;
+// Dynamic shared memory the kernel is allowed (every supported shape fits).
+constexpr size_t kActSmemMax = 200 * 1024;
 
 template <int E>
 __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActParams p) {
@@ -168,18 +186,20 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
   extern __shared__ __align__(128) uint8_t smem[];
 
   pdl_launch_dependents();  // let the GEMM start streaming its weights
+  // announce this CTA to the cluster; remote stores wait for every peer
+  cluster_arrive_relaxed();
   pdl_wait();
 
   const int P = p.passes_per_cta;
-  const ActSmem<E> L(P, p.r, p.kc, p.l1_bufs);
-  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* l1s = reinterpret_cast<__nv_bfloat16*>(smem + L.off_l1);
-  float* part = reinterpret_cast<float*>(smem + L.off_part);
-  float* amax_part = reinterpret_cast<float*>(smem + L.off_amax);
-  float* amax_row = amax_part + kActRows;
-
   const uint32_t crank = cluster_ctarank();
   const uint32_t csize = cluster_nctarank();
+  const ActSmem<E> L(P, p.r, p.kc, p.l1_bufs, p.kparts, (int)csize);
+  __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* l1s = reinterpret_cast<__nv_bfloat16*>(smem + L.off_l1);
+  float* partk = reinterpret_cast<float*>(smem + L.off_part);
+  float* recv = reinterpret_cast<float*>(smem + L.off_recv);
+  float* amax_all = reinterpret_cast<float*>(smem + L.off_amax);  // [C][16]
+  float* amax_row = amax_all + csize * kActRows;
   const int pass0 = (int)crank * P;
   const int np = min(P, p.total_passes - pass0);
   const int slice = np * W;
@@ -267,17 +287,26 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
     }
   }
   amax = warp_max(amax);
-  if (lane == 0) amax_part[warp] = amax;
+  cluster_wait_acquire();  // every peer is running before it is written to
+  // every CTA of the cluster gets this CTA's partial absmax of token `warp`
+  if (lane < (int)csize)
+    dsmem_st_f32(dsmem_map(smem_u32(&amax_all[crank * kActRows + warp]), (uint32_t)lane), amax);
 
-  // ---- X L1 partial over this CTA's slice: warps own 8-column tiles of r
+  // ---- X L1 partial over this CTA's slice: warp w owns 8-column tile
+  //      (w % NT) of r and k-part (w / NT) of every staged chunk
   if (nchunks > 0) {
     const int ntiles = p.r / 8;
+    const int KP = p.kparts;
+    const int kp = warp / min(ntiles, 16);
+    const bool active = warp < min(ntiles, 16) * KP;
     constexpr int kMaxTilesPerWarp = 4;  // r <= 512
     float acc[kMaxTilesPerWarp][4];
 #pragma unroll
     for (int t = 0; t < kMaxTilesPerWarp; ++t)
       acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
     const uint32_t xs_base = smem_u32(xs);
+    const int ksteps = p.kc / 16;
+    const int ks0 = kp * ksteps / KP, ks1 = (kp + 1) * ksteps / KP;
     for (int ci = 0; ci < nchunks; ++ci) {
       if (!all_l1) {
         if (ci + 1 < nchunks) {
@@ -290,49 +319,65 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
       }
       const int buf = all_l1 ? ci : (ci & 1);
       const uint32_t l1_base = smem_u32(l1s + (size_t)buf * p.r * L.l1_stride);
-      for (int kk = 0; kk < p.kc; kk += 16) {
-        uint32_t a[4];
-        {
-          const int mat = lane >> 3, rin = lane & 7;
-          const int rr = rin + (mat & 1) * 8;
-          const int cc = ci * p.kc + kk + (mat >> 1) * 8;
-          ldmatrix_x4(a, xs_base + (uint32_t)((rr * L.xs_stride + cc) * 2));
-        }
+      if (active) {
+        for (int ks = ks0; ks < ks1; ++ks) {
+          const int kk = ks * 16;
+          uint32_t a[4];
+          {
+            const int mat = lane >> 3, rin = lane & 7;
+            const int rr = rin + (mat & 1) * 8;
+            const int cc = ci * p.kc + kk + (mat >> 1) * 8;
+            ldmatrix_x4(a, xs_base + (uint32_t)((rr * L.xs_stride + cc) * 2));
+          }
 #pragma unroll
-        for (int t = 0; t < kMaxTilesPerWarp; ++t) {
-          const int tile = warp + 16 * t;
-          if (tile < ntiles) {
-            uint32_t bb[2];
-            const int l = lane & 15;
-            const int jr = tile * 8 + (l & 7);
-            const int cc = kk + (l >> 3) * 8;
-            ldmatrix_x2(bb, l1_base + (uint32_t)((jr * L.l1_stride + cc) * 2));
-            mma_16816(acc[t], a, bb);
+          for (int t = 0; t < kMaxTilesPerWarp; ++t) {
+            const int tile = (warp % min(ntiles, 16)) + 16 * t;
+            if (tile < ntiles) {
+              uint32_t bb[2];
+              const int l = lane & 15;
+              const int jr = tile * 8 + (l & 7);
+              const int cc = kk + (l >> 3) * 8;
+              ldmatrix_x2(bb, l1_base + (uint32_t)((jr * L.l1_stride + cc) * 2));
+              mma_16816(acc[t], a, bb);
+            }
           }
         }
       }
       if (!all_l1) __syncthreads();  // buffer (ci & 1) is refilled two chunks later
     }
     // C fragment: rows lane/4 and lane/4 + 8, columns 2*(lane%4) + {0, 1}
+    if (active) {
+      float* pk = partk + (size_t)kp * kActRows * p.r;
 #pragma unroll
-    for (int t = 0; t < kMaxTilesPerWarp; ++t) {
-      const int tile = warp + 16 * t;
-      if (tile < ntiles) {
-        const int rr = lane >> 2, cc = tile * 8 + 2 * (lane & 3);
-        part[rr * p.r + cc] = acc[t][0];
-        part[rr * p.r + cc + 1] = acc[t][1];
-        part[(rr + 8) * p.r + cc] = acc[t][2];
-        part[(rr + 8) * p.r + cc + 1] = acc[t][3];
+      for (int t = 0; t < kMaxTilesPerWarp; ++t) {
+        const int tile = (warp % min(ntiles, 16)) + 16 * t;
+        if (tile < ntiles) {
+          const int rr = lane >> 2, cc = tile * 8 + 2 * (lane & 3);
+          pk[rr * p.r + cc] = acc[t][0];
+          pk[rr * p.r + cc + 1] = acc[t][1];
+          pk[(rr + 8) * p.r + cc] = acc[t][2];
+          pk[(rr + 8) * p.r + cc + 1] = acc[t][3];
+        }
       }
+    }
+    __syncthreads();
+    // this CTA's partial (k-parts summed in order) -> the column's owner CTA
+    for (int idx = tid; idx < kActRows * p.r; idx += kActThreads) {
+      const int rr = idx / p.r, col = idx - rr * p.r;
+      float v = 0.f;
+      for (int k = 0; k < KP; ++k) v += partk[(size_t)k * kActRows * p.r + idx];
+      const int owner = col * (int)csize / p.r;
+      const int lo = (owner * p.r + (int)csize - 1) / (int)csize;
+      const uint32_t dst = smem_u32(&recv[((int)crank * kActRows + rr) * L.cols_max + (col - lo)]);
+      dsmem_st_f32(dsmem_map(dst, (uint32_t)owner), v);
     }
   }
 
-  cluster_sync();  // partial absmax and X L1 of every CTA are visible
+  cluster_sync();  // every partial absmax and X L1 has been delivered
 
   if (tid < kActRows) {
-    const uint32_t a_addr = smem_u32(&amax_part[tid]);
     float m = 0.f;
-    for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, dsmem_ld_f32(dsmem_map(a_addr, c)));
+    for (uint32_t c = 0; c < csize; ++c) m = fmaxf(m, amax_all[c * kActRows + tid]);
     amax_row[tid] = m;
   }
   __syncthreads();
@@ -354,20 +399,19 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
     if (crank == 0 && lane == 0) p.s_x[my_row] = am * p.scale_mul;
   }
 
-  // ---- leader: X L1 = sum over the cluster's CTAs, in rank order
-  if (crank == 0 && p.r > 0) {
-    const uint32_t part_addr = smem_u32(part);
-    for (int idx = tid; idx < kActRows * p.r; idx += kActThreads) {
-      const int rr = idx / p.r;
+  // ---- X L1 of the columns this CTA owns: sum over the cluster in rank order
+  if (p.r > 0) {
+    const int lo = ((int)crank * p.r + (int)csize - 1) / (int)csize;
+    const int hi = (((int)crank + 1) * p.r + (int)csize - 1) / (int)csize;
+    const int ncol = hi - lo;
+    for (int idx = tid; idx < kActRows * ncol; idx += kActThreads) {
+      const int rr = idx / ncol, cc = idx - rr * ncol;
       if (row0 + rr >= p.M) continue;
-      float s = 0.f;
-      for (uint32_t c = 0; c < csize; ++c)
-        s += dsmem_ld_f32(dsmem_map(part_addr + (uint32_t)idx * 4u, c));
-      p.XL1[(size_t)(row0 + rr) * p.r + (idx % p.r)] = s;
+      float v = 0.f;
+      for (uint32_t c = 0; c < csize; ++c) v += recv[((int)c * kActRows + rr) * L.cols_max + cc];
+      p.XL1[(size_t)(row0 + rr) * p.r + lo + cc] = v;
     }
   }
-
-  cluster_sync();  // keep shared memory alive until every peer has read it
 }
 
 // ------------------------------------------------------------ weight pack
@@ -435,7 +479,9 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   const int nchunks_max = (P * W) / prm.kc;
   const size_t all_bytes = (size_t)nchunks_max * prm.r * (prm.kc + 8) * 2;
   prm.l1_bufs = (all_bytes <= kL1AllBudget) ? nchunks_max : 2;
-  const ActSmem<E> L(P, prm.r, prm.kc, prm.l1_bufs);
+  const int ntiles = prm.r / 8;
+  prm.kparts = (ntiles == 0) ? 1 : std::max(1, std::min(16 / std::min(ntiles, 16), prm.kc / 16));
+  const ActSmem<E> L(P, prm.r, prm.kc, prm.l1_bufs, prm.kparts, C);
   auto kern = quantize_act_kernel<E>;
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
@@ -443,13 +489,13 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   if (!(attr_set >> dev & 1u)) {
     // the largest carve-up any supported shape needs (P * W <= 2048, r <= 512)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)ActSmem<E>(PMAX, 512, 32, 2).total);
+                                         (int)kActSmemMax);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
-  if (L.total > ActSmem<E>(PMAX, 512, 32, 2).total) return cudaErrorInvalidValue;
+  if (L.total > kActSmemMax) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, (prm.M + kActRows - 1) / kActRows, 1);
   cfg.blockDim = dim3(kActThreads, 1, 1);

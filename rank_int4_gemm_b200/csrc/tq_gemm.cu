@@ -48,8 +48,7 @@ constexpr int kBM = 128;         // MMA M
 constexpr int kKB = 128;         // codes per k-block (one 128-byte int8 row)
 constexpr int kPackedRow = 64;   // packed bytes per row per k-block
 constexpr int kLrChunk = 64;     // bf16 columns per low-rank chunk (128 bytes)
-constexpr int kConvThreads = 128;
-constexpr int kThreads = 192;    // 4 converter/epilogue warps + producer + MMA
+constexpr int kEpiThreads = 128;  // warps 0-3: TMEM lanes 0-127, the epilogue
 
 struct GemmParams {
   const float* s_p;
@@ -66,6 +65,7 @@ struct GemmParams {
 };
 
 constexpr int kKBS = 2;          // k-blocks per TMA stage: 128-byte rows, 128B swizzle
+constexpr int kMaxSplits = 8;    // split-K cluster size limit (portable clusters)
 
 template <int BN, int NSTG, int NOPS, bool RECV>
 struct SmemLayout {
@@ -107,6 +107,16 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
                "r"(v.z), "r"(v.w)
                : "memory");
+}
+__device__ __forceinline__ int ld_shared_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
 }
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -162,12 +172,17 @@ __device__ __forceinline__ void tmem_acc16(uint32_t taddr, int (&out)[16]) {
 // One 128 x BN output tile over k-blocks [split*kb_per_split, ...).  SWAP
 // kernels are launched as clusters of `splits` CTAs along z; the CTAs of a
 // cluster combine their INT32 partials through distributed shared memory.
-template <int BN, bool SWAP, int NSTG, int NOPS, int NACC, bool RECV>
-__global__ void __launch_bounds__(kThreads, 1)
+// Warps 0..CW-1 convert (warps 0-3 also run the epilogue), warp CW is the TMA
+// producer, warp CW+1 allocates TMEM and issues the MMAs.
+template <int BN, bool SWAP, int NSTG, int NOPS, int NACC, bool RECV, int CW>
+__global__ void __launch_bounds__(32 * (CW + 2), 1)
     w4a4_lr_gemm_kernel(const __grid_constant__ CUtensorMap map_p,
                         const __grid_constant__ CUtensorMap map_q, const GemmParams prm) {
   using L = SmemLayout<BN, NSTG, NOPS, RECV>;
   constexpr int kRows = kBM + BN;
+  constexpr int kConvThreads = 32 * CW;
+  constexpr int kProducerWarp = CW, kMmaWarp = CW + 1;
+  static_assert(CW >= 4, "warps 0-3 own the TMEM lanes of the epilogue");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -200,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Warp 4, lane 0 initialises the barriers and immediately starts streaming
   // the first NSTG stages of weights, which do not depend on the preceding
   // kernel (programmatic dependent launch), while warp 5 allocates TMEM.
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     for (int i = 0; i < NSTG; ++i) {
       mbar_init(&stg_full[i], 1);
       mbar_init(&stg_empty[i], kConvThreads);
@@ -225,17 +240,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(sp + L::kStgP, &map_q, &stg_full[i], x, tile_q * BN, pol_w);
     }
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // split-K clusters with a dedicated receive area: announce this CTA now;
+  // the epilogue waits for every peer before its first remote store
+  if constexpr (SWAP && RECV) cluster_arrive_relaxed();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const uint32_t tmem_lr = tmem_base + NACC * BN;  // fp32, BN columns
+  constexpr int kScPer = (kRows + kEpiThreads - 1) / kEpiThreads;
+  float sc_reg[kScPer];
+#pragma unroll
+  for (int u = 0; u < kScPer; ++u) sc_reg[u] = 0.f;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------ TMA producer
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
@@ -264,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     const uint32_t id_i8 = idesc_i8_s32(BN);
     const uint32_t id_bf = idesc_bf16_f32(BN);
@@ -298,12 +320,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------- converters
-    const int tid = threadIdx.x;  // 0..127
+    const int tid = threadIdx.x;  // 0..kConvThreads-1
     pdl_wait();
-    // scales of this tile's rows and columns, for the epilogue
-    for (int i = tid; i < kRows; i += kConvThreads) {
+    // scales of this tile's rows and columns, for the epilogue: loaded now,
+    // stored to shared memory after the main loop (the load latency hides
+    // under the weight stream)
+#pragma unroll
+    for (int u = 0; u < kScPer; ++u) {
+      const int i = tid + u * kEpiThreads;
       float v = 0.f;
-      if (!prm.acc_out) {
+      if (!prm.acc_out && i < kRows && tid < kEpiThreads) {
         if (i < kBM) {
           const int g = tile_p * kBM + i;
           if (g < prm.rows_p) v = __ldg(prm.s_p + g);
@@ -312,9 +338,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (g < prm.rows_q) v = __ldg(prm.s_q + g);
         }
       }
-      sc[i] = v;
+      sc_reg[u] = v;
     }
-    named_bar_sync(2, kConvThreads);  // scales visible to every epilogue thread
     bool alive = true;
     // low-rank chunks first; each thread issues all its global loads before
     // any of its shared-memory stores
@@ -369,11 +394,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // int4 -> int8: a thread expands one 128-code row segment (64 packed
     // bytes, 4 swizzled chunks of the staged row) into the 8 chunks of the
-    // operand row, 16 * code per byte
+    // operand row, 16 * code per byte.  One k-block (one operand slot) at a
+    // time, so the expansion of k-block i+1 overlaps the MMAs of k-block i.
     for (int st = 0; st < n_st && alive; ++st) {
       const int sg_slot = st % NSTG;
       if (!mbar_wait(&stg_full[sg_slot], (uint32_t)(st / NSTG) & 1u, prm.status, abort_flag)) break;
       const int nsub = min(kKBS, n_kb - st * kKBS);
+      const uint32_t sg = base + L::kStgBase + sg_slot * L::kStgStage;
       for (int sub = 0; sub < nsub; ++sub) {
         const int i = n_lr + st * kKBS + sub;
         if (!mbar_wait(&op_empty[i % NOPS], ((uint32_t)(i / NOPS) & 1u) ^ 1u, prm.status,
@@ -381,36 +408,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           alive = false;
           break;
         }
+        const uint32_t dst0 = base + L::kOpBase + (uint32_t)(i % NOPS) * L::kOpStage;
+        for (int row = tid; row < kRows; row += kConvThreads) {
+          const uint32_t x7 = (uint32_t)row & 7u;
+          const uint32_t src = sg + (uint32_t)row * 128u;
+          uint4 w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            w[q] = ld_shared_v4(src + (((uint32_t)(sub * 4 + q) ^ x7) << 4));
+          const uint32_t dst = dst0 + (uint32_t)row * 128u;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 lo, hi;
+            lo.x = (w[q].x << 4) & 0xF0F0F0F0u;
+            lo.y = (w[q].y << 4) & 0xF0F0F0F0u;
+            lo.z = (w[q].z << 4) & 0xF0F0F0F0u;
+            lo.w = (w[q].w << 4) & 0xF0F0F0F0u;
+            hi.x = w[q].x & 0xF0F0F0F0u;
+            hi.y = w[q].y & 0xF0F0F0F0u;
+            hi.z = w[q].z & 0xF0F0F0F0u;
+            hi.w = w[q].w & 0xF0F0F0F0u;
+            st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
+            st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&op_full[i % NOPS]);
       }
       if (!alive) break;
-      const uint32_t sg = base + L::kStgBase + sg_slot * L::kStgStage;
-      for (int task = tid; task < kRows * nsub; task += kConvThreads) {
-        const int sub = task / kRows, row = task - sub * kRows;
-        const uint32_t x7 = (uint32_t)row & 7u;
-        const uint32_t src = sg + (uint32_t)row * 128u;
-        uint4 w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(sub * 4 + q) ^ x7) << 4));
-        const int i = n_lr + st * kKBS + sub;
-        const uint32_t dst = base + L::kOpBase + (uint32_t)(i % NOPS) * L::kOpStage +
-                             (uint32_t)row * 128u;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 lo, hi;
-          lo.x = (w[q].x << 4) & 0xF0F0F0F0u;
-          lo.y = (w[q].y << 4) & 0xF0F0F0F0u;
-          lo.z = (w[q].z << 4) & 0xF0F0F0F0u;
-          lo.w = (w[q].w << 4) & 0xF0F0F0F0u;
-          hi.x = w[q].x & 0xF0F0F0F0u;
-          hi.y = w[q].y & 0xF0F0F0F0u;
-          hi.z = w[q].z & 0xF0F0F0F0u;
-          hi.w = w[q].w & 0xF0F0F0F0u;
-          st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
-          st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
-        }
-      }
-      fence_proxy_async_smem();
-      for (int sub = 0; sub < nsub; ++sub) mbar_arrive(&op_full[(n_lr + st * kKBS + sub) % NOPS]);
       mbar_arrive(&stg_empty[sg_slot]);
     }
   }
@@ -423,6 +448,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t t_row = (uint32_t)(warp * 32) << 16;
   bool ok = true;
   if (is_epi) {
+#pragma unroll
+    for (int u = 0; u < kScPer; ++u)
+      if (threadIdx.x + u * kEpiThreads < kRows) sc[threadIdx.x + u * kEpiThreads] = sc_reg[u];
+    named_bar_sync(2, kEpiThreads);  // scales visible to every epilogue thread
     ok = __all_sync(0xffffffffu, mbar_wait(acc_full, 0u, prm.status, abort_flag));
     tc_fence_after();
   }
@@ -455,7 +484,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (do_lr) dsmem_st_u32(dst_f + (uint32_t)((cb + j) * rows_max * 4), af[j]);
       }
     };
-    if constexpr (!RECV) cluster_wait();    // ... and so are every peer's
+    cluster_wait();  // every peer is running (RECV) / has freed its rings (!RECV)
     if (is_epi && ok) {
       for (int cb = 0; cb < BN; cb += 16) push16(cb);
     }
@@ -464,21 +493,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int me = split;
       const int lo_m = owned_lo(me, S);
       const int rows_m = owned_lo(me + 1, S) - lo_m;
-      const int32_t* red_i = reinterpret_cast<const int32_t*>(smem + L::kRecvBase);
-      const float* red_f = reinterpret_cast<const float*>(smem + L::kRecvBase) + S * BN * rows_max;
-      for (int idx = threadIdx.x; idx < BN * rows_m; idx += kConvThreads) {
+      const uint32_t red_i = base + L::kRecvBase;                       // int [S][BN][rows_max]
+      const uint32_t red_f = red_i + (uint32_t)(S * BN * rows_max) * 4u;  // fp32 [BN][rows_max]
+      const uint32_t scs = smem_u32(sc);
+      for (int idx = threadIdx.x; idx < BN * rows_m; idx += kEpiThreads) {
         const int col = idx / rows_m, rr = idx - col * rows_m;
         const int g_p = tile_p * kBM + lo_m + rr, g_q = tile_q * BN + col;
+        // all shared-memory loads of this element first, then the sums
+        int part[kMaxSplits];
+#pragma unroll
+        for (int z = 0; z < kMaxSplits; ++z)
+          part[z] = z < S ? ld_shared_s32(red_i + (uint32_t)(((z * BN + col) * rows_max + rr) * 4))
+                          : 0;
+        const float s_p = ld_shared_f32(scs + (uint32_t)(lo_m + rr) * 4u);
+        const float s_q = ld_shared_f32(scs + (uint32_t)(kBM + col) * 4u);
+        const float lr = prm.use_lr ? ld_shared_f32(red_f + (uint32_t)((col * rows_max + rr) * 4)) : 0.f;
         if (g_p >= prm.rows_p || g_q >= prm.rows_q) continue;
         int acc = 0;
-        for (int z = 0; z < S; ++z) acc += red_i[(z * BN + col) * rows_max + rr];
+#pragma unroll
+        for (int z = 0; z < kMaxSplits; ++z) acc += part[z];  // split order
         // out[m][n] with m = token (Q side), n = channel (P side)
         if (prm.acc_out) {
           prm.acc_out[(size_t)g_q * prm.ldy + g_p] = acc;
         } else {
-          float y = sc[lo_m + rr] * sc[kBM + col] * (float)acc;
-          if (prm.use_lr) y += red_f[col * rows_max + rr];
-          prm.Y[(size_t)g_q * prm.ldy + g_p] = __float2bfloat16_rn(y);
+          prm.Y[(size_t)g_q * prm.ldy + g_p] = __float2bfloat16_rn(s_p * s_q * (float)acc + lr);
         }
       }
     }
@@ -522,9 +560,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_shared_v4(ys + cb * 2, make_uint4(pk[0], pk[1], pk[2], pk[3]));
           st_shared_v4(ys + cb * 2 + 16, make_uint4(pk[4], pk[5], pk[6], pk[7]));
         }
-        named_bar_sync(1, kConvThreads);
+        named_bar_sync(1, kEpiThreads);
         constexpr int kChunksPerRow = BN / 8;
-        for (int c = threadIdx.x; c < kBM * kChunksPerRow; c += kConvThreads) {
+        for (int c = threadIdx.x; c < kBM * kChunksPerRow; c += kEpiThreads) {
           const int rr = c / kChunksPerRow, cc = c % kChunksPerRow;
           const int g_p = tile_p * kBM + rr, g_q = tile_q * BN + cc * 8;
           if (g_p >= prm.rows_p || g_q >= prm.rows_q) continue;  // N % 8 == 0
@@ -538,7 +576,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ------------------------------------------------------------ teardown
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
@@ -593,7 +631,6 @@ int num_sms() {
   return n;
 }
 
-constexpr int kMaxSplits = 8;  // portable cluster size
 
 Plan make_plan(int M, int N, int K) {
   Plan p{};
@@ -626,7 +663,7 @@ Plan make_plan(int M, int N, int K) {
   return p;
 }
 
-template <int BN, bool SWAP, int NSTG, int NOPS, int NACC, bool RECV>
+template <int BN, bool SWAP, int NSTG, int NOPS, int NACC, bool RECV, int CW>
 cudaError_t launch_variant(const GemmArgs& a, const Plan& pl, const GemmParams& prm,
                            cudaStream_t stream) {
   using L = SmemLayout<BN, NSTG, NOPS, RECV>;
@@ -635,7 +672,7 @@ cudaError_t launch_variant(const GemmArgs& a, const Plan& pl, const GemmParams& 
   const uint8_t* Q = SWAP ? a.Xq : a.Wq;
   if (!make_packed_map(&map_p, P, prm.rows_p, a.K, kBM)) return cudaErrorInvalidValue;
   if (!make_packed_map(&map_q, Q, prm.rows_q, a.K, BN)) return cudaErrorInvalidValue;
-  auto kern = w4a4_lr_gemm_kernel<BN, SWAP, NSTG, NOPS, NACC, RECV>;
+  auto kern = w4a4_lr_gemm_kernel<BN, SWAP, NSTG, NOPS, NACC, RECV, CW>;
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
@@ -647,7 +684,7 @@ cudaError_t launch_variant(const GemmArgs& a, const Plan& pl, const GemmParams& 
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pl.tiles_p, pl.tiles_q, pl.splits);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(32 * (CW + 2), 1, 1);
   cfg.dynamicSmemBytes = L::kAlloc;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -690,13 +727,13 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream) {
   prm.acc_out = a.acc_out;
   prm.status = reinterpret_cast<uint32_t*>(a.ws);
   prm.use_lr = (a.r > 0 && !debug) ? 1 : 0;
-  //                                BN  SWAP  NSTG NOPS NACC RECV
-  if (!pl.swap) return launch_variant<256, false, 2, 2, 1, false>(a, pl, prm, stream);
+  //                                BN  SWAP  NSTG NOPS NACC RECV  CW
+  if (!pl.swap) return launch_variant<256, false, 2, 2, 1, false, 8>(a, pl, prm, stream);
   switch (pl.bn) {
-    case 16: return launch_variant<16, true, 4, 4, 4, true>(a, pl, prm, stream);
-    case 32: return launch_variant<32, true, 4, 4, 4, true>(a, pl, prm, stream);
-    case 64: return launch_variant<64, true, 4, 4, 4, false>(a, pl, prm, stream);
-    default: return launch_variant<128, true, 2, 4, 2, false>(a, pl, prm, stream);
+    case 16: return launch_variant<16, true, 4, 4, 1, true, 8>(a, pl, prm, stream);
+    case 32: return launch_variant<32, true, 4, 4, 1, true, 8>(a, pl, prm, stream);
+    case 64: return launch_variant<64, true, 4, 4, 1, false, 8>(a, pl, prm, stream);
+    default: return launch_variant<128, true, 2, 4, 1, false, 8>(a, pl, prm, stream);
   }
 }
 
