@@ -27,8 +27,9 @@ namespace tq {
 
 namespace {
 
-constexpr int kActRows = 16;       // tokens per cluster (one warp each)
-constexpr int kActThreads = 512;   // 16 warps
+constexpr int kActRows = 16;       // tokens per cluster
+constexpr int kActWarps = 8;       // warp w handles tokens w and w + 8
+constexpr int kActThreads = 32 * kActWarps;
 constexpr unsigned kFull = 0xffffffffu;
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -137,7 +138,7 @@ struct ActParams {
   float* s_x;
   float* XL1;
   int M, K, b, r;
-  int passes_per_cta;  // P
+  int passes_per_cta;  // P: warp passes of W = 32E columns in this CTA's slice
   int total_passes;    // K / W
   int kc;              // L1 k-chunk (columns) staged per step
   int l1_bufs;         // staged chunk buffers (all chunks, or 2)
@@ -173,16 +174,49 @@ struct ActSmem {
     total = off_amax + (size_t)(C + 1) * kActRows * 4;
   }
 };
-// Staged L1^T chunks: all of the slice at once when it fits in this budget
-// (one round trip to memory), else a double buffer.
-constexpr size_t kL1AllBudget = 81920;
+// Staged L1^T chunks: all of the slice at once when they fit in this budget
+// (one round trip to memory), else a double buffer.  Kept small so that
+// several CTAs share an SM and hide each other's latencies.
+constexpr size_t kL1AllBudget = 40 * 1024;
 // Dynamic shared memory the kernel is allowed (every supported shape fits).
 constexpr size_t kActSmemMax = 200 * 1024;
 
+// Loads E consecutive bf16 values of a row from shared memory as fp32.
 template <int E>
-__global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActParams p) {
+__device__ __forceinline__ void load_row_values(const __nv_bfloat16* src, float (&v)[E]) {
+  if constexpr (E >= 8) {
+#pragma unroll
+    for (int i = 0; i < E; i += 8) {  // 16-byte aligned: lane * E * 2 bytes
+      const uint4 u = *reinterpret_cast<const uint4*>(src + i);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        v[i + 2 * j] = f.x;
+        v[i + 2 * j + 1] = f.y;
+      }
+    }
+  } else {  // E == 4: one 8-byte load
+    const uint2 u = *reinterpret_cast<const uint2*>(src);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float2 f = __bfloat1622float2(h2[j]);
+      v[2 * j] = f.x;
+      v[2 * j + 1] = f.y;
+    }
+  }
+}
+
+// One cluster of C CTAs owns 16 tokens; CTA c owns columns
+// [c*P*W, (c+1)*P*W) of K.  Warp w handles tokens w and w+8.  The transform
+// is computed twice from the shared-memory copy of X -- once for the absmax,
+// once for the codes after the cluster has combined the absmax -- so no
+// rotated values have to be kept.  Both passes run the same butterflies in
+// the same order, so they give the same bits.
+template <int E>
+__global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActParams p) {
   constexpr int W = 32 * E;
-  constexpr int PMAX = 64 / E;  // register budget: PMAX * E values per lane
   extern __shared__ __align__(128) uint8_t smem[];
 
   pdl_launch_dependents();  // let the GEMM start streaming its weights
@@ -200,6 +234,7 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
   float* recv = reinterpret_cast<float*>(smem + L.off_recv);
   float* amax_all = reinterpret_cast<float*>(smem + L.off_amax);  // [C][16]
   float* amax_row = amax_all + csize * kActRows;
+
   const int pass0 = (int)crank * P;
   const int np = min(P, p.total_passes - pass0);
   const int slice = np * W;
@@ -240,70 +275,47 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
   } else if (nchunks > 0) {
     stage_l1(0, 0);
   }
-  // X is the oldest group; wait for it only (L1 chunks may still be in flight)
-  if (nchunks == 0) cp_async_wait<0>();
-  else if (all_l1) {
-    // groups: X, chunk 0..nchunks-1 -> at most nchunks pending means X done;
-    // wait_group takes an immediate, so wait for everything when chunks are few
-    cp_async_wait<0>();
-  } else {
-    cp_async_wait<1>();
-  }
+  // X is the oldest group: wait for it alone when L1 is double-buffered
+  if (nchunks == 0 || all_l1) cp_async_wait<0>();
+  else cp_async_wait<1>();
   __syncthreads();
 
-  // ---- rotation of this warp's token: PMAX passes of W columns
-  float v[PMAX][E];
-  float amax = 0.f;
-  const int my_row = row0 + warp;
+  // ---- pass 1: transform, absmax of tokens warp and warp + 8
+  float amax[2] = {0.f, 0.f};
+  for (int t = 0; t < 2; ++t) {
+    const int rr = warp + 8 * t;
+    for (int ps = 0; ps < np; ++ps) {
+      float v[E];
+      load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
+      fwht_warp<E>(v, p.b);
 #pragma unroll
-  for (int ps = 0; ps < PMAX; ++ps) {
-    if (ps < np) {
-      const __nv_bfloat16* src = xs + (size_t)warp * L.xs_stride + ps * W + lane * E;
-      if constexpr (E >= 8) {
-#pragma unroll
-        for (int i = 0; i < E; i += 8) {  // 16-byte aligned: lane * E * 2 bytes
-          const uint4 u = *reinterpret_cast<const uint4*>(src + i);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const float2 f = __bfloat1622float2(h2[j]);
-            v[ps][i + 2 * j] = f.x;
-            v[ps][i + 2 * j + 1] = f.y;
-          }
-        }
-      } else {  // E == 4: one 8-byte load
-        const uint2 u = *reinterpret_cast<const uint2*>(src);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const float2 f = __bfloat1622float2(h2[j]);
-          v[ps][2 * j] = f.x;
-          v[ps][2 * j + 1] = f.y;
-        }
-      }
-      fwht_warp<E>(v[ps], p.b);
-#pragma unroll
-      for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[ps][i]));
+      for (int i = 0; i < E; ++i) amax[t] = fmaxf(amax[t], fabsf(v[i]));
     }
+    amax[t] = warp_max(amax[t]);
   }
-  amax = warp_max(amax);
   cluster_wait_acquire();  // every peer is running before it is written to
-  // every CTA of the cluster gets this CTA's partial absmax of token `warp`
-  if (lane < (int)csize)
-    dsmem_st_f32(dsmem_map(smem_u32(&amax_all[crank * kActRows + warp]), (uint32_t)lane), amax);
+  // every CTA of the cluster gets this CTA's partial absmax of both tokens
+  if (lane < (int)csize) {
+    dsmem_st_f32(dsmem_map(smem_u32(&amax_all[crank * kActRows + warp]), (uint32_t)lane), amax[0]);
+    dsmem_st_f32(dsmem_map(smem_u32(&amax_all[crank * kActRows + warp + 8]), (uint32_t)lane),
+                 amax[1]);
+  }
 
-  // ---- X L1 partial over this CTA's slice: warp w owns 8-column tile
-  //      (w % NT) of r and k-part (w / NT) of every staged chunk
+  // ---- X L1 partial over this CTA's slice: warp w owns 8-column tiles
+  //      (w % NT8) + 8j of r and k-part w / NT8 of every staged chunk; two
+  //      accumulator chains per tile (even / odd k steps)
   if (nchunks > 0) {
     const int ntiles = p.r / 8;
+    const int nt8 = min(ntiles, kActWarps);
     const int KP = p.kparts;
-    const int kp = warp / min(ntiles, 16);
-    const bool active = warp < min(ntiles, 16) * KP;
-    constexpr int kMaxTilesPerWarp = 4;  // r <= 512
-    float acc[kMaxTilesPerWarp][4];
+    const int kp = warp / nt8;
+    const bool active = warp < nt8 * KP;
+    constexpr int kMaxTilesPerWarp = 8;  // r <= 512
+    float acc[kMaxTilesPerWarp][2][4];
 #pragma unroll
     for (int t = 0; t < kMaxTilesPerWarp; ++t)
-      acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) acc[t][h][0] = acc[t][h][1] = acc[t][h][2] = acc[t][h][3] = 0.f;
     const uint32_t xs_base = smem_u32(xs);
     const int ksteps = p.kc / 16;
     const int ks0 = kp * ksteps / KP, ks1 = (kp + 1) * ksteps / KP;
@@ -322,6 +334,7 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
       if (active) {
         for (int ks = ks0; ks < ks1; ++ks) {
           const int kk = ks * 16;
+          const int h = ks & 1;
           uint32_t a[4];
           {
             const int mat = lane >> 3, rin = lane & 7;
@@ -331,14 +344,15 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
           }
 #pragma unroll
           for (int t = 0; t < kMaxTilesPerWarp; ++t) {
-            const int tile = (warp % min(ntiles, 16)) + 16 * t;
+            const int tile = (warp % nt8) + kActWarps * t;
             if (tile < ntiles) {
               uint32_t bb[2];
               const int l = lane & 15;
               const int jr = tile * 8 + (l & 7);
               const int cc = kk + (l >> 3) * 8;
               ldmatrix_x2(bb, l1_base + (uint32_t)((jr * L.l1_stride + cc) * 2));
-              mma_16816(acc[t], a, bb);
+              if (h == 0) mma_16816(acc[t][0], a, bb);
+              else mma_16816(acc[t][1], a, bb);
             }
           }
         }
@@ -350,13 +364,13 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
       float* pk = partk + (size_t)kp * kActRows * p.r;
 #pragma unroll
       for (int t = 0; t < kMaxTilesPerWarp; ++t) {
-        const int tile = (warp % min(ntiles, 16)) + 16 * t;
+        const int tile = (warp % nt8) + kActWarps * t;
         if (tile < ntiles) {
           const int rr = lane >> 2, cc = tile * 8 + 2 * (lane & 3);
-          pk[rr * p.r + cc] = acc[t][0];
-          pk[rr * p.r + cc + 1] = acc[t][1];
-          pk[(rr + 8) * p.r + cc] = acc[t][2];
-          pk[(rr + 8) * p.r + cc + 1] = acc[t][3];
+          pk[rr * p.r + cc] = acc[t][0][0] + acc[t][1][0];
+          pk[rr * p.r + cc + 1] = acc[t][0][1] + acc[t][1][1];
+          pk[(rr + 8) * p.r + cc] = acc[t][0][2] + acc[t][1][2];
+          pk[(rr + 8) * p.r + cc + 1] = acc[t][0][3] + acc[t][1][3];
         }
       }
     }
@@ -382,19 +396,22 @@ __global__ void __launch_bounds__(kActThreads, 1) quantize_act_kernel(const ActP
   }
   __syncthreads();
 
-  // ---- codes of this CTA's slice
-  if (my_row < p.M) {
-    const float am = amax_row[warp];
+  // ---- pass 2: the same transform again, then codes of this CTA's slice
+  for (int t = 0; t < 2; ++t) {
+    const int rr = warp + 8 * t;
+    const int my_row = row0 + rr;
+    if (my_row >= p.M) continue;  // warp-uniform
+    const float am = amax_row[rr];
     const float inv = am > 0.f ? 7.f / am : 0.f;
     uint8_t* xrow = p.Xq + (size_t)my_row * (p.K / 2);
+    for (int ps = 0; ps < np; ++ps) {
+      float v[E];
+      load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
+      fwht_warp<E>(v, p.b);
+      int q[E];
 #pragma unroll
-    for (int ps = 0; ps < PMAX; ++ps) {
-      if (ps < np) {
-        int q[E];
-#pragma unroll
-        for (int i = 0; i < E; ++i) q[i] = quant_code(v[ps][i], inv);
-        store_packed<E>(q, xrow + (kbase + ps * W) / 2);
-      }
+      for (int i = 0; i < E; ++i) q[i] = quant_code(v[i], inv);
+      store_packed<E>(q, xrow + (kbase + ps * W) / 2);
     }
     if (crank == 0 && lane == 0) p.s_x[my_row] = am * p.scale_mul;
   }
@@ -465,7 +482,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const float* 
 template <int E>
 cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t stream) {
   constexpr int W = 32 * E;
-  constexpr int PMAX = 64 / E;
+  constexpr int PMAX = 2048 / W;  // X tile of at most 2048 columns per CTA
   ActParams prm = prm_in;
   const int tp = prm.K / W;
   int P = (tp + max_cluster - 1) / max_cluster;
@@ -475,19 +492,20 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   prm.passes_per_cta = P;
   prm.total_passes = tp;
   prm.kc = prm.r > 256 ? 32 : (prm.r > 128 ? 64 : 128);
-  if (prm.kc > P * W) prm.kc = P * W;
+  if (prm.kc > W) prm.kc = W;
   const int nchunks_max = (P * W) / prm.kc;
   const size_t all_bytes = (size_t)nchunks_max * prm.r * (prm.kc + 8) * 2;
   prm.l1_bufs = (all_bytes <= kL1AllBudget) ? nchunks_max : 2;
   const int ntiles = prm.r / 8;
-  prm.kparts = (ntiles == 0) ? 1 : std::max(1, std::min(16 / std::min(ntiles, 16), prm.kc / 16));
+  prm.kparts = (ntiles == 0)
+                   ? 1
+                   : std::max(1, std::min(kActWarps / std::min(ntiles, kActWarps), prm.kc / 16));
   const ActSmem<E> L(P, prm.r, prm.kc, prm.l1_bufs, prm.kparts, C);
   auto kern = quantize_act_kernel<E>;
   static uint64_t attr_set = 0;  // one bit per device
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set >> dev & 1u)) {
-    // the largest carve-up any supported shape needs (P * W <= 2048, r <= 512)
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kActSmemMax);
     if (e != cudaSuccess) return e;
