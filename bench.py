@@ -181,6 +181,8 @@ def build_layers(tq, torch, M, L, seed0, device):
             "Y": torch.empty(M, N_DIM, dtype=torch.bfloat16, device=device),
             "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N_DIM, K_DIM, RANK),
                               dtype=torch.uint8, device=device),
+            "lws": torch.zeros(tq.tq_layer_workspace_bytes(M, N_DIM, K_DIM, RANK),
+                               dtype=torch.uint8, device=device),
         }
         layers.append(lay)
     torch.cuda.synchronize()
@@ -188,13 +190,20 @@ def build_layers(tq, torch, M, L, seed0, device):
 
 
 def layer_call(tq, lay, ev=None):
-    tq.tq_quantize_act(lay["X"], HAD, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
+    """The layer through tq_w4a4_lr_layer (one fused kernel at these sizes)."""
     if ev is not None:
         ev[0].record()
-    tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"], lay["L2t"],
-                       Y=lay["Y"], workspace=lay["ws"])
+    tq.tq_w4a4_lr_layer(lay["X"], lay["L1t"], lay["Wq"], lay["s_w"], lay["L2t"], HAD,
+                        Y=lay["Y"], workspace=lay["lws"])
     if ev is not None:
         ev[1].record()
+
+
+def layer_call_two(tq, lay):
+    """The same layer through the two-call path (tq_quantize_act, tq_w4a4_lr_gemm)."""
+    tq.tq_quantize_act(lay["X"], HAD, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
+    tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"], lay["L2t"],
+                       Y=lay["Y"], workspace=lay["ws"])
 
 
 def capture(torch, fn):
@@ -289,6 +298,11 @@ def run_tq(args, rank, world, local_rank, dist):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms_e2e = float(t.item())
 
+    # the two-call path on the same layers, for comparison
+    g_two = capture(torch, lambda: [layer_call_two(tq, l) for l in layers])
+    ms_two = time_graph(torch, g_two, args.steps, args.warmup)
+    del g_two
+
     sweep = {}
     if not args.no_sweep and world == 1:
         for m2 in (1, 128):
@@ -311,10 +325,10 @@ def run_tq(args, rank, world, local_rank, dist):
     value = world * bytes_step / ms / 1e6          # GB/s, all ranks
     e2e = world * bytes_step / ms_e2e / 1e6
     peak, peak_src = measured_peaks()
-    gb = gemm_bytes(M, K_DIM, N_DIM, RANK)
+    gb = layer_bytes(M, K_DIM, N_DIM, RANK)   # the fused kernel reads X, writes Y
     achieved = gb / (gemm_ms_avg * 1e-3) / 1e9
-    traffic = profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm.cu",
-                               "w4a4_lr_gemm_decode_m16.md") if M == 16 else None
+    traffic = profiled_traffic("rank_int4_gemm_b200/csrc/tq_layer.cu",
+                               "w4a4_lr_layer_decode_m16.md") if M == 16 else None
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
@@ -328,23 +342,27 @@ def run_tq(args, rank, world, local_rank, dist):
             "layers_per_step": L,
             "l2": f"inputs larger than L2: {L} layers x {gb / 1e6:.1f} MB of GEMM operands",
             "parallelism": f"{world} independent replica(s), no data-path collective",
-            "graph": "one CUDA graph per step; GEMM launched with programmatic dependent launch",
+            "graph": "one CUDA graph per step; one tq_w4a4_lr_layer launch per layer "
+                     "(fused decode kernel), launched with programmatic dependent launch",
         },
         "TOPS": round(world * L * 2 * M * N_DIM * K_DIM / ms / 1e9, 3),
         "us_per_layer": round(ms * 1e3 / L, 3),
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "w4a4_lr_gemm_kernel (decode tiling, split-K)",
-            "gemm_us": round(gemm_ms_avg * 1e3, 3),
+            "kernel": "w4a4_lr_layer_decode_kernel (whole layer, split-K cluster)",
+            "kernel_us": round(gemm_ms_avg * 1e3, 3),
             "algorithmic_bytes_per_launch": gb, "peak_source": peak_src,
         },
         "e2e": {"value": round(e2e, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": sum(x.numel() * x.element_size() for x in hx),
                 "d2h_bytes_per_step": sum(y.numel() * y.element_size() for y in hy),
                 "ms_per_step": round(ms_e2e, 5)},
-        "gpu_launches": 2 * L * args.steps,
+        "gpu_launches": L * args.steps,
         "clocks": clocks,
+        "two_call_path": {"GB/s": round(world * bytes_step / ms_two / 1e6, 1),
+                          "us_per_layer": round(ms_two * 1e3 / L, 3),
+                          "calls": "tq_quantize_act + tq_w4a4_lr_gemm"},
     }
     if sweep:
         out["sweep"] = sweep

@@ -133,6 +133,34 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * tq_w4a4_lr_layer -- the whole layer from bf16 activations:
+ *
+ *   Y = bf16( s_x s_w (Q4(X H) . Wq) + bf16(X L1) L2 )
+ *
+ * i.e. tq_quantize_act followed by tq_w4a4_lr_gemm, with the same codes,
+ * scales and tolerances.  At decode sizes (M <= 16, r <= 64, K % 512 == 0,
+ * K <= 8192) it runs as ONE kernel: each split-K cluster rotates and
+ * quantizes its own slice of X, exchanges the absmax and X L1 partials in
+ * distributed shared memory and feeds the codes straight to the tensor
+ * cores, while the weights stream in (TwinQuant notes section 04.C: the
+ * residual GEMM quantizes activations concurrently and both paths share one
+ * epilogue).  Other shapes run the two kernels, keeping Xq, s_x and XL1 in
+ * the workspace.
+ *
+ *   X [M][K] bf16, L1t [r][K] bf16 (NULL iff r == 0), Wq [N][K/2] u8,
+ *   s_w [N] fp32, L2t [N][r] bf16 (NULL iff r == 0), Y [M][N] bf16 (out)
+ *   workspace: >= tq_layer_workspace_bytes(M, N, K, r) bytes, zero-filled
+ *   before first use (its first 4 bytes are the watchdog status word)
+ */
+TQ_API size_t tq_layer_workspace_bytes(int M, int N, int K, int r);
+TQ_API int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t,
+                            const uint8_t* Wq, const float* s_w,
+                            const uint16_t* L2t, int M, int N, int K, int r,
+                            int had_block, uint16_t* Y,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
  * tq_debug_w4a4_gemm_acc -- test hook: the same GEMM kernel with the
  * low-rank branch off, writing the raw INT32 accumulators
  * acc[m][n] = sum_k qx[m][k] qw[n][k] to `acc` [M][N] (int32) instead of Y.

@@ -140,6 +140,71 @@ int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
                      workspace, workspace_bytes, stream);
 }
 
+// Layer workspace: [status 256][Xq M*K/2][s_x 4M][XL1 4Mr], 256-aligned parts.
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {
+  if (M <= 0 || N <= 0 || K <= 0 || r < 0) return 256;
+  return 256 + align256((size_t)M * K / 2) + align256((size_t)M * 4) + align256((size_t)M * r * 4);
+}
+
+int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
+                     const uint16_t* L2t, int M, int N, int K, int r, int had_block, uint16_t* Y,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  if (!X || !Wq || !s_w || !Y || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y) ||
+      (L1t && !aligned16(L1t)) || (L2t && !aligned16(L2t)) ||
+      (workspace && !aligned16(workspace)))
+    return TQ_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < tq_layer_workspace_bytes(M, N, K, r))
+    return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (tq::layer_decode_supported(M, N, K, r, had_block)) {
+    tq::LayerArgs a{};
+    a.X = X;
+    a.L1t = L1t;
+    a.Wq = Wq;
+    a.s_w = s_w;
+    a.L2t = L2t;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.had_block = had_block;
+    a.Y = Y;
+    a.ws = workspace;
+    return from_cuda(tq::launch_layer_decode(a, st));
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Xq = ws + 256;
+  float* s_x = reinterpret_cast<float*>(Xq + align256((size_t)M * K / 2));
+  float* XL1 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + align256((size_t)M * 4));
+  if (cudaError_t e = tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x,
+                                              r > 0 ? XL1 : nullptr, st))
+    return from_cuda(e);
+  tq::GemmArgs g{};
+  g.Xq = Xq;
+  g.s_x = s_x;
+  g.Wq = Wq;
+  g.s_w = s_w;
+  g.XL1 = r > 0 ? XL1 : nullptr;
+  g.L2t = L2t;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.r = r;
+  g.Y = Y;
+  g.acc_out = nullptr;
+  g.ws = workspace;
+  g.ws_bytes = 256;
+  return from_cuda(tq::launch_gemm(g, st));
+}
+
 int tq_query_device_status(void* workspace, void* stream) {
   if (!workspace) return TQ_ERR_INVALID_VALUE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

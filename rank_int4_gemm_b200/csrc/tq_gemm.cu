@@ -620,7 +620,7 @@ struct Plan {
   int tiles_p, tiles_q;
 };
 
-int num_sms() {
+int num_sms_cached() {
   static int n = 0;
   if (!n) {
     int dev = 0;
@@ -643,7 +643,7 @@ Plan make_plan(int M, int N, int K) {
     p.tiles_p = (N + kBM - 1) / kBM;
     p.tiles_q = (M + p.bn - 1) / p.bn;
     int s = tuning().split_k;
-    if (s <= 0) s = std::max(1, num_sms() / (p.tiles_p * p.tiles_q));
+    if (s <= 0) s = std::max(1, num_sms_cached() / (p.tiles_p * p.tiles_q));
     s = std::max(1, std::min(std::min(s, kb), kMaxSplits));
     p.kb_per_split = (kb + s - 1) / s;
     // whole staged stages per split when that keeps the split count
@@ -700,6 +700,22 @@ cudaError_t launch_variant(const GemmArgs& a, const Plan& pl, const GemmParams& 
 }
 
 }  // namespace
+
+int num_sms() { return num_sms_cached(); }
+
+bool encode_tiled_2d(CUtensorMap* m, CUtensorMapDataType dtype, const void* ptr, uint64_t inner,
+                     uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                     CUtensorMapSwizzle swizzle) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t gemm_workspace_bytes(int M, int N, int K, int r) {
   (void)M; (void)N; (void)K; (void)r;

@@ -2,6 +2,7 @@
 #pragma once
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace tq {
@@ -36,5 +37,25 @@ struct GemmArgs {
 
 size_t gemm_workspace_bytes(int M, int N, int K, int r);
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream);
+
+// The whole layer from bf16 X (decode sizes: one fused kernel).
+struct LayerArgs {
+  const uint16_t* X;
+  const uint16_t* L1t;
+  const uint8_t* Wq;
+  const float* s_w;
+  const uint16_t* L2t;
+  int M, N, K, r, had_block;
+  uint16_t* Y;
+  void* ws;  // status word at offset 0
+};
+bool layer_decode_supported(int M, int N, int K, int r, int had_block);
+cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
+
+// Shared host helpers (defined in tq_gemm.cu).
+int num_sms();
+bool encode_tiled_2d(CUtensorMap* m, CUtensorMapDataType dtype, const void* ptr,
+                     uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
+                     uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 }  // namespace tq

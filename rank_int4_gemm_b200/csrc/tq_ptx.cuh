@@ -70,6 +70,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps (up to `ns`) instead
+// of spinning, leaving issue slots to the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // kWaitBudgetCycles: records kDevTimeout in *status (if not null), raises the
 // CTA-wide abort flag and returns false.  Callers stop their role loop then.
@@ -78,8 +92,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   for (uint32_t it = 0;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 63u) {
+    if (mbar_try_wait_sleep(bar, parity, 200u)) return true;
+    if ((it & 15u) == 15u) {
       if (abort_flag && *abort_flag) return false;
       if (clock64() - t0 > kWaitBudgetCycles) {
         if (status) atomicExch(status, kDevTimeout);

@@ -40,6 +40,11 @@ _lib.tq_debug_w4a4_gemm_acc.restype = _I
 _lib.tq_debug_w4a4_gemm_acc.argtypes = [_P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
 _lib.tq_w4a4_lr_gemm_noalloc.restype = _I
 _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
+_lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.tq_w4a4_lr_layer.restype = _I
+_lib.tq_w4a4_lr_layer.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                                  ctypes.c_size_t, _P]
 _lib.tq_query_device_status.restype = _I
 _lib.tq_query_device_status.argtypes = [_P, _P]
 
@@ -198,8 +203,29 @@ def tq_query_device_status(workspace, stream=None) -> int:
     return int(_lib.tq_query_device_status(_ptr(ws), _stream(stream)))
 
 
+def tq_layer_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    return int(_lib.tq_layer_workspace_bytes(M, N, K, r))
+
+
+def tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None, stream=None):
+    """The whole layer from bf16 X: Y [M][N] bf16 (one kernel at decode sizes)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    r = 0 if L1t is None else L1t.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = Workspace(X.device)
+    need = tq_layer_workspace_bytes(M, N, K, r)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_layer(_ptr(X), _ptr(L1t) if r else None, _ptr(Wq), _ptr(s_w),
+                                 _ptr(L2t) if r else None, M, N, K, r, int(had_block), _ptr(Y),
+                                 _ptr(ws), ws.numel(), _stream(stream)), "tq_w4a4_lr_layer")
+    return Y
+
+
 def layer_forward(X, L1t, L2t, Wq, s_w, had_block, workspace=None, stream=None, out=None):
-    """One layer: tq_quantize_act then tq_w4a4_lr_gemm (two kernel launches)."""
+    """One layer through the two-call path: tq_quantize_act then tq_w4a4_lr_gemm."""
     Xq, s_x, XL1 = tq_quantize_act(X, had_block, L1t, stream=stream)
     return tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w, XL1, L2t, Y=out, workspace=workspace,
                            stream=stream)
