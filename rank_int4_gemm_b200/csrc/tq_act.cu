@@ -276,16 +276,20 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     const int my_row = row0 + rr;
     if (my_row >= p.M) continue;  // warp-uniform
     const float am = amax_row[rr];
-    const float inv = am > 0.f ? 7.f / am : 0.f;
+    const CodeScale cs = code_scale(am);
     uint8_t* xrow = p.Xq + (size_t)my_row * (p.K / 2);
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
       fwht_warp<E>(v, p.b);
-      int q[E];
+      if (cs.pre != 1.f) {
 #pragma unroll
-      for (int i = 0; i < E; ++i) q[i] = quant_code(v[i], inv);
-      store_packed<E>(q, xrow + (kbase + ps * W) / 2);
+        for (int i = 0; i < E; ++i) v[i] *= cs.pre;
+      }
+      uint32_t cb[E];
+#pragma unroll
+      for (int i = 0; i < E; ++i) cb[i] = code_bits(v[i], cs.inv);
+      store_packed<E>(cb, xrow + (kbase + ps * W) / 2);
     }
     if (crank == 0 && lane == 0) p.s_x[my_row] = am * p.scale_mul;
   }

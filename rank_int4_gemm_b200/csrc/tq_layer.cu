@@ -2,27 +2,36 @@
 //
 //   Y = dequant( Q4(X H) . Q4(H^T R) ) + bf16(X L1) L2
 //
-// Per output tile of 128 channels, a cluster of S CTAs splits K (split-K).
-// CTA z owns k-blocks [z*kbps, ...) of K.  Its warps:
+// Per output tile of 128 channels, a cluster of S CTAs splits K (split-K);
+// CTA z owns k-blocks [z*kbps, ...) of K, at most 1024 columns.  Its warps:
 //
-//   warps 0-7   activation: read the tokens' slice of X straight from L2,
-//               Sylvester transform (the same warp butterflies as
-//               tq_quantize_act, so the codes are the same bits), partial
-//               absmax, X.L1 partial on mma.sync; the cluster exchanges
-//               absmax and X.L1 partials through distributed shared memory;
-//               then the token codes are written as int8 (16 * code) straight
-//               into the MMA's B operand.  Warps 0-3 run the epilogue.
-//   warps 8-11  expand the streamed int4 weights to int8 operand tiles and,
-//               in split 0, stage the L2^T rows of the tile.
-//   warp 12     TMA producer of the packed weights (started before the
-//               kernel waits on its predecessor: weights never depend on it).
-//   warp 13     TMEM allocation and MMA issue: kind::i8 for the codes,
+//   warps 0-15  activation, warp t = token t: the token's slice of X is
+//               staged once in shared memory; Sylvester transform (the warp
+//               butterflies of tq_quantize_act, so the codes are the same
+//               bits) and partial absmax, exchanged across the cluster through
+//               distributed shared memory; the rotated values stay in
+//               registers and become the codes, written as int8 (16 * code)
+//               straight into the MMA's B operand.  Only then, off the path
+//               to the integer MMAs, the same warps compute the slice's X.L1
+//               partial on mma.sync (L1^T fragments were fetched into
+//               registers before the kernel waited on its predecessor) and
+//               push it to split 0.  Warps 0-3 run the epilogue.
+//   warps 16-19 expand the streamed int4 weights into int8 operand slots;
+//               the first kNOPS k-blocks are expanded before the token codes
+//               exist, so only the rest wait on the MMA.  In split 0 they also
+//               place the tile's L2^T rows (the low-rank A operand).
+//   warp 20     TMA producer of the packed weights (started before the kernel
+//               waits on its predecessor: weights never depend on it).
+//   warp 21     TMEM allocation and MMA issue: kind::i8 for the codes,
 //               kind::f16 for the low-rank branch (split 0).
 //
-// The epilogue is the split-K reduction of the GEMM kernel: each split pushes
-// its INT32 partial rows to the row's owner CTA, owners reduce in split order
-// and store Y.  Nothing goes through global memory except X, the weights and
-// Y.  No TMA multicast.
+// Cluster barriers, all threads of all CTAs in order: B0 (every CTA is
+// running), B1 (absmax partials delivered), B2 (X.L1 partials delivered),
+// B3 (split-K partial rows delivered).  The epilogue is the GEMM kernel's
+// split-K reduction: each split pushes its INT32 partial rows to the row's
+// owner CTA, owners reduce in split order and store Y.  Nothing goes through
+// global memory except X, the weights, L1^T, L2^T, s_w and Y.  No TMA
+// multicast.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -41,20 +50,20 @@ constexpr int kBN = 16;            // tokens (MMA N)
 constexpr int kKB = 128;           // codes per k-block
 constexpr int kPackedRow = 64;     // packed bytes per row per k-block
 constexpr int kKBS = 2;            // k-blocks per TMA stage (128-byte swizzled rows)
-constexpr int kNSTG = 2;           // TMA stages
-constexpr int kNOPS = 2;           // int8 operand slots
+constexpr int kNSTG = 4;           // TMA stages: a whole 1024-column slice requested at once
+constexpr int kNOPS = 4;           // int8 operand slots
 constexpr int kMaxKb = 8;          // k-blocks per CTA (slice <= 1024 columns)
-constexpr int kMaxSplits = 4;     // split-K cluster size limit of this kernel
-constexpr int kMaxR = 64;          // low-rank width handled here
+constexpr int kMaxSplits = 4;      // split-K cluster size limit of this kernel
+constexpr int kMaxR = 32;          // low-rank width handled here
 constexpr int kE = 16;             // values per lane per warp pass
 constexpr int kW = 32 * kE;        // 512 columns per warp pass
-constexpr int kL1Chunk = 256;      // L1^T columns per staged chunk
-constexpr int kActWarps = 8, kConvWarps = 4;
-constexpr int kProducerWarp = 12, kMmaWarp = 13;
-constexpr int kThreads = 14 * 32;
+constexpr int kActWarps = 16, kConvWarps = 4;
+constexpr int kProducerWarp = kActWarps + kConvWarps, kMmaWarp = kProducerWarp + 1;
+constexpr int kThreads = (kMmaWarp + 1) * 32;
 constexpr int kActThreads = kActWarps * 32;
 constexpr int kConvThreads = kConvWarps * 32;
 constexpr int kEpiThreads = 128;
+constexpr int kMaxBPair = 8;       // X L1 k-step pairs per warp (B fragments held in registers)
 
 struct LayerParams {
   const __nv_bfloat16* X;    // [M][K]
@@ -70,24 +79,23 @@ struct LayerParams {
 
 // Shared-memory map (offsets from the 1024-aligned base).
 struct Smem {
-  static constexpr uint32_t kStg = kBM * 128;                 // one TMA stage
   static constexpr uint32_t kOp = kBM * 128;                  // one int8 weight k-block
-  static constexpr uint32_t kStgBase = 0;
-  static constexpr uint32_t kOpBase = kStgBase + kNSTG * kStg;  // also the L2^T tile (split 0)
-  static constexpr uint32_t kBBase = kOpBase + kNOPS * kOp;   // token codes [kb][16][128]
+  static constexpr uint32_t kStg = kBM * 128;                 // one TMA stage (2 k-blocks packed)
+  static constexpr uint32_t kOpBase = 0;                      // also the L2^T tile (split 0)
+  static constexpr uint32_t kStgBase = kOpBase + kNOPS * kOp;
+  static constexpr uint32_t kBBase = kStgBase + kNSTG * kStg;  // token codes [kb][16][128]
   static constexpr uint32_t kBBytes = kMaxKb * kBN * 128;
   static constexpr uint32_t kLrBBase = kBBase + kBBytes;      // bf16(XL1) [16][64], SW128
-  static constexpr uint32_t kXBase = kLrBBase + kBN * 128;    // X slice [16][1024 + 8] bf16
-  static constexpr uint32_t kXStride = kMaxKb * kKB + 8;      // bf16 elements per row
-  static constexpr uint32_t kXBytes = kBN * kXStride * 2;
-  static constexpr uint32_t kL1Base = kXBase + kXBytes;       // L1^T chunks [4|2][r][256 + 8]
-  static constexpr uint32_t kL1Stride = kL1Chunk + 8;         // bf16 elements per row
-  static constexpr uint32_t kL1Bytes = 2 * kMaxR * kL1Stride * 2;
-  static constexpr uint32_t kXRecv = kL1Base + kL1Bytes;      // XL1 partials [S][16][r] fp32
-  static constexpr uint32_t kXRecvBytes = kMaxSplits * kBN * kMaxR * 4;
-  static constexpr uint32_t kKRecv = kXRecv + kXRecvBytes;    // split-K [S][16][rows], lr [16][rows]
+  static constexpr uint32_t kXBase = kLrBBase + kBN * 128;    // X slice [16][1024] bf16, swizzled
+  static constexpr uint32_t kXRow = kMaxKb * kKB * 2;         // bytes per X row
+  static constexpr uint32_t kXBytes = kBN * kXRow;
+  // split-K partials [S][16][rows] + low-rank [16][rows]; before the epilogue
+  // the X L1 k-part partials [KP][16][r]
+  static constexpr uint32_t kKRecv = kXBase + kXBytes;
   static constexpr uint32_t kKRecvBytes = 2 * kBN * kBM * 4;  // largest at S = 1
-  static constexpr uint32_t kAmax = kKRecv + kKRecvBytes;     // [S][16] + [16]
+  static constexpr uint32_t kXRecv = kKRecv + kKRecvBytes;    // XL1 partials [S][16][r] fp32
+  static constexpr uint32_t kXRecvBytes = kMaxSplits * kBN * kMaxR * 4;
+  static constexpr uint32_t kAmax = kXRecv + kXRecvBytes;     // [S][16] + [16]
   static constexpr uint32_t kScale = kAmax + (kMaxSplits + 1) * kBN * 4;  // s_w [128]
   static constexpr uint32_t kBar = kScale + kBM * 4;
   // barriers: stg_full, stg_empty, op_full, op_empty, b_ready, lr_ready, acc_full
@@ -97,6 +105,7 @@ struct Smem {
   static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 static_assert(Smem::kAlloc <= 227 * 1024, "fused layer shared memory");
+static_assert(kActWarps * kBN * 8 * 4 <= Smem::kKRecvBytes, "X L1 k-part partials");
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -120,6 +129,9 @@ __device__ __forceinline__ float ld_shared_f32(uint32_t addr) {
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
   return v;
 }
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -133,11 +145,35 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t ldg_u32(const __nv_bfloat16* p) {
+  return __ldg(reinterpret_cast<const unsigned int*>(p));
+}
 __device__ __forceinline__ int owned_lo(int o, int S) { return (o * kBM + S - 1) / S; }
 
 // 16-byte chunk j (0..7) of row `row` of a 128-byte-swizzled K-major tile.
 __device__ __forceinline__ uint32_t sw_off(uint32_t row, uint32_t j) {
   return row * 128u + ((j ^ (row & 7u)) << 4);
+}
+// 16-byte chunk c (0..127) of row `row` (0..15) of the staged X slice; the
+// chunk index is XORed with the row so that the 8 rows of an ldmatrix land
+// in different banks.
+__device__ __forceinline__ uint32_t x_off(uint32_t row, uint32_t c) {
+  return row * Smem::kXRow + ((c ^ (row & 7u)) << 4);
+}
+
+// This lane's kE = 16 consecutive values of token `row`, columns
+// col0 .. col0 + 15 of the staged slice, as fp32.
+__device__ __forceinline__ void load_x16(uint32_t xbase, int row, int col0, float (&v)[kE]) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint4 u = ld_shared_v4(xbase + x_off((uint32_t)row, (uint32_t)(col0 / 8 + h)));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
+      v[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -158,9 +194,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* acc_full = b_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S_::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S_::kMisc + 4);
-  float* amax_all = reinterpret_cast<float*>(smem + S_::kAmax);  // [S][16]
-  float* amax_row = amax_all + kMaxSplits * kBN;                  // [16]
-  float* sw_tile = reinterpret_cast<float*>(smem + S_::kScale);   // s_w of the tile
+  const uint32_t amax_all = base + S_::kAmax;                 // [S][16] fp32
+  const uint32_t amax_row = amax_all + kMaxSplits * kBN * 4;  // [16] fp32
+  float* sw_tile = reinterpret_cast<float*>(smem + S_::kScale);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -170,10 +206,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_kb = min(p.kb_total - kb0, p.kb_per_split);
   const int n_st = (n_kb + kKBS - 1) / kKBS;
   const int kbase = kb0 * kKB;           // first column of this CTA's slice
-  const int slice = n_kb * kKB;
+  const int slice = n_kb * kKB;          // 512 or 1024 columns
   const bool do_lr = p.r > 0 && split == 0;
   constexpr uint32_t kTmemCols = 32;     // INT32 [16] + fp32 low-rank [16]
 
+  pdl_launch_dependents();  // the next layer may start staging its weights
   // ---------------------------------------------------------------- prologue
   if (warp == kProducerWarp && lane == 0) {
     for (int i = 0; i < kNSTG; ++i) {
@@ -211,189 +248,96 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kActWarps) {
     // =================================================== activation warps
-    const int tid = threadIdx.x;  // 0..255
-    // L1^T chunks 0 and 1 of this slice (a weight: needs no predecessor)
-    const int n_l1 = (p.r > 0) ? slice / kL1Chunk : 0;
-    // chunk buffers of r rows: all chunks of the slice fit when r <= 32
-    const int l1_bufs = (p.r <= kMaxR / 2) ? 4 : 2;
-    const uint32_t l1_buf_bytes = (uint32_t)p.r * S_::kL1Stride * 2u;
-    auto stage_l1 = [&](int ci) {
-      const uint32_t dst = base + S_::kL1Base + (uint32_t)(ci % l1_bufs) * l1_buf_bytes;
-      const int cpr = kL1Chunk / 8;
-      for (int c = tid; c < p.r * cpr; c += kActThreads) {
-        const int j = c / cpr, cc = c - j * cpr;
-        const __nv_bfloat16* src = p.L1t + (size_t)j * p.K + kbase + ci * kL1Chunk + cc * 8;
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                         dst + (uint32_t)(j * S_::kL1Stride + cc * 8) * 2u),
-                     "l"(src)
-                     : "memory");
-      }
-      cp_async_commit();
-    };
-    for (int ci = 0; ci < min(n_l1, l1_bufs); ++ci) stage_l1(ci);
-    // scales of the tile's channels (weights: no predecessor)
-    for (int i = tid; i < kBM; i += kActThreads) {
-      const int g = tile * kBM + i;
-      sw_tile[i] = g < p.N ? __ldg(p.s_w + g) : 0.f;
-    }
-
+    const int tid = threadIdx.x;  // 0..511
+    const int g = lane >> 2, c = lane & 3;
+    // X L1 work split: warp = (n-tile nt, k-part kp); KP k-parts of kspp
+    // k-steps (16 columns) each
+    const int ntiles = p.r / 8;
+    const int KP = ntiles > 0 ? kActWarps / ntiles : 1;
+    const bool xl1_warp = ntiles > 0 && warp < ntiles * KP;
+    const int nt = ntiles > 0 ? warp % ntiles : 0, kp = ntiles > 0 ? warp / ntiles : 0;
+    const int kspp = (slice / 16) / KP;
     pdl_wait();  // X comes from the preceding kernel
 
     // ---- X slice [16][slice] -> shared memory (rows past M are zero)
-    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(smem + S_::kXBase);
+    const uint32_t xbase = base + S_::kXBase;
     {
       const int cpr = slice / 8;  // 16-byte chunks per row
-      for (int c = tid; c < kBN * cpr; c += kActThreads) {
-        const int row = c / cpr, cc = c - row * cpr;
+      for (int ch = tid; ch < kBN * cpr; ch += kActThreads) {
+        const int row = ch / cpr, cc = ch - row * cpr;
         const bool ok = row < p.M;
         const __nv_bfloat16* src = p.X + (size_t)(ok ? row : 0) * p.K + kbase + cc * 8;
-        cp_async16(xs + (size_t)row * S_::kXStride + cc * 8, src, ok);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                         xbase + x_off((uint32_t)row, (uint32_t)cc)),
+                     "l"(src), "r"(ok ? 16u : 0u)
+                     : "memory");
       }
       cp_async_commit();
-      cp_async_wait<0>();  // also completes the L1^T chunks staged above
-      named_bar_sync(3, kActThreads);
     }
+    // L1^T fragments of this warp's k-steps, fetched while X lands.  Inside
+    // each pair of k-steps (32 columns) lane (g, c) takes columns 8c .. 8c+7
+    // of both operands, so one 16-byte load gives its B fragments for the
+    // pair: mma k-step 0 uses columns 8c + {0,1 | 2,3}, k-step 1 uses
+    // 8c + {4,5 | 6,7} (the same bijection on A and B, so every product
+    // X[t][k] L1[k][j] is summed exactly once).
+    uint4 bq[kMaxBPair];
+#pragma unroll
+    for (int i = 0; i < kMaxBPair; ++i) {
+      bq[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (xl1_warp && 2 * i < kspp)
+        bq[i] = __ldg(reinterpret_cast<const uint4*>(
+            p.L1t + (size_t)(nt * 8 + g) * p.K + kbase + 32 * (kp * kspp / 2 + i) + 8 * c));
+    }
+    cp_async_wait<0>();
+    named_bar_sync(1, kActThreads);
 
-    // ---- transform of tokens warp and warp + 8 over this slice; values kept
-    const int np = slice / kW;  // 1 or 2 passes of 512 columns
-    float v[2][2][kE];
-    float amax[2] = {0.f, 0.f};
+    // ---- transform of token `warp` over the slice (kept in registers),
+    //      partial absmax
+    const int np = slice / kW;  // 1 or 2 warp passes
+    float v[2][kE];
+    float amax = 0.f;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int row = warp + 8 * t;
+    for (int ps = 0; ps < 2; ++ps) {
+      if (ps < np) {
+        load_x16(xbase, warp, ps * kW + lane * kE, v[ps]);
+        fwht_warp<kE>(v[ps], p.b);
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
-        if (ps < np) {
-          load_row_values<kE>(xs + (size_t)row * S_::kXStride + ps * kW + lane * kE, v[t][ps]);
-          fwht_warp<kE>(v[t][ps], p.b);
-#pragma unroll
-          for (int i = 0; i < kE; ++i) amax[t] = fmaxf(amax[t], fabsf(v[t][ps][i]));
-        }
+        for (int i = 0; i < kE; ++i) amax = fmaxf(amax, fabsf(v[ps][i]));
       }
-      amax[t] = warp_max(amax[t]);
     }
+    amax = warp_max(amax);
     cluster_wait_acquire();  // B0 complete: every peer is running
-    if (lane < S) {
-      dsmem_st_f32(dsmem_map(smem_u32(&amax_all[split * kBN + warp]), (uint32_t)lane), amax[0]);
-      dsmem_st_f32(dsmem_map(smem_u32(&amax_all[split * kBN + warp + 8]), (uint32_t)lane),
-                   amax[1]);
-    }
-
-    // ---- X L1 partial over the slice: warp w takes k16-steps w, w+8, ...;
-    //      A fragments (tokens x k) straight from global, B from L1^T chunks
-    if (n_l1 > 0) {
-      const int ntiles = p.r / 8;
-      float acc[kMaxR / 8][4];
-#pragma unroll
-      for (int t = 0; t < kMaxR / 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
-      const int r0 = lane >> 2, c0 = 2 * (lane & 3);
-      // warp w owns k16-steps w and w + 8 of every 256-column chunk
-      const uint32_t xs_base = smem_u32(xs);
-      for (int ci = 0; ci < n_l1; ci += 2) {
-        if (l1_bufs == 2) {
-          cp_async_wait<0>();
-          named_bar_sync(3, kActThreads);
-        }
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          if (ci + cc < n_l1) {
-            const uint32_t l1b = base + S_::kL1Base + (uint32_t)((ci + cc) % l1_bufs) * l1_buf_bytes;
-#pragma unroll
-            for (int k2 = 0; k2 < 2; ++k2) {
-              const int ks = warp + 8 * k2;
-              uint32_t a[4];
-              {
-                const int mat = lane >> 3, rin = lane & 7;
-                const int rr = rin + (mat & 1) * 8;
-                const int col = (ci + cc) * kL1Chunk + ks * 16 + (mat >> 1) * 8;
-                ldmatrix_x4(a, xs_base + (uint32_t)((rr * S_::kXStride + col) * 2));
-              }
-#pragma unroll
-              for (int t = 0; t < kMaxR / 8; ++t) {
-                if (t < ntiles) {
-                  uint32_t bb[2];
-                  const int l = lane & 15;
-                  const int jr = t * 8 + (l & 7);
-                  const int c2 = ks * 16 + (l >> 3) * 8;
-                  ldmatrix_x2(bb, l1b + (uint32_t)((jr * S_::kL1Stride + c2) * 2));
-                  mma_16816(acc[t], a, bb);
-                }
-              }
-            }
-          }
-        }
-        if (l1_bufs == 2 && ci + 2 < n_l1) {
-          named_bar_sync(3, kActThreads);  // both buffers consumed
-          stage_l1(ci + 2);
-          if (ci + 3 < n_l1) stage_l1(ci + 3);
-        }
-      }
-      // cross-warp sum in a fixed order through the (still unused) token-code
-      // area: warps 0-3 write, warps 4-7 add, then warp pairs are summed
-      float* red = reinterpret_cast<float*>(smem + S_::kBBase);  // [4][16][r]
-      if (warp < 4) {
-#pragma unroll
-        for (int t = 0; t < kMaxR / 8; ++t)
-          if (t < ntiles) {
-            float* d = red + (warp * kBN) * p.r;
-            d[r0 * p.r + t * 8 + c0] = acc[t][0];
-            d[r0 * p.r + t * 8 + c0 + 1] = acc[t][1];
-            d[(r0 + 8) * p.r + t * 8 + c0] = acc[t][2];
-            d[(r0 + 8) * p.r + t * 8 + c0 + 1] = acc[t][3];
-          }
-      }
-      named_bar_sync(3, kActThreads);
-      if (warp >= 4) {
-#pragma unroll
-        for (int t = 0; t < kMaxR / 8; ++t)
-          if (t < ntiles) {
-            float* d = red + ((warp - 4) * kBN) * p.r;
-            d[r0 * p.r + t * 8 + c0] += acc[t][0];
-            d[r0 * p.r + t * 8 + c0 + 1] += acc[t][1];
-            d[(r0 + 8) * p.r + t * 8 + c0] += acc[t][2];
-            d[(r0 + 8) * p.r + t * 8 + c0 + 1] += acc[t][3];
-          }
-      }
-      named_bar_sync(3, kActThreads);
-      // this CTA's partial [16][r] -> split 0's receive area, slot `split`
-      const uint32_t dst0 = dsmem_map(base + S_::kXRecv, 0u);
-      for (int idx = tid; idx < kBN * p.r; idx += kActThreads) {
-        const float s4 = (red[idx] + red[kBN * p.r + idx]) + (red[2 * kBN * p.r + idx] + red[3 * kBN * p.r + idx]);
-        dsmem_st_f32(dst0 + (uint32_t)((split * kBN * p.r + idx) * 4), s4);
-      }
-    }
-
-    cluster_arrive_release();  // B1: absmax and X L1 partials delivered
+    if (lane < S)
+      dsmem_st_f32(dsmem_map(amax_all + (uint32_t)((split * kBN + warp) * 4), (uint32_t)lane), amax);
+    cluster_arrive_release();  // B1: this CTA's absmax partials delivered
     cluster_wait_acquire();
 
-    // ---- token absmax, then the codes of this slice as int8 B operand
-    if (tid < kBN) {
-      float m = 0.f;
-      for (int c = 0; c < S; ++c) m = fmaxf(m, amax_all[c * kBN + tid]);
-      amax_row[tid] = m;
-    }
-    named_bar_sync(3, kActThreads);
+    // ---- codes of token `warp` as the int8 B operand (16 * code: the code's
+    //      low nibble in the high nibble)
+    {
+      float am = 0.f;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int row = warp + 8 * t;
-      const float am = amax_row[row];
-      const float inv = am > 0.f ? 7.f / am : 0.f;
+      for (int z = 0; z < kMaxSplits; ++z)
+        if (z < S) am = fmaxf(am, ld_shared_f32(amax_all + (uint32_t)((z * kBN + warp) * 4)));
+      if (lane == 0) st_shared_f32(amax_row + (uint32_t)(warp * 4), am);
+      const CodeScale cs = code_scale(am);
 #pragma unroll
       for (int ps = 0; ps < 2; ++ps) {
         if (ps < np) {
-          // this lane's 16 codes = one 16-byte chunk of the operand row
+          if (cs.pre != 1.f) {
+#pragma unroll
+            for (int i = 0; i < kE; ++i) v[ps][i] *= cs.pre;
+          }
           uint32_t w4[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t wv = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              wv |= ((uint32_t)(quant_code(v[t][ps][4 * q + j], inv) << 4) & 0xFFu) << (8 * j);
-            w4[q] = wv;
-          }
+          for (int q = 0; q < 4; ++q)
+            w4[q] = (low_bytes4(code_bits(v[ps][4 * q], cs.inv), code_bits(v[ps][4 * q + 1], cs.inv),
+                                code_bits(v[ps][4 * q + 2], cs.inv), code_bits(v[ps][4 * q + 3], cs.inv))
+                     << 4) &
+                    0xF0F0F0F0u;
           const int col = ps * kW + lane * kE;  // within the slice
           const int kb = col / kKB, j = (col % kKB) / 16;
-          st_shared_v4(base + S_::kBBase + (uint32_t)(kb * kBN * 128) + sw_off((uint32_t)row, (uint32_t)j),
+          st_shared_v4(base + S_::kBBase + (uint32_t)(kb * kBN * 128) + sw_off((uint32_t)warp, (uint32_t)j),
                        make_uint4(w4[0], w4[1], w4[2], w4[3]));
         }
       }
@@ -401,20 +345,57 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
     mbar_arrive(b_ready);
 
+    // ---- X L1 partial over the slice, off the path to the integer MMAs:
+    //      A fragments from the staged X (tokens x 16 columns), B from the
+    //      registers
+    const uint32_t part = base + S_::kKRecv;  // [KP][16][r] fp32
+    if (xl1_warp) {
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int i = 0; i < kMaxBPair; ++i) {
+        if (2 * i < kspp) {
+          const uint32_t q = (uint32_t)(4 * (kp * kspp / 2 + i) + c);  // 16-byte chunk of the slice
+          const uint4 x0 = ld_shared_v4(xbase + x_off((uint32_t)g, q));
+          const uint4 x8 = ld_shared_v4(xbase + x_off((uint32_t)(g + 8), q));
+          const uint32_t a0[4] = {x0.x, x8.x, x0.y, x8.y}, b0[2] = {bq[i].x, bq[i].y};
+          const uint32_t a1[4] = {x0.z, x8.z, x0.w, x8.w}, b1[2] = {bq[i].z, bq[i].w};
+          mma_16816(acc[0], a0, b0);
+          mma_16816(acc[1], a1, b1);
+        }
+      }
+      // C fragment: tokens g and g + 8, columns nt*8 + 2c, +1
+      const uint32_t d0 = part + (uint32_t)(((kp * kBN + g) * p.r + nt * 8 + 2 * c) * 4);
+      const uint32_t d1 = d0 + (uint32_t)(8 * p.r * 4);
+      st_shared_f32(d0, acc[0][0] + acc[1][0]);
+      st_shared_f32(d0 + 4, acc[0][1] + acc[1][1]);
+      st_shared_f32(d1, acc[0][2] + acc[1][2]);
+      st_shared_f32(d1 + 4, acc[0][3] + acc[1][3]);
+    }
+    named_bar_sync(1, kActThreads);
+    // k-parts summed in order; this CTA's partial [16][r] -> split 0's
+    // receive area, slot `split`
+    if (ntiles > 0 && tid < kBN * p.r) {
+      float s = 0.f;
+      for (int k = 0; k < KP; ++k) s += ld_shared_f32(part + (uint32_t)((k * kBN * p.r + tid) * 4));
+      dsmem_st_f32(dsmem_map(base + S_::kXRecv + (uint32_t)((split * kBN * p.r + tid) * 4), 0u), s);
+    }
+    cluster_arrive_release();  // B2: this CTA's X L1 partial delivered
+    cluster_wait_acquire();
+
     // ---- split 0: X L1 = sum of the splits' partials (split order), bf16
-    //      into the low-rank B operand
+    //      into the low-rank B operand [16][64] (columns past r are zero)
     if (do_lr) {
-      const uint32_t xr = base + S_::kXRecv;
-      for (int c = tid; c < kBN * 8; c += kActThreads) {  // 16 rows x 8 chunks
-        const int row = c >> 3, j = c & 7;
+      if (tid < kBN * 8) {
+        const int row = tid >> 3, j = tid & 7;
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = 0.f;
         if (j * 8 < p.r) {
+          const uint32_t xr = base + S_::kXRecv + (uint32_t)((row * p.r + j * 8) * 4);
           for (int z = 0; z < S; ++z)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              f[e] += ld_shared_f32(xr + (uint32_t)(((z * kBN + row) * p.r + j * 8 + e) * 4));
+              f[e] += ld_shared_f32(xr + (uint32_t)((z * kBN * p.r + e) * 4));
         }
         st_shared_v4(base + S_::kLrBBase + sw_off((uint32_t)row, (uint32_t)j),
                      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
@@ -426,9 +407,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < kActWarps + kConvWarps) {
     // ==================================================== weight converters
     const int tid = threadIdx.x - kActThreads;  // 0..127
+    // split 0: the tile's L2^T row `tid` ([r] bf16, r <= 32: 4 chunks),
+    // fetched now and placed once its operand slot is free
+    uint4 l2row[kMaxR / 8];
+    // the scale of channel `tid`, for the epilogue (stored after the loop, so
+    // that no thread waits on this load early)
+    const float sw = (tile * kBM + tid < p.N) ? __ldg(p.s_w + tile * kBM + tid) : 0.f;
+#pragma unroll
+    for (int j = 0; j < kMaxR / 8; ++j) {
+      l2row[j] = make_uint4(0u, 0u, 0u, 0u);
+      const int gn = tile * kBM + tid;
+      if (do_lr && gn < p.N && j * 8 < p.r)
+        l2row[j] = __ldg(reinterpret_cast<const uint4*>(p.L2t + (size_t)gn * p.r + j * 8));
+    }
     cluster_wait_acquire();    // B0
     cluster_arrive_release();  // B1 (nothing to publish from these warps)
-    bool alive = true;
+    bool alive = true, b1_done = false;
     for (int st = 0; st < n_st && alive; ++st) {
       const int sg_slot = st % kNSTG;
       if (!mbar_wait(&stg_full[sg_slot], (uint32_t)(st / kNSTG) & 1u, p.status, abort_flag)) break;
@@ -436,33 +430,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t sg = base + S_::kStgBase + sg_slot * S_::kStg;
       for (int sub = 0; sub < nsub; ++sub) {
         const int i = st * kKBS + sub;
+        if (i == kNOPS && !b1_done) {  // slots reused from here on: meet B1/B2 first
+          cluster_wait_acquire();
+          cluster_arrive_release();
+          b1_done = true;
+        }
         if (!mbar_wait(&op_empty[i % kNOPS], ((uint32_t)(i / kNOPS) & 1u) ^ 1u, p.status,
                        abort_flag)) {
           alive = false;
           break;
         }
-        const uint32_t dst0 = base + S_::kOpBase + (uint32_t)(i % kNOPS) * S_::kOp;
-        for (int row = tid; row < kBM; row += kConvThreads) {
-          const uint32_t x7 = (uint32_t)row & 7u;
-          const uint32_t src = sg + (uint32_t)row * 128u;
-          uint4 w[4];
+        const uint32_t dst = base + S_::kOpBase + (uint32_t)(i % kNOPS) * S_::kOp + (uint32_t)tid * 128u;
+        const uint32_t x7 = (uint32_t)tid & 7u;
+        const uint32_t src = sg + (uint32_t)tid * 128u;
+        uint4 w[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(sub * 4 + q) ^ x7) << 4));
-          const uint32_t dst = dst0 + (uint32_t)row * 128u;
+        for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(sub * 4 + q) ^ x7) << 4));
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 lo, hi;
-            lo.x = (w[q].x << 4) & 0xF0F0F0F0u;
-            lo.y = (w[q].y << 4) & 0xF0F0F0F0u;
-            lo.z = (w[q].z << 4) & 0xF0F0F0F0u;
-            lo.w = (w[q].w << 4) & 0xF0F0F0F0u;
-            hi.x = w[q].x & 0xF0F0F0F0u;
-            hi.y = w[q].y & 0xF0F0F0F0u;
-            hi.z = w[q].z & 0xF0F0F0F0u;
-            hi.w = w[q].w & 0xF0F0F0F0u;
-            st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
-            st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
-          }
+        for (int q = 0; q < 4; ++q) {
+          uint4 lo, hi;
+          lo.x = (w[q].x << 4) & 0xF0F0F0F0u;
+          lo.y = (w[q].y << 4) & 0xF0F0F0F0u;
+          lo.z = (w[q].z << 4) & 0xF0F0F0F0u;
+          lo.w = (w[q].w << 4) & 0xF0F0F0F0u;
+          hi.x = w[q].x & 0xF0F0F0F0u;
+          hi.y = w[q].y & 0xF0F0F0F0u;
+          hi.z = w[q].z & 0xF0F0F0F0u;
+          hi.w = w[q].w & 0xF0F0F0F0u;
+          st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
+          st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
         }
         fence_proxy_async_smem();
         mbar_arrive(&op_full[i % kNOPS]);
@@ -470,25 +466,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!alive) break;
       mbar_arrive(&stg_empty[sg_slot]);
     }
-    // split 0: the tile's L2^T rows [128][r] bf16 -> the next operand slot,
-    // the A operand of the low-rank MMA
+    if (!b1_done) {
+      cluster_wait_acquire();    // B1
+      cluster_arrive_release();  // B2
+    }
+    // split 0: L2^T rows -> operand slot n_kb % kNOPS, the low-rank A operand
     if (alive && do_lr) {
       const int i = n_kb;
       if (mbar_wait(&op_empty[i % kNOPS], ((uint32_t)(i / kNOPS) & 1u) ^ 1u, p.status, abort_flag)) {
         const uint32_t dst0 = base + S_::kOpBase + (uint32_t)(i % kNOPS) * S_::kOp;
-        for (int c = tid; c < kBM * 8; c += kConvThreads) {
-          const int row = c >> 3, j = c & 7;
-          const int g = tile * kBM + row;
-          uint4 val = make_uint4(0u, 0u, 0u, 0u);
-          if (g < p.N && j * 8 < p.r)
-            val = __ldg(reinterpret_cast<const uint4*>(p.L2t + (size_t)g * p.r + j * 8));
-          st_shared_v4(dst0 + sw_off((uint32_t)row, (uint32_t)j), val);
-        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          st_shared_v4(dst0 + sw_off((uint32_t)tid, (uint32_t)j),
+                       j < kMaxR / 8 ? l2row[j] : make_uint4(0u, 0u, 0u, 0u));
         fence_proxy_async_smem();
       }
     }
     if (p.r > 0) mbar_arrive(lr_ready);
-    cluster_wait_acquire();
+    sw_tile[tid] = sw;         // read by the epilogue after B3
+    cluster_wait_acquire();  // B2
   } else if (warp == kProducerWarp) {
     // =========================================================== producer
     cluster_wait_acquire();    // B0
@@ -504,11 +500,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     }
+    cluster_wait_acquire();    // B1
+    cluster_arrive_release();  // B2
     cluster_wait_acquire();
   } else {
     // ========================================================== MMA issuer
     cluster_wait_acquire();    // B0
     cluster_arrive_release();  // B1
+    cluster_wait_acquire();
+    cluster_arrive_release();  // B2
     const uint32_t id_i8 = idesc_i8_s32(kBN);
     const uint32_t id_bf = idesc_bf16_f32(kBN);
     bool alive = mbar_wait(b_ready, 0u, p.status, abort_flag);
@@ -541,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) mma_commit(acc_full);
     __syncwarp();
-    cluster_wait_acquire();
+    cluster_wait_acquire();  // B2
   }
 
   // ------------------------------------------------------------- epilogue
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   }
-  cluster_sync();  // B2: every split's partial rows delivered
+  cluster_sync();  // B3: every split's partial rows delivered
   if (is_epi && !*abort_flag) {
     const int lo_m = owned_lo(split, S);
     const int rows_m = owned_lo(split + 1, S) - lo_m;
@@ -588,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int acc = 0;
 #pragma unroll
       for (int z = 0; z < kMaxSplits; ++z) acc += part[z];  // split order
-      const float s_x = amax_row[col] * p.scale_mul;
+      const float s_x = ld_shared_f32(amax_row + (uint32_t)(col * 4)) * p.scale_mul;
       p.Y[(size_t)col * p.N + g_n] = __float2bfloat16_rn(s_x * sw_tile[lo_m + rr] * (float)acc + lr);
     }
   }

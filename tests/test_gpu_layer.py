@@ -18,20 +18,21 @@ def tq(cuda_ok):
 
 
 CASES = [
-    # name, M, K, N, r, b      (fused: M<=16, r<=64, K%512==0, K<=8192)
+    # name, M, K, N, r, b      (fused: M<=16, r<=64, K%512==0, K<=4096)
     ("decode_m1", 1, 4096, 4096, 32, 128),
     ("decode_m3", 3, 4096, 4096, 32, 128),
     ("decode_m16", 16, 4096, 4096, 32, 128),
     ("one_split", 16, 512, 256, 16, 128),
     ("ragged_splits", 5, 1536, 136, 16, 128),
     ("rank0", 7, 2048, 264, 0, 128),
-    ("rank64_block256", 16, 8192, 512, 64, 256),
+    ("rank64_block256", 16, 4096, 512, 64, 256),
     ("no_rotation", 2, 1024, 128, 32, 1),
     ("block2", 9, 1024, 384, 48, 2),
     # two-kernel path inside the same entry point
     ("fallback_m17", 17, 1024, 256, 32, 128),
     ("fallback_rank128", 8, 1024, 256, 128, 128),
     ("fallback_k384", 4, 384, 136, 16, 128),
+    ("fallback_k8192", 16, 8192, 512, 64, 256),
 ]
 
 
@@ -52,6 +53,21 @@ def test_layer_entry_matches_oracle_and_two_call_path(tq, name, M, K, N, r, b):
     a, c = y_one.double().cpu().numpy(), y_two.double().cpu().numpy()
     tol = 2.0 ** -7 * np.abs(c) + 1e-3 * np.abs(c).max()
     assert np.all(np.abs(a - c) <= tol), f"{name}: {np.abs(a - c).max()}"
+
+
+def test_layer_entry_tiny_row(tq):
+    sh = synth.CONFIGS["decode"].with_(M=4, K=1024, N=256, r=32)
+    L = synth.make_layer(sh)
+    L["X"][1] = (L["X"][1].float() * 2.0 ** -110).to(torch.bfloat16)  # absmax ~1e-31
+    X, Rt, L1t, L2t = (L[k].cuda() for k in ("X", "Rt", "L1t", "L2t"))
+    Wq, s_w = tq.tq_pack_weight(Rt, 128)
+    y = tq.tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, 128)
+    torch.cuda.synchronize()
+    o = oracle.layer(L["X"], L["L1t"], L["L2t"], L["Rt"], 128)
+    check_y(y.double().cpu().numpy(), o["Y64"], "tiny row")
+    # the tiny row on its own scale
+    y1, o1 = y[1].double().cpu().numpy(), o["Y64"][1]
+    assert np.linalg.norm(y1 - o1) <= 2e-3 * np.linalg.norm(o1)
 
 
 def test_layer_entry_deterministic(tq):

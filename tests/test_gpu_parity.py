@@ -142,6 +142,21 @@ def test_zero_rows_and_channels(tq):
     _check_layer(g, L, 128)
 
 
+def test_tiny_rows(tq):
+    # rows whose absmax is far below 1 (down to ~1e-36): 7 / absmax would
+    # overflow fp32 without the kernel's exact power-of-two prescale
+    sh = synth.CONFIGS["decode"].with_(M=12, K=512, N=128, r=16)
+    L = synth.make_layer(sh)
+    L["X"][2] = (L["X"][2].float() * 2.0 ** -120).to(torch.bfloat16)
+    L["X"][7] = (L["X"][7].float() * 2.0 ** -60).to(torch.bfloat16)
+    assert L["X"][2].abs().max() > 0
+    g = _run_layer(tq, L, 128)
+    o = oracle.layer(L["X"], L["L1t"], L["L2t"], L["Rt"], 128)
+    check_codes(g["Xq"].numpy(), o["qx"], o["t_x"], "activation codes")
+    check_scales(g["s_x"].numpy(), o["s_x"], "s_x")
+    assert g["Xq"][2].any() and g["Xq"][7].any()
+
+
 def test_deterministic(tq):
     sh = synth.CONFIGS["decode"].with_(M=16, K=1024, N=512, r=32)
     L = synth.make_layer(sh)
