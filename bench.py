@@ -418,6 +418,8 @@ def run_prefill(args, rank, world, local_rank, dist):
     torch.cuda.synchronize()
 
     def one(lay, ev=None):
+        if ev is not None:
+            ev[2].record()
         tq.tq_quantize_act(lay["X"], b, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
         if ev is not None:
             ev[0].record()
@@ -433,17 +435,19 @@ def run_prefill(args, rank, world, local_rank, dist):
         t = torch.tensor([ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         ms = float(t.item())
-    evs = [(torch.cuda.Event(enable_timing=True, external=True),
-            torch.cuda.Event(enable_timing=True, external=True)) for _ in layers]
+    evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
+           for _ in layers]
     g_ev = capture(torch, lambda: [one(l, e) for l, e in zip(layers, evs)])
-    gemm_ms = []
+    gemm_ms, act_ms = [], []
     for _ in range(3):
         g_ev.replay()
     for _ in range(max(1, min(args.steps, 20))):
         g_ev.replay()
         torch.cuda.synchronize()
-        gemm_ms.extend(a.elapsed_time(bb) for a, bb in evs)
+        gemm_ms.extend(e[0].elapsed_time(e[1]) for e in evs)
+        act_ms.extend(e[2].elapsed_time(e[0]) for e in evs)
     gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
+    act_ms_avg = sum(act_ms) / len(act_ms)
     ops = 2 * M * N * K
     peak, src = int8_peak(sustained=False)
     achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
@@ -462,6 +466,7 @@ def run_prefill(args, rank, world, local_rank, dist):
                      "unit": "TOPS", "frac": round(achieved / peak, 4), "traffic": None,
                      "kernel": "w4a4_lr_gemm_kernel (prefill tiling)",
                      "gemm_us": round(gemm_ms_avg * 1e3, 2), "peak_source": src,
+                     "act_us": round(act_ms_avg * 1e3, 2),
                      "lowrank_flops_per_launch": 2 * M * r * (K + N)},
         "gpu_launches": 2 * L * args.steps,
         "clocks": clk.summary(),

@@ -1,0 +1,436 @@
+// tq_act_tc.cu -- the activation stage for many tokens on 5th-generation
+// tensor cores.
+//
+// For a tile of 128 tokens the rotation of one 128-column block of X is a
+// dense product with the block-diagonal Sylvester matrix,
+//
+//   Xh[t][j] = sum_k X[t][k] Hd[k][j],   Hd = diag(H_b, ..., H_b) (b <= 128),
+//
+// so it runs as tcgen05.mma kind::f16 (bf16 X, +-1 entries, fp32 TMEM
+// accumulator) instead of warp shuffles, whose throughput bounds the
+// butterfly kernel when M is large.  The products are exact; only the fp32
+// summation order differs from the butterflies.  X.L1 is a second MMA on the
+// same staged X tiles.  A cluster of C CTAs splits K:
+//
+//   pass 1  rotation of each block -> TMEM -> per-token partial absmax,
+//           pushed to every CTA of the cluster (distributed shared memory)
+//   pass 2  X tiles again (now from L2), rotation -> codes, packed into the
+//           ABI layout and stored; X.L1 accumulated in TMEM over the slice
+//   then    X.L1 partials pushed to the owner CTA of each column, summed in
+//           cluster-rank order (deterministic) and stored.
+//
+// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-5:
+// TMEM readers (warp w reads lanes 32*(w%4)..: token rows of the tile).
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "tq_act_common.cuh"
+#include "tq_internal.h"
+#include "tq_ptx.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kTok = 128;          // tokens per tile (MMA M)
+constexpr int kBlk = 128;          // columns per block (MMA N of the rotation, MMA K)
+constexpr int kNS = 2;             // X / L1^T stages
+constexpr int kMaxC = 8;           // CTAs per cluster along K
+constexpr int kMaxRtc = 128;       // X L1 width handled here
+constexpr int kThreadsTc = 192;
+constexpr int kEpiFirstWarp = 2;
+constexpr int kEpiThreadsTc = 128;
+
+struct TcParams {
+  uint8_t* Xq;       // [M][K/2]
+  float* s_x;        // [M]
+  float* XL1;        // [M][r]
+  int M, K, b, r;
+  int kb_total, nb;  // 128-column blocks in K, blocks per CTA
+  float scale_mul;   // 1 / (7 sqrt(b))
+};
+
+// Shared memory (offsets from the 1024-aligned base).  Atoms are 128-byte
+// swizzled K-major tiles of 64 bf16 columns.
+struct TcSmem {
+  static constexpr uint32_t kH = 0;                         // Hd^T: 2 atoms x 128 rows
+  static constexpr uint32_t kHBytes = 2 * kBlk * 128;
+  static constexpr uint32_t kStage0 = kH + kHBytes;
+  static constexpr uint32_t kXBytes = 2 * kTok * 128;       // X block: 2 atoms x 128 rows
+  static constexpr uint32_t kL1Max = 2 * kMaxRtc * 128;     // L1^T block: 2 atoms x r rows
+  static constexpr uint32_t kStage = kXBytes + kL1Max;
+  static constexpr uint32_t kAmax = kStage0 + kNS * kStage; // [C][128] fp32
+  static constexpr uint32_t kBar = kAmax + kMaxC * kTok * 4;
+  // full[kNS], empty[kNS], rot_full[2], rot_empty[2], xl1_full
+  static constexpr uint32_t kNumBars = 2 * kNS + 5;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+static_assert(TcSmem::kAlloc <= 227 * 1024, "activation tile shared memory");
+// the X L1 receive area [C][128][ceil(r/C)] reuses the stages after pass 2
+static_assert(kTok * (kMaxRtc + kMaxC) * 4 <= kNS * TcSmem::kStage, "X L1 receive area");
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void st_shared_v4_tc(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ float ld_shared_f32_tc(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ void cluster_arrive_rel() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+// 16-byte chunk c (0..15) of row `row` of a two-atom (128 bf16 columns) tile
+// with `rows` rows per atom.
+__device__ __forceinline__ uint32_t atom_off(uint32_t row, uint32_t c, uint32_t rows) {
+  return (c >> 3) * rows * 128u + row * 128u + (((c & 7u) ^ (row & 7u)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreadsTc, 1)
+    quantize_act_tc_kernel(const __grid_constant__ CUtensorMap map_x,
+                           const __grid_constant__ CUtensorMap map_l1, const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  using L = TcSmem;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kNS;
+  uint64_t* rot_full = bars + 2 * kNS;
+  uint64_t* rot_empty = rot_full + 2;
+  uint64_t* xl1_full = rot_full + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();
+  const uint32_t csize = cluster_nctarank();
+  const int tile = blockIdx.y;
+  const int kb0 = (int)crank * p.nb;
+  const int nb = max(0, min(p.nb, p.kb_total - kb0));  // blocks of this CTA
+  const int r = p.r;
+  const uint32_t l1_bytes = (uint32_t)r * 256u;         // one L1^T block, 2 atoms
+
+  // ---------------------------------------------------------------- prologue
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&rot_full[i], 1);
+      mbar_init(&rot_empty[i], kEpiThreadsTc);
+    }
+    mbar_init(xl1_full, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_x);
+    if (r > 0) tma_prefetch_desc(&map_l1);
+  }
+  // Hd^T as the B operand of the rotation: row j (output column), column k;
+  // Hd is symmetric.  +-1 (or 0 off the diagonal blocks), unnormalised.
+  for (int ch = threadIdx.x; ch < kBlk * 16; ch += kThreadsTc) {
+    const int j = ch >> 4, c = ch & 15;
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t two = 0;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int k = c * 8 + 2 * e + h;
+        uint32_t bits = 0;  // bf16 0
+        if ((j / p.b) == (k / p.b))
+          bits = (__popc((unsigned)(j & k & (p.b - 1))) & 1) ? 0xBF80u : 0x3F80u;
+        two |= bits << (16 * h);
+      }
+      w[e] = two;
+    }
+    st_shared_v4_tc(base + L::kH + atom_off((uint32_t)j, (uint32_t)c, kBlk),
+                    make_uint4(w[0], w[1], w[2], w[3]));
+  }
+  fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  cluster_arrive_relaxed();  // B0: this CTA is running
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_rot = tmem;        // 2 x 128 columns
+  const uint32_t tmem_xl1 = tmem + 256;  // r columns
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    // ======================================================== TMA producer
+    cluster_wait_acquire();    // B0
+    cluster_arrive_rel();      // B1 (nothing to publish)
+    if (lane == 0) {
+      pdl_wait();  // X comes from the preceding kernel
+      const uint64_t pol_x = policy_evict_last();    // read again in pass 2
+      const uint64_t pol_w = policy_evict_first();
+      for (int i = 0; i < 2 * nb; ++i) {
+        const int s = i % kNS;
+        const bool second = i >= nb;
+        const int j = second ? i - nb : i;
+        if (!mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, nullptr, abort_flag)) break;
+        const uint32_t st = base + L::kStage0 + (uint32_t)s * L::kStage;
+        const bool with_l1 = second && r > 0;
+        mbar_arrive_expect_tx(&full[s], L::kXBytes + (with_l1 ? l1_bytes : 0u));
+        const int x = (kb0 + j) * kBlk;
+        tma_load_2d(smem + (st - base), &map_x, &full[s], x, tile * kTok, pol_x);
+        tma_load_2d(smem + (st - base) + kTok * 128, &map_x, &full[s], x + 64, tile * kTok, pol_x);
+        if (with_l1) {
+          tma_load_2d(smem + (st - base) + L::kXBytes, &map_l1, &full[s], x, 0, pol_w);
+          tma_load_2d(smem + (st - base) + L::kXBytes + (uint32_t)r * 128u, &map_l1, &full[s],
+                      x + 64, 0, pol_w);
+        }
+      }
+    }
+    __syncwarp();
+    cluster_wait_acquire();    // B1
+    cluster_arrive_rel();      // B2
+    cluster_wait_acquire();
+    cluster_arrive_rel();      // B3
+    cluster_wait_acquire();
+  } else if (warp == 1) {
+    // ========================================================== MMA issuer
+    cluster_wait_acquire();    // B0
+    cluster_arrive_rel();      // B1
+    const uint32_t id_rot = idesc_bf16_f32(kBlk);
+    const uint32_t id_xl1 = idesc_bf16_f32(r > 0 ? r : 16);
+    for (int i = 0; i < 2 * nb; ++i) {
+      const int s = i % kNS, u = i & 1;
+      const bool second = i >= nb;
+      const int j = second ? i - nb : i;
+      if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, nullptr, abort_flag)) break;
+      if (!mbar_wait(&rot_empty[u], ((uint32_t)(i / 2) & 1u) ^ 1u, nullptr, abort_flag)) break;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t st = base + L::kStage0 + (uint32_t)s * L::kStage;
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const uint32_t atom = (uint32_t)kk >> 2, ko = ((uint32_t)kk & 3u) * 2u;  // 32 B steps
+          const uint64_t da = sdesc_sw128(st + atom * (kTok * 128u)) + ko;
+          const uint64_t dh = sdesc_sw128(base + L::kH + atom * (kBlk * 128u)) + ko;
+          mma_bf16(tmem_rot + (uint32_t)u * kBlk, da, dh, id_rot, kk > 0 ? 1u : 0u);
+          if (second && r > 0) {
+            const uint64_t dl = sdesc_sw128(st + L::kXBytes + atom * ((uint32_t)r * 128u)) + ko;
+            mma_bf16(tmem_xl1, da, dl, id_xl1, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(&empty[s]);
+        mma_commit(&rot_full[u]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0 && r > 0) mma_commit(xl1_full);
+    __syncwarp();
+    cluster_wait_acquire();    // B1
+    cluster_arrive_rel();      // B2
+    cluster_wait_acquire();
+    cluster_arrive_rel();      // B3
+    cluster_wait_acquire();
+  } else {
+    // ===================================================== TMEM readers
+    const int q = warp & 3;                       // TMEM lane quarter
+    const int row = q * 32 + lane;                // token row in the tile
+    const int grow = tile * kTok + row;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    cluster_wait_acquire();  // B0: peers are running before they are written to
+
+    // ---- pass 1: partial absmax of this token over the CTA's slice
+    float amax = 0.f;
+    for (int i = 0; i < nb; ++i) {
+      const int u = i & 1;
+      const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
+                                                  abort_flag));
+      tc_fence_after();
+      if (ok) {
+#pragma unroll
+        for (int g = 0; g < kBlk / 32; ++g) {
+          uint32_t v[32];
+          tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(v[e])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&rot_empty[u]);
+    }
+    for (uint32_t z = 0; z < csize; ++z)
+      dsmem_st_f32(dsmem_map(base + L::kAmax + (crank * kTok + (uint32_t)row) * 4u, z), amax);
+    cluster_arrive_rel();  // B1: partial absmax delivered
+    cluster_wait_acquire();
+    float am = 0.f;
+    for (uint32_t z = 0; z < csize; ++z)
+      am = fmaxf(am, ld_shared_f32_tc(base + L::kAmax + (z * kTok + (uint32_t)row) * 4u));
+    if (crank == 0 && grow < p.M) p.s_x[grow] = am * p.scale_mul;
+    const CodeScale cs = code_scale(am);
+
+    // ---- pass 2: the same rotation again -> codes in the packed layout
+    //      (inside each 32-code group byte i = code i | code i+16 << 4)
+    for (int i = nb; i < 2 * nb; ++i) {
+      const int u = i & 1;
+      const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
+                                                  abort_flag));
+      tc_fence_after();
+      if (ok) {
+        uint8_t* dst = p.Xq + (size_t)grow * (size_t)(p.K / 2) + (size_t)(kb0 + i - nb) * 64;
+#pragma unroll
+        for (int g = 0; g < kBlk / 32; ++g) {
+          uint32_t v[32];
+          tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
+          tmem_ld_wait();
+          uint32_t cb[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float f = __uint_as_float(v[e]);
+            if (cs.pre != 1.f) f *= cs.pre;
+            cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
+          }
+          uint32_t w[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h)
+            w[h] = (low_bytes4(cb[4 * h], cb[4 * h + 1], cb[4 * h + 2], cb[4 * h + 3]) & 0x0F0F0F0Fu) |
+                   ((low_bytes4(cb[16 + 4 * h], cb[17 + 4 * h], cb[18 + 4 * h], cb[19 + 4 * h])
+                     << 4) & 0xF0F0F0F0u);
+          if (grow < p.M) *reinterpret_cast<uint4*>(dst + 16 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&rot_empty[u]);
+    }
+
+    // ---- X L1: partial over the slice -> the column's owner CTA
+    bool xl1_ok = true;
+    if (r > 0) xl1_ok = __all_sync(kFull, mbar_wait(xl1_full, 0u, nullptr, abort_flag));
+    cluster_arrive_rel();  // B2: every CTA is past pass 2 (stages free)
+    cluster_wait_acquire();
+    const int cols_max = r > 0 ? (r + (int)csize - 1) / (int)csize : 0;
+    const uint32_t recv = base + L::kStage0;  // [C][128][cols_max] fp32
+    if (r > 0 && xl1_ok) {
+      tc_fence_after();
+      for (int c0 = 0; c0 < r; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_xl1 + (uint32_t)c0 + lane_off, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int col = c0 + e;
+          const int owner = col * (int)csize / r;
+          const int lo = (owner * r + (int)csize - 1) / (int)csize;
+          dsmem_st_f32(dsmem_map(recv + (uint32_t)(((int)crank * kTok + row) * cols_max + col - lo) * 4u,
+                                 (uint32_t)owner),
+                       __uint_as_float(v[e]));
+        }
+      }
+    }
+    cluster_arrive_rel();  // B3: partials delivered
+    cluster_wait_acquire();
+    if (r > 0 && grow < p.M && !*abort_flag) {
+      const int lo = ((int)crank * r + (int)csize - 1) / (int)csize;
+      const int hi = (((int)crank + 1) * r + (int)csize - 1) / (int)csize;
+      for (int cc = 0; cc < hi - lo; ++cc) {
+        float s = 0.f;
+        for (uint32_t z = 0; z < csize; ++z)
+          s += ld_shared_f32_tc(recv + (uint32_t)(((int)z * kTok + row) * cols_max + cc) * 4u);
+        p.XL1[(size_t)grow * r + lo + cc] = s;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool act_tc_supported(int M, int K, int had_block, int r) {
+  (void)K;
+  return M >= 64 && had_block <= kBlk && r <= kMaxRtc;
+}
+
+cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
+                          int r, uint8_t* Xq, float* s_x, float* XL1, cudaStream_t stream) {
+  TcParams p{};
+  p.Xq = Xq;
+  p.s_x = s_x;
+  p.XL1 = XL1;
+  p.M = M;
+  p.K = K;
+  p.b = had_block;
+  p.r = r;
+  p.kb_total = K / kBlk;
+  p.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  const int tiles = (M + kTok - 1) / kTok;
+  // a cluster of C CTAs along K per 128-token tile, about one CTA per SM
+  int C = std::max(1, std::min(kMaxC, num_sms() / tiles));
+  C = std::min(C, p.kb_total);
+  p.nb = (p.kb_total + C - 1) / C;
+  C = (p.kb_total + p.nb - 1) / p.nb;  // every CTA owns at least one block
+  CUtensorMap map_x, map_l1;
+  if (!encode_tiled_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
+                       (uint64_t)K * 2, 64, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (r > 0) {
+    if (!encode_tiled_2d(&map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, (uint64_t)K, (uint64_t)r,
+                         (uint64_t)K * 2, 64, (uint32_t)r, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    map_l1 = map_x;  // never read
+  }
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_set >> dev & 1u)) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)TcSmem::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(C, tiles, 1);
+  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.dynamicSmemBytes = TcSmem::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, quantize_act_tc_kernel, map_x, map_l1, p);
+}
+
+}  // namespace tq

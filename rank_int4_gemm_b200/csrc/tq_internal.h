@@ -21,6 +21,11 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
                                 float* XL1, cudaStream_t stream);
 
+// Activation stage on tensor cores (many tokens): rotation and X L1 as MMAs.
+bool act_tc_supported(int M, int K, int had_block, int r);
+cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
+                          int r, uint8_t* Xq, float* s_x, float* XL1, cudaStream_t stream);
+
 struct GemmArgs {
   const uint8_t* Xq;
   const float* s_x;

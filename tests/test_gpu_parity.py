@@ -62,6 +62,30 @@ SHAPES = [
 ]
 
 
+# tq_quantize_act on tensor cores (M >= 64, b <= 128, r <= 128): 128-token
+# tiles, ragged last tile, one and several CTAs along K, every block size
+TC_SHAPES = [
+    ("tc_min_m", 64, 256, 128, 16, 128),
+    ("tc_ragged", 129, 1024, 136, 32, 128),
+    ("tc_one_block", 200, 128, 64, 16, 128),
+    ("tc_rank0", 300, 512, 264, 0, 128),
+    ("tc_rank128", 140, 2048, 256, 128, 128),
+    ("tc_block2", 96, 512, 128, 48, 2),
+    ("tc_block64", 70, 768, 128, 64, 64),
+    ("tc_no_rotation", 65, 384, 64, 16, 1),
+    ("tc_many_tiles", 1100, 1536, 256, 64, 128),
+]
+
+
+@pytest.mark.parametrize("name,M,K,N,r,b", TC_SHAPES, ids=[s[0] for s in TC_SHAPES])
+def test_activation_tensor_core_path(tq, name, M, K, N, r, b):
+    sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=r, had_block=b)
+    L = synth.make_layer(sh, seed=3)
+    g = _run_layer(tq, L, b)
+    fw, fx, fro, mx = _check_layer(g, L, b)
+    print(f"{name}: flips x={fx:.1e} w={fw:.1e} fro={fro:.2e} max={mx:.2e}")
+
+
 @pytest.mark.parametrize("name,M,K,N,r,b", SHAPES, ids=[s[0] for s in SHAPES])
 def test_layer_small(tq, name, M, K, N, r, b):
     base = synth.CONFIGS["tiny"] if name == "tiny" else synth.CONFIGS["decode"]
