@@ -429,6 +429,10 @@ def run_prefill(args, rank, world, local_rank, dist):
             ev[1].record()
 
     g = capture(torch, lambda: [one(l) for l in layers])
+    if args.profile:
+        time_graph(torch, g, args.steps, args.warmup)
+        return {"profile": f"{args.workload} step graph", "layers": L, "steps": args.steps,
+                "warmup": args.warmup}
     with ClockSampler(local_rank) as clk:
         ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
     if world > 1:

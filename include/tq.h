@@ -138,14 +138,16 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  *   Y = bf16( s_x s_w (Q4(X H) . Wq) + bf16(X L1) L2 )
  *
  * i.e. tq_quantize_act followed by tq_w4a4_lr_gemm, with the same codes,
- * scales and tolerances.  At decode sizes (M <= 16, r <= 64, K % 512 == 0,
- * K <= 8192) it runs as ONE kernel: each split-K cluster rotates and
- * quantizes its own slice of X, exchanges the absmax and X L1 partials in
- * distributed shared memory and feeds the codes straight to the tensor
- * cores, while the weights stream in (TwinQuant notes section 04.C: the
- * residual GEMM quantizes activations concurrently and both paths share one
- * epilogue).  Other shapes run the two kernels, keeping Xq, s_x and XL1 in
- * the workspace.
+ * scales and tolerances.  At decode sizes (M <= 16, r <= 32, K % 512 == 0,
+ * K <= 4096, had_block <= 512) it runs as ONE kernel: each split-K cluster
+ * rotates and quantizes its own slice of X, exchanges the absmax and X L1
+ * partials in distributed shared memory and feeds the codes straight to the
+ * tensor cores, while the weights stream in (TwinQuant notes section 04.C:
+ * the residual GEMM quantizes activations concurrently and both paths share
+ * one epilogue).  For M > 128 with had_block <= 128 and r <= 128 it runs
+ * tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte in the
+ * workspace).  Other shapes run tq_quantize_act + tq_w4a4_lr_gemm, keeping
+ * Xq, s_x and XL1 in the workspace.
  *
  *   X [M][K] bf16, L1t [r][K] bf16 (NULL iff r == 0), Wq [N][K/2] u8,
  *   s_w [N] fp32, L2t [N][r] bf16 (NULL iff r == 0), Y [M][N] bf16 (out)
@@ -159,6 +161,43 @@ TQ_API int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t,
                             int had_block, uint16_t* Y,
                             void* workspace, size_t workspace_bytes,
                             void* stream);
+
+/*
+ * tq_quantize_act_i8 -- tq_quantize_act for many tokens, with the codes one
+ * per byte: the same rotation (CoQuant Eq. (3), block Hadamard), per-token
+ * scale and RoundClip codes (CoQuant Eq. (1)) and the same X L1
+ * (TwinQuant notes section 02.A), written for tq_w4a4_lr_gemm_a8.  tcgen05
+ * has no dense int4 MMA kind, so the GEMM consumes int8 operands; codes in
+ * int8 containers reach it without any unpacking (they are still INT4 values
+ * in [-7, 7]).
+ *
+ *   X    [M][K] bf16    in : activations
+ *   L1t  [r][K] bf16    in : L1^T; NULL iff r == 0
+ *   Xq8  [M][K] s8     out : codes of X H, one per byte, in column order
+ *   s_x  [M] fp32      out : per-token scales
+ *   XL1b [M][r] bf16   out : bf16(X L1) (round to nearest even), the
+ *                            low-rank GEMM operand; NULL iff r == 0
+ * Limits: had_block <= 128, r <= 128 (else TQ_ERR_UNSUPPORTED_SHAPE).
+ */
+TQ_API int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block,
+                              const uint16_t* L1t, int r,
+                              int8_t* Xq8, float* s_x, uint16_t* XL1b, void* stream);
+
+/*
+ * tq_w4a4_lr_gemm_a8 -- tq_w4a4_lr_gemm with the activation codes one per
+ * byte (from tq_quantize_act_i8):
+ *
+ *   Y[m][n] = bf16( s_x[m] s_w[n] sum_k qx[m][k] qw[n][k]
+ *                   + sum_j XL1b[m][j] L2t[n][j] )
+ *
+ * the integer sum exact in INT32.  Same workspace rules as tq_w4a4_lr_gemm
+ * (tq_gemm_workspace_bytes bytes, zeroed before first use).
+ */
+TQ_API int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x,
+                              const uint8_t* Wq, const float* s_w,
+                              const uint16_t* XL1b, const uint16_t* L2t,
+                              int M, int N, int K, int r, uint16_t* Y,
+                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * tq_debug_w4a4_gemm_acc -- test hook: the same GEMM kernel with the

@@ -425,7 +425,7 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores.
   if (act_tc_supported(M, K, had_block, r))
-    return launch_act_tc(X, M, K, had_block, L1t, r, Xq, s_x, XL1, stream);
+    return launch_act_tc(X, M, K, had_block, L1t, r, Xq, nullptr, s_x, XL1, nullptr, stream);
   // Few token groups (decode): spread K over up to 16 CTAs of 256 columns.
   const int groups = (M + kActRows - 1) / kActRows;
   if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);

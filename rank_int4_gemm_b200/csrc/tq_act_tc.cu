@@ -44,9 +44,11 @@ constexpr int kEpiFirstWarp = 2;
 constexpr int kEpiThreadsTc = 128;
 
 struct TcParams {
-  uint8_t* Xq;       // [M][K/2]
+  uint8_t* Xq;       // [M][K/2] packed codes, or null
+  int8_t* Xq8;       // [M][K] one code per byte, or null
   float* s_x;        // [M]
-  float* XL1;        // [M][r]
+  float* XL1;        // [M][r] fp32, or null
+  __nv_bfloat16* XL1b;  // [M][r] rounded to bf16, or null
   int M, K, b, r;
   int kb_total, nb;  // 128-column blocks in K, blocks per CTA
   float scale_mul;   // 1 / (7 sqrt(b))
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
                                                   abort_flag));
       tc_fence_after();
       if (ok) {
-        uint8_t* dst = p.Xq + (size_t)grow * (size_t)(p.K / 2) + (size_t)(kb0 + i - nb) * 64;
+        const size_t blk = (size_t)(kb0 + i - nb);
 #pragma unroll
         for (int g = 0; g < kBlk / 32; ++g) {
           uint32_t v[32];
@@ -313,13 +315,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             if (cs.pre != 1.f) f *= cs.pre;
             cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
           }
-          uint32_t w[4];
+          if (grow < p.M) {
+            if (p.Xq8) {  // one code per byte, in column order
+              uint32_t w[8];
 #pragma unroll
-          for (int h = 0; h < 4; ++h)
-            w[h] = (low_bytes4(cb[4 * h], cb[4 * h + 1], cb[4 * h + 2], cb[4 * h + 3]) & 0x0F0F0F0Fu) |
-                   ((low_bytes4(cb[16 + 4 * h], cb[17 + 4 * h], cb[18 + 4 * h], cb[19 + 4 * h])
-                     << 4) & 0xF0F0F0F0u);
-          if (grow < p.M) *reinterpret_cast<uint4*>(dst + 16 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+              for (int h = 0; h < 8; ++h)
+                w[h] = low_bytes4(cb[4 * h], cb[4 * h + 1], cb[4 * h + 2], cb[4 * h + 3]);
+              int8_t* dst = p.Xq8 + (size_t)grow * (size_t)p.K + blk * kBlk + 32 * g;
+              reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+              uint32_t w[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h)
+                w[h] = (low_bytes4(cb[4 * h], cb[4 * h + 1], cb[4 * h + 2], cb[4 * h + 3]) &
+                        0x0F0F0F0Fu) |
+                       ((low_bytes4(cb[16 + 4 * h], cb[17 + 4 * h], cb[18 + 4 * h], cb[19 + 4 * h])
+                         << 4) &
+                        0xF0F0F0F0u);
+              uint8_t* dst = p.Xq + (size_t)grow * (size_t)(p.K / 2) + blk * 64;
+              *reinterpret_cast<uint4*>(dst + 16 * g) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          }
         }
       }
       tc_fence_before();
@@ -359,7 +376,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
         float s = 0.f;
         for (uint32_t z = 0; z < csize; ++z)
           s += ld_shared_f32_tc(recv + (uint32_t)(((int)z * kTok + row) * cols_max + cc) * 4u);
-        p.XL1[(size_t)grow * r + lo + cc] = s;
+        if (p.XL1) p.XL1[(size_t)grow * r + lo + cc] = s;
+        if (p.XL1b) p.XL1b[(size_t)grow * r + lo + cc] = __float2bfloat16_rn(s);
       }
     }
   }
@@ -380,11 +398,14 @@ bool act_tc_supported(int M, int K, int had_block, int r) {
 }
 
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
-                          int r, uint8_t* Xq, float* s_x, float* XL1, cudaStream_t stream) {
+                          int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
+                          cudaStream_t stream) {
   TcParams p{};
   p.Xq = Xq;
+  p.Xq8 = Xq8;
   p.s_x = s_x;
   p.XL1 = XL1;
+  p.XL1b = reinterpret_cast<__nv_bfloat16*>(XL1b);
   p.M = M;
   p.K = K;
   p.b = had_block;

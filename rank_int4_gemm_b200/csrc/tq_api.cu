@@ -3,6 +3,7 @@
 // (except tq_query_device_status, which exists to synchronise).
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "../../include/tq.h"
@@ -140,12 +141,66 @@ int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq, int M, int N, i
                      workspace, workspace_bytes, stream);
 }
 
-// Layer workspace: [status 256][Xq M*K/2][s_x 4M][XL1 4Mr], 256-aligned parts.
+int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t, int r,
+                       int8_t* Xq8, float* s_x, uint16_t* XL1b, void* stream) {
+  if (!X || !Xq8 || !s_x || M <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (had_block > 128 || r > 128) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1b != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Xq8) || !aligned16(s_x) || (r > 0 && !aligned16(L1t)) ||
+      (r > 0 && !aligned16(XL1b)))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x, nullptr, XL1b,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x, const uint8_t* Wq, const float* s_w,
+                       const uint16_t* XL1b, const uint16_t* L2t, int M, int N, int K, int r,
+                       uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!Xq8 || !s_x || !Wq || !s_w || !Y || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (XL1b != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Xq8) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y) ||
+      (XL1b && !aligned16(XL1b)) || (L2t && !aligned16(L2t)) || (ws && !aligned16(ws)))
+    return TQ_ERR_MISALIGNED;
+  if (!ws || ws_bytes < tq::gemm_workspace_bytes(M, N, K, r)) return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  tq::GemmA8Args a{};
+  a.Xq8 = Xq8;
+  a.s_x = s_x;
+  a.Wq = Wq;
+  a.s_w = s_w;
+  a.XL1b = XL1b;
+  a.L2t = L2t;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.Y = Y;
+  a.ws = ws;
+  return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
+}
+
+// Layer workspace, 256-aligned parts after the 256-byte status word: either
+// [Xq M*K/2][s_x 4M][XL1 4Mr] (packed codes) or [Xq8 M*K][s_x 4M][XL1b 2Mr]
+// (codes one per byte, M > 128).
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static bool layer_uses_a8(int M, int r, int had_block) {
+  return tq::tuning().layer_a8 && M > 128 && had_block <= 128 && r <= 128;
+}
 
 size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {
   if (M <= 0 || N <= 0 || K <= 0 || r < 0) return 256;
-  return 256 + align256((size_t)M * K / 2) + align256((size_t)M * 4) + align256((size_t)M * r * 4);
+  const size_t packed =
+      align256((size_t)M * K / 2) + align256((size_t)M * 4) + align256((size_t)M * r * 4);
+  const size_t bytes8 =
+      align256((size_t)M * K) + align256((size_t)M * 4) + align256((size_t)M * r * 2);
+  return 256 + (M > 128 ? std::max(packed, bytes8) : packed);
 }
 
 int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
@@ -181,6 +236,29 @@ int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, 
     return from_cuda(tq::launch_layer_decode(a, st));
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (layer_uses_a8(M, r, had_block)) {
+    int8_t* Xq8 = reinterpret_cast<int8_t*>(ws + 256);
+    float* s_x8 = reinterpret_cast<float*>(ws + 256 + align256((size_t)M * K));
+    uint16_t* XL1b =
+        reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(s_x8) + align256((size_t)M * 4));
+    if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8, nullptr,
+                                          r > 0 ? XL1b : nullptr, st))
+      return from_cuda(e);
+    tq::GemmA8Args a{};
+    a.Xq8 = Xq8;
+    a.s_x = s_x8;
+    a.Wq = Wq;
+    a.s_w = s_w;
+    a.XL1b = r > 0 ? XL1b : nullptr;
+    a.L2t = L2t;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.r = r;
+    a.Y = Y;
+    a.ws = workspace;
+    return from_cuda(tq::launch_gemm_a8(a, st));
+  }
   uint8_t* Xq = ws + 256;
   float* s_x = reinterpret_cast<float*>(Xq + align256((size_t)M * K / 2));
   float* XL1 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + align256((size_t)M * 4));

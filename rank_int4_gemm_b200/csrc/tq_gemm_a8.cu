@@ -1,0 +1,425 @@
+// tq_gemm_a8.cu -- the W4A4 + low-rank GEMM for many tokens, with the
+// activation codes stored one per byte.
+//
+// tcgen05 has no dense int4 kind, so both operands must reach the tensor core
+// as int8.  Expanding both in shared memory costs more shared-memory
+// bandwidth per k-block than the MMA has cycles (the packed-activation GEMM
+// in tq_gemm.cu is bound by it at large M).  Here:
+//
+//   * the token codes arrive as int8 (tq_quantize_act_i8), so TMA writes them
+//     straight into the MMA's B operand layout (128-byte swizzle, K-major);
+//   * the packed int4 weights are expanded in registers and written to tensor
+//     memory with tcgen05.st: the MMA reads its A operand from TMEM, so the
+//     expanded weights never touch shared memory.  A nibble becomes the byte
+//     16*q, the codes stay q, so the INT32 accumulator holds 16 * sum(qx qw)
+//     exactly (|acc| <= 16*49*K < 2^31); the epilogue shifts it back.
+//
+// Tile: 128 channels (MMA M = TMEM lanes) x 192 tokens (MMA N).  TMEM:
+// INT32 accumulator [192] | two 32-column A buffers | fp32 low-rank [192].
+// Persistent CTAs walk the tiles; a 3-stage TMA ring carries two k-blocks of
+// tokens and weights per stage, then the low-rank chunks (64 columns of
+// bf16(XL1) and L2^T per stage, kind::f16 into the low-rank accumulator).
+//
+// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-5:
+// weight expansion into TMEM, then the epilogue of the tile (warp w owns
+// lanes 32*(w%4)..: channel rows).  No TMA multicast.
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "tq_internal.h"
+#include "tq_ptx.cuh"
+
+namespace tq {
+
+namespace {
+
+constexpr int kCh = 128;           // channels per tile (MMA M)
+constexpr int kTk = 192;           // tokens per tile (MMA N)
+constexpr int kKb = 128;           // codes per k-block
+constexpr int kNS = 3;             // stages
+constexpr int kThreadsA8 = 192;
+constexpr int kConvThreadsA8 = 128;
+constexpr uint32_t kColAcc = 0;    // INT32 accumulator, kTk columns
+constexpr int kNA = 4;             // int8 weight k-blocks in TMEM (A operand buffers)
+constexpr uint32_t kColA = 192;    // kNA x 32 columns: one int8 weight k-block each
+constexpr uint32_t kColLr = 320;   // fp32 low-rank accumulator, kTk columns
+
+struct A8Params {
+  const float* s_x;    // [M]
+  const float* s_w;    // [N]
+  __nv_bfloat16* Y;    // [M][N]
+  uint32_t* status;
+  int M, N, K, r;
+  int kb_total, n_st, n_lr;  // k-blocks, k-block stages, low-rank stages per tile
+  int tiles_m, tiles;        // token tiles, all tiles
+};
+
+// Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
+// [2 k-blocks][192 rows][128 B] then packed weights [128 rows][128 B]
+// (2 k-blocks).  A low-rank stage holds bf16(XL1) [192][64] in the first token
+// sub-tile and L2^T [128][64] in the weight part.
+struct A8Smem {
+  static constexpr uint32_t kTokSub = kTk * 128;            // 24 KB
+  static constexpr uint32_t kWBytes = kCh * 128;            // 16 KB
+  static constexpr uint32_t kStage = 2 * kTokSub + kWBytes;  // 64 KB
+  static constexpr uint32_t kBar = kNS * kStage;
+  // full[kNS], empty[kNS], a_full[kNA], a_empty[kNA], acc_full, acc_empty
+  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNA + 2;
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMisc + 16;
+  static constexpr uint32_t kAlloc = kBytes + 1024;
+};
+static_assert(A8Smem::kAlloc <= 227 * 1024, "a8 GEMM shared memory");
+static_assert(A8Smem::kTokSub % 1024 == 0 && A8Smem::kStage % 1024 == 0, "1024-B aligned atoms");
+
+__device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, signed int8, int32 accumulator.
+__device__ __forceinline__ void mma_i8_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+      "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+      "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+      "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+      "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32_a8(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+        "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+        "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+        "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+        "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+        "=r"(v[31])
+      : "r"(taddr));
+}
+
+__global__ void __launch_bounds__(kThreadsA8, 1)
+    w4a4_lr_gemm_a8_kernel(const __grid_constant__ CUtensorMap map_t,   // tokens int8 [M][K]
+                           const __grid_constant__ CUtensorMap map_w,   // weights [N][K/2]
+                           const __grid_constant__ CUtensorMap map_xb,  // bf16(XL1) [M][r]
+                           const __grid_constant__ CUtensorMap map_l2,  // L2^T [N][r]
+                           const A8Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_addr);
+  using L = A8Smem;
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kNS;
+  uint64_t* a_full = bars + 2 * kNS;
+  uint64_t* a_empty = a_full + kNA;
+  uint64_t* acc_full = a_full + 2 * kNA;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < kNS; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], 1);
+    }
+    for (int i = 0; i < kNA; ++i) {
+      mbar_init(&a_full[i], kConvThreadsA8);
+      mbar_init(&a_empty[i], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kConvThreadsA8);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&map_t);
+    tma_prefetch_desc(&map_w);
+    if (p.r > 0) {
+      tma_prefetch_desc(&map_xb);
+      tma_prefetch_desc(&map_l2);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ======================================================== TMA producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();  // weights: streamed once per token tile
+      const uint64_t pol_t = policy_evict_last();   // tokens: reused by every channel tile
+      bool waited = false;                          // the weights need no predecessor
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
+        const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+        for (int st = 0; st < p.n_st + p.n_lr; ++st, ++it) {
+          const int s = it % kNS;
+          if (!mbar_wait(&empty[s], ((uint32_t)(it / kNS) & 1u) ^ 1u, p.status, abort_flag)) break;
+          uint8_t* sp = smem + (uint32_t)s * L::kStage;
+          if (st < p.n_st) {
+            const int kb = 2 * st;
+            const bool two = kb + 1 < p.kb_total;
+            mbar_arrive_expect_tx(&full[s], L::kWBytes + (two ? 2u : 1u) * L::kTokSub);
+            tma_load_2d(sp + 2 * L::kTokSub, &map_w, &full[s], st * 128, tn * kCh, pol_w);
+            if (!waited) {
+              pdl_wait();  // token codes come from the preceding kernel
+              waited = true;
+            }
+            tma_load_2d(sp, &map_t, &full[s], kb * kKb, tm * kTk, pol_t);
+            if (two) tma_load_2d(sp + L::kTokSub, &map_t, &full[s], (kb + 1) * kKb, tm * kTk, pol_t);
+          } else {
+            const int c = st - p.n_st;  // 64-column low-rank chunk
+            mbar_arrive_expect_tx(&full[s], L::kWBytes + L::kTokSub);
+            if (!waited) {
+              pdl_wait();
+              waited = true;
+            }
+            tma_load_2d(sp + 2 * L::kTokSub, &map_l2, &full[s], c * 64, tn * kCh, pol_w);
+            tma_load_2d(sp, &map_xb, &full[s], c * 64, tm * kTk, pol_t);
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ========================================================== MMA issuer
+    const uint32_t id_i8 = idesc_i8_s32(kTk);
+    const uint32_t id_bf = idesc_bf16_f32(kTk);
+    int it = 0, ab = 0, tcount = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < p.tiles && alive && !*abort_flag;
+         tile += gridDim.x, ++tcount) {
+      // the epilogue has drained the accumulators of the previous tile
+      if (!mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, p.status, abort_flag)) break;
+      tc_fence_after();
+      for (int st = 0; st < p.n_st + p.n_lr && alive; ++st, ++it) {
+        const int s = it % kNS;
+        if (!mbar_wait(&full[s], (uint32_t)(it / kNS) & 1u, p.status, abort_flag)) {
+          alive = false;
+          break;
+        }
+        const uint32_t sp = base + (uint32_t)s * L::kStage;
+        if (st < p.n_st) {
+          for (int sub = 0; sub < 2 && 2 * st + sub < p.kb_total; ++sub, ++ab) {
+            const int u = ab % kNA;
+            if (!mbar_wait(&a_full[u], (uint32_t)(ab / kNA) & 1u, p.status, abort_flag)) {
+              alive = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint64_t db = sdesc_sw128(sp + (uint32_t)sub * L::kTokSub);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)  // K = 32 int8 = 8 TMEM columns per step
+                mma_i8_tmem_a(tmem + kColAcc, tmem + kColA + 32u * (uint32_t)u + 8u * (uint32_t)kk,
+                              db + 2 * kk, id_i8, (st > 0 || sub > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(&a_empty[u]);
+            }
+            __syncwarp();
+          }
+        } else {
+          tc_fence_after();
+          if (lane == 0) {
+            const int c = st - p.n_st;
+            const uint64_t da = sdesc_sw128(sp + 2 * L::kTokSub);  // L2^T chunk [128][64]
+            const uint64_t db = sdesc_sw128(sp);                    // bf16(XL1) chunk [192][64]
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 B per step
+              mma_bf16(tmem + kColLr, da + 2 * kk, db + 2 * kk, id_bf, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          __syncwarp();
+        }
+        if (lane == 0) mma_commit(&empty[s]);
+        __syncwarp();
+      }
+      if (lane == 0) mma_commit(acc_full);
+      __syncwarp();
+    }
+  } else {
+    // =============================== weight expansion into TMEM, epilogue
+    const int q = warp & 3;                          // TMEM lane quarter
+    const int row = q * 32 + lane;                   // channel row of the tile
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const uint32_t x7 = (uint32_t)row & 7u;
+    pdl_wait();  // s_x comes from the preceding kernel
+    int it = 0, ab = 0, tcount = 0;
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < p.tiles && alive && !*abort_flag;
+         tile += gridDim.x, ++tcount) {
+      const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
+      const int gc = tn * kCh + row;
+      const float sw = gc < p.N ? __ldg(p.s_w + gc) : 0.f;
+      // int4 -> int8 (16 * code) for this thread's channel row, one k-block
+      // (32 TMEM columns) at a time; inside each 16-byte packed chunk the low
+      // nibbles are codes 0-15 and the high nibbles codes 16-31 of the group
+      for (int st = 0; st < p.n_st && alive; ++st, ++it) {
+        const int s = it % kNS;
+        if (!mbar_wait(&full[s], (uint32_t)(it / kNS) & 1u, p.status, abort_flag)) {
+          alive = false;
+          break;
+        }
+        const uint32_t wrow = base + (uint32_t)s * L::kStage + 2 * L::kTokSub + (uint32_t)row * 128u;
+        const int nsub = (2 * st + 1 < p.kb_total) ? 2 : 1;
+        uint4 w[2][4];
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub)
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            if (sub < nsub) w[sub][c4] = ld_shared_v4_a8(wrow + ((((uint32_t)(sub * 4 + c4)) ^ x7) << 4));
+        bool ok = true;
+#pragma unroll
+        for (int sub = 0; sub < 2; ++sub) {
+          if (sub < nsub) {
+            uint32_t v[32];
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+              const uint32_t ww[4] = {w[sub][c4].x, w[sub][c4].y, w[sub][c4].z, w[sub][c4].w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[8 * c4 + e] = (ww[e] << 4) & 0xF0F0F0F0u;
+                v[8 * c4 + 4 + e] = ww[e] & 0xF0F0F0F0u;
+              }
+            }
+            const int u = (ab + sub) % kNA;
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(&a_empty[u],
+                                                         ((uint32_t)((ab + sub) / kNA) & 1u) ^ 1u,
+                                                         p.status, abort_flag));
+            if (ok) {
+              tc_fence_after();
+              tmem_st32(tmem + kColA + 32u * (uint32_t)u + lane_off, v);
+            }
+          }
+        }
+        if (!ok) {
+          alive = false;
+          break;
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        for (int sub = 0; sub < nsub; ++sub) mbar_arrive(&a_full[(ab + sub) % kNA]);
+        ab += nsub;
+      }
+      it += p.n_lr;  // low-rank stages go to the MMA only
+      if (!alive) break;
+      // ---- epilogue: Y[t][c] = s_x[t] s_w[c] (acc >> 4) + lr, bf16
+      if (!__all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)tcount & 1u, p.status, abort_flag)))
+        break;
+      tc_fence_after();
+      for (int j = 0; j < kTk / 32; ++j) {
+        uint32_t a[32], l[32];
+        tmem_ld32_a8(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
+        if (p.r > 0) tmem_ld32_a8(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
+        tmem_ld_wait();
+        if (gc < p.N) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int t = tm * kTk + 32 * j + e;
+            if (t < p.M) {
+              float y = __ldg(p.s_x + t) * sw * (float)(((int)a[e]) >> 4);
+              if (p.r > 0) y += __uint_as_float(l[e]);
+              p.Y[(size_t)t * p.N + gc] = __float2bfloat16_rn(y);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
+  A8Params p{};
+  p.s_x = a.s_x;
+  p.s_w = a.s_w;
+  p.Y = reinterpret_cast<__nv_bfloat16*>(a.Y);
+  p.status = reinterpret_cast<uint32_t*>(a.ws);
+  p.M = a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.r = a.r;
+  p.kb_total = a.K / kKb;
+  p.n_st = (p.kb_total + 1) / 2;
+  p.n_lr = (a.r + 63) / 64;
+  p.tiles_m = (a.M + kTk - 1) / kTk;
+  p.tiles = p.tiles_m * ((a.N + kCh - 1) / kCh);
+  CUtensorMap map_t, map_w, map_xb, map_l2;
+  if (!encode_tiled_2d(&map_t, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq8, (uint64_t)a.K, (uint64_t)a.M,
+                       (uint64_t)a.K, 128, kTk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tiled_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, (uint64_t)(a.K / 2),
+                       (uint64_t)a.N, (uint64_t)(a.K / 2), 128, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (a.r > 0) {
+    if (!encode_tiled_2d(&map_xb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.XL1b, (uint64_t)a.r,
+                         (uint64_t)a.M, (uint64_t)a.r * 2, 64, kTk, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tiled_2d(&map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L2t, (uint64_t)a.r,
+                         (uint64_t)a.N, (uint64_t)a.r * 2, 64, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    map_xb = map_t;  // never read
+    map_l2 = map_t;
+  }
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_set >> dev & 1u)) {
+    cudaError_t e = cudaFuncSetAttribute(w4a4_lr_gemm_a8_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)A8Smem::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(p.tiles, num_sms()), 1, 1);
+  cfg.blockDim = dim3(kThreadsA8, 1, 1);
+  cfg.dynamicSmemBytes = A8Smem::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = tuning().pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel, map_t, map_w, map_xb, map_l2, p);
+}
+
+}  // namespace tq

@@ -11,6 +11,7 @@ namespace tq {
 struct Tuning {
   int split_k = 0;        // decode GEMM: number of K splits
   int pdl = 1;            // launch the GEMM with programmatic dependent launch
+  int layer_a8 = 0;       // tq_w4a4_lr_layer at M > 128: codes one per byte
 };
 Tuning& tuning();
 
@@ -22,9 +23,26 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 float* XL1, cudaStream_t stream);
 
 // Activation stage on tensor cores (many tokens): rotation and X L1 as MMAs.
+// Codes packed (Xq, [M][K/2]) or one int8 per code (Xq8, [M][K]); X L1 as
+// fp32 (XL1) and / or rounded to bf16 (XL1b), either may be null.
 bool act_tc_supported(int M, int K, int had_block, int r);
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
-                          int r, uint8_t* Xq, float* s_x, float* XL1, cudaStream_t stream);
+                          int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
+                          cudaStream_t stream);
+
+// GEMM with one int8 per activation code (weights expanded into TMEM).
+struct GemmA8Args {
+  const int8_t* Xq8;      // [M][K]
+  const float* s_x;
+  const uint8_t* Wq;      // [N][K/2]
+  const float* s_w;
+  const uint16_t* XL1b;   // [M][r] bf16
+  const uint16_t* L2t;    // [N][r] bf16
+  int M, N, K, r;
+  uint16_t* Y;
+  void* ws;               // status word at offset 0
+};
+cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
 
 struct GemmArgs {
   const uint8_t* Xq;

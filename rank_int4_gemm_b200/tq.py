@@ -45,6 +45,11 @@ _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_w4a4_lr_layer.restype = _I
 _lib.tq_w4a4_lr_layer.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
                                   ctypes.c_size_t, _P]
+_lib.tq_quantize_act_i8.restype = _I
+_lib.tq_quantize_act_i8.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]
+_lib.tq_w4a4_lr_gemm_a8.restype = _I
+_lib.tq_w4a4_lr_gemm_a8.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
+                                    ctypes.c_size_t, _P]
 _lib.tq_query_device_status.restype = _I
 _lib.tq_query_device_status.argtypes = [_P, _P]
 
@@ -127,6 +132,28 @@ def tq_quantize_act(X: torch.Tensor, had_block: int, L1t=None, Xq=None, s_x=None
     return Xq, s_x, (XL1 if r else None)
 
 
+def tq_quantize_act_i8(X: torch.Tensor, had_block: int, L1t=None, Xq8=None, s_x=None, XL1b=None,
+                       stream=None):
+    """X [M][K] bf16 (+ L1^T) -> (Xq8 [M][K] int8 codes, s_x [M] f32, XL1b [M][r] bf16)."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, (M, K), "X")
+    r = 0 if L1t is None else L1t.shape[0]
+    if r:
+        _need(L1t, torch.bfloat16, (r, K), "L1t")
+    dev = X.device
+    if Xq8 is None:
+        Xq8 = torch.empty(M, K, dtype=torch.int8, device=dev)
+    if s_x is None:
+        s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    if r and XL1b is None:
+        XL1b = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    _check(_lib.tq_quantize_act_i8(_ptr(X), M, K, int(had_block), _ptr(L1t) if r else None, r,
+                                   _ptr(Xq8), _ptr(s_x), _ptr(XL1b) if r else None,
+                                   _stream(stream)),
+           "tq_quantize_act_i8")
+    return Xq8, s_x, (XL1b if r else None)
+
+
 def tq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
     return int(_lib.tq_gemm_workspace_bytes(M, N, K, r))
 
@@ -161,6 +188,25 @@ def tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, workspace=None
                                 _ptr(XL1) if r else None, _ptr(L2t) if r else None,
                                 M, N, K, r, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
            "tq_w4a4_lr_gemm")
+    return Y
+
+
+def tq_w4a4_lr_gemm_a8(Xq8, s_x, Wq, s_w, XL1b=None, L2t=None, Y=None, workspace=None,
+                       stream=None):
+    """Y [M][N] bf16 = s_x s_w (Xq8 . Wq) + XL1b L2^T, codes one per byte."""
+    M, K = Xq8.shape
+    N = Wq.shape[0]
+    r = 0 if XL1b is None else XL1b.shape[1]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
+    if workspace is None:
+        workspace = Workspace(Xq8.device)
+    need = tq_gemm_workspace_bytes(M, N, K, r)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_gemm_a8(_ptr(Xq8), _ptr(s_x), _ptr(Wq), _ptr(s_w),
+                                   _ptr(XL1b) if r else None, _ptr(L2t) if r else None,
+                                   M, N, K, r, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
+           "tq_w4a4_lr_gemm_a8")
     return Y
 
 

@@ -14,13 +14,17 @@ Y_MAX_ABS = 1e-2
 MIDPOINT_REL = 1e-6
 
 
-def check_codes(gpu_packed, orc_q, orc_t, what="codes"):
-    """Unpack the GPU's packed codes and compare them with the oracle's.
+def check_codes(gpu_packed, orc_q, orc_t, what="codes", packed=True):
+    """Unpack the GPU's packed codes (or take them one per byte when
+    packed=False) and compare them with the oracle's.
 
     Returns the fraction of codes that differ (all of them allowed midpoint
     flips); raises AssertionError on any other difference.
     """
-    gq = oracle.unpack_int4(np.ascontiguousarray(gpu_packed))
+    if packed:
+        gq = oracle.unpack_int4(np.ascontiguousarray(gpu_packed))
+    else:
+        gq = np.asarray(gpu_packed).astype(np.int8)
     assert gq.shape == orc_q.shape, (gq.shape, orc_q.shape)
     diff = gq.astype(np.int32) - orc_q.astype(np.int32)
     bad = diff != 0
@@ -63,3 +67,12 @@ def check_y(gpu_y, y64, what="Y"):
     assert fro <= Y_REL_FRO, f"{what}: relative Frobenius error {fro:.3e} > {Y_REL_FRO}"
     assert mx <= Y_MAX_ABS, f"{what}: max-abs error {mx:.3e} of max|Y| > {Y_MAX_ABS}"
     return fro, mx
+
+
+def y_given_codes(gpu_codes, o):
+    """The oracle's epilogue evaluated on the GPU's activation codes (already
+    checked by check_codes to differ from the oracle's only by midpoint
+    flips) with the oracle's scales, weight codes and low-rank term: the
+    reference for Y when the codes may legitimately differ."""
+    acc = oracle.int_gemm(np.asarray(gpu_codes).astype(np.int8), o["qw"])
+    return oracle.epilogue(o["s_x"], o["s_w"], acc, o["lr"])
