@@ -3,12 +3,14 @@
 
 Workload (one GPU): the Llama-3-8B attention projection in the decode
 regime, K = N = 4096, rank 32, Hadamard block 128, M = 16 tokens (other M via
---m).  One "step" is one pass of the hot path -- tq_quantize_act (rotation,
-per-token INT4 codes, X L1) then tq_w4a4_lr_gemm (INT4 GEMM, INT32
-accumulation, bf16 low-rank branch, epilogue) -- over 16 distinct layers, so
-the 16 x 8.9 MB of packed weights (143 MB) exceed the 126 MB L2 and every
-layer streams its weights from HBM.  The offline weight packing is not part
-of a step.  A step is replayed as one CUDA graph.
+--m).  One "step" is one pass of the hot path -- rotation, per-token INT4
+codes, X L1, INT4 GEMM with INT32 accumulation, bf16 low-rank branch and the
+shared epilogue, one tq_w4a4_lr_layer call (one fused kernel) per layer --
+over 16 distinct layers, so the 16 x 9.2 MB of operands (147 MB) exceed the
+126 MB L2 and every layer streams its weights from HBM.  The offline weight
+packing is not part of a step.  A step is replayed as one CUDA graph.
+--workload prefill_gateup|prefill_down|large_gateup|large_down|sweep times
+tq_quantize_act + tq_w4a4_lr_gemm on the prefill and sweep shapes instead.
 
 Metric: algorithmic GB/s of the layer (X + L1^T + Wq + s_w + L2^T + Y bytes
 per layer), the decode roofline quantity; TOPS (2 M N K) is reported beside it.
@@ -222,6 +224,28 @@ def capture(torch, fn):
     return g
 
 
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The slowest rank's value (every rank gets it); identity on one rank.
+    The tensor lives on `device`: a CUDA device under NCCL, the CPU under gloo."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_seed(rank: int) -> int:
+    """Seed base of a rank's independent batch of layers (weak scaling: every
+    rank streams its own weights, no data-path collective)."""
+    return 1000 * rank
+
+
+def whole_job(per_rank_units: float, world: int, ms: float) -> float:
+    """Units per second of all ranks together, timed by the slowest rank."""
+    return world * per_rank_units / (ms * 1e-3)
+
+
 def time_graph(torch, g, steps, warmup, dist=None):
     for _ in range(warmup):
         g.replay()
@@ -248,7 +272,7 @@ def run_tq(args, rank, world, local_rank, dist):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     M, L = args.m, args.layers
-    layers = build_layers(tq, torch, M, L, seed0=1000 * rank, device=dev)
+    layers = build_layers(tq, torch, M, L, seed0=replica_seed(rank), device=dev)
 
     def step():
         for lay in layers:
@@ -262,10 +286,7 @@ def run_tq(args, rank, world, local_rank, dist):
     with ClockSampler(local_rank) as clk:
         ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
     clocks = clk.summary()
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
 
     # per-kernel durations of the same step, events captured in the graph
     evs = [(torch.cuda.Event(enable_timing=True, external=True),
@@ -298,10 +319,7 @@ def run_tq(args, rank, world, local_rank, dist):
 
     g_e2e = capture(torch, step_e2e)
     ms_e2e = time_graph(torch, g_e2e, args.steps, args.warmup, dist if world > 1 else None)
-    if world > 1:
-        t = torch.tensor([ms_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = max_over_ranks(ms_e2e, dist if world > 1 else None, dev)
 
     # the two-call path on the same layers, for comparison
     g_two = capture(torch, lambda: [layer_call_two(tq, l) for l in layers])
@@ -327,8 +345,8 @@ def run_tq(args, rank, world, local_rank, dist):
             del ls, g2
 
     bytes_step = L * layer_bytes(M, K_DIM, N_DIM, RANK)
-    value = world * bytes_step / ms / 1e6          # GB/s, all ranks
-    e2e = world * bytes_step / ms_e2e / 1e6
+    value = whole_job(bytes_step, world, ms) / 1e9        # GB/s, all ranks
+    e2e = whole_job(bytes_step, world, ms_e2e) / 1e9
     peak, peak_src = measured_peaks()
     gb = layer_bytes(M, K_DIM, N_DIM, RANK)   # the fused kernel reads X, writes Y
     # the step is L launches of the one fused kernel, back to back (each
@@ -401,12 +419,12 @@ def run_prefill(args, rank, world, local_rank, dist):
     L = max(1, min(args.layers, -(-200_000_000 // per_layer)))
     layers = []
     for i in range(L):
-        w = synth.make_weights(sh, seed=1000 * rank + 10 * i, device="cuda")
+        w = synth.make_weights(sh, seed=replica_seed(rank) + 10 * i, device="cuda")
         Rt = w["Rt"].to(dev)
         Wq, s_w = tq.tq_pack_weight(Rt, b)
         del Rt
         layers.append({
-            "X": synth.make_activations(sh, seed=1000 * rank + 10 * i, M=M).to(dev),
+            "X": synth.make_activations(sh, seed=replica_seed(rank) + 10 * i, M=M).to(dev),
             "L1t": w["L1t"].to(dev) if r else None, "L2t": w["L2t"].to(dev) if r else None,
             "Wq": Wq, "s_w": s_w,
             "Xq": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
@@ -435,10 +453,7 @@ def run_prefill(args, rank, world, local_rank, dist):
                 "warmup": args.warmup}
     with ClockSampler(local_rank) as clk:
         ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
     evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
            for _ in layers]
     g_ev = capture(torch, lambda: [one(l, e) for l, e in zip(layers, evs)])
@@ -456,7 +471,7 @@ def run_prefill(args, rank, world, local_rank, dist):
     peak, src = int8_peak(sustained=False)
     achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
     out = {
-        "metric": METRIC, "value": round(world * L * ops / ms / 1e9, 2), "unit": "TOPS",
+        "metric": METRIC, "value": round(whole_job(L * ops, world, ms) / 1e12, 2), "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int4", "data": "synthetic",
@@ -467,7 +482,10 @@ def run_prefill(args, rank, world, local_rank, dist):
         "GB/s": round(world * L * per_layer / ms / 1e6, 1),
         "us_per_layer": round(ms * 1e3 / L, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
-                     "unit": "TOPS", "frac": round(achieved / peak, 4), "traffic": None,
+                     "unit": "TOPS", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm.cu",
+                                                 "w4a4_lr_gemm_prefill_sweep4096.md")
+                     if (M, K, N, r) == (4096, 4096, 4096, 64) else None,
                      "kernel": "w4a4_lr_gemm_kernel (prefill tiling)",
                      "gemm_us": round(gemm_ms_avg * 1e3, 2), "peak_source": src,
                      "act_us": round(act_ms_avg * 1e3, 2),
