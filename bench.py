@@ -428,21 +428,35 @@ def run_prefill(args, rank, world, local_rank, dist):
             "L1t": w["L1t"].to(dev) if r else None, "L2t": w["L2t"].to(dev) if r else None,
             "Wq": Wq, "s_w": s_w,
             "Xq": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            "Xq8": torch.empty(M, K, dtype=torch.int8, device=dev),
             "s_x": torch.empty(M, dtype=torch.float32, device=dev),
             "XL1": torch.empty(M, r, dtype=torch.float32, device=dev) if r else None,
+            "XL1b": torch.empty(M, r, dtype=torch.bfloat16, device=dev) if r else None,
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
             "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev),
         })
+    # codes one per byte when the activation stage runs on tensor cores
+    # (b <= 128, r <= 128): the path tq_w4a4_lr_layer takes for M > 128
+    a8 = b <= 128 and r <= 128
     torch.cuda.synchronize()
 
-    def one(lay, ev=None):
+    def one(lay, ev=None, packed=not a8):
         if ev is not None:
             ev[2].record()
-        tq.tq_quantize_act(lay["X"], b, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"], XL1=lay["XL1"])
+        if packed:
+            tq.tq_quantize_act(lay["X"], b, lay["L1t"], Xq=lay["Xq"], s_x=lay["s_x"],
+                               XL1=lay["XL1"])
+        else:
+            tq.tq_quantize_act_i8(lay["X"], b, lay["L1t"], Xq8=lay["Xq8"], s_x=lay["s_x"],
+                                  XL1b=lay["XL1b"])
         if ev is not None:
             ev[0].record()
-        tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"], lay["L2t"],
-                           Y=lay["Y"], workspace=lay["ws"])
+        if packed:
+            tq.tq_w4a4_lr_gemm(lay["Xq"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1"],
+                               lay["L2t"], Y=lay["Y"], workspace=lay["ws"])
+        else:
+            tq.tq_w4a4_lr_gemm_a8(lay["Xq8"], lay["s_x"], lay["Wq"], lay["s_w"], lay["XL1b"],
+                                  lay["L2t"], Y=lay["Y"], workspace=lay["ws"])
         if ev is not None:
             ev[1].record()
 
@@ -468,6 +482,11 @@ def run_prefill(args, rank, world, local_rank, dist):
     gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
     act_ms_avg = sum(act_ms) / len(act_ms)
     ops = 2 * M * N * K
+    packed_ms = None
+    if a8:
+        g_p = capture(torch, lambda: [one(l, packed=True) for l in layers])
+        packed_ms = time_graph(torch, g_p, args.steps, args.warmup)
+        del g_p
     peak, src = int8_peak(sustained=False)
     achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
     out = {
@@ -483,14 +502,17 @@ def run_prefill(args, rank, world, local_rank, dist):
         "us_per_layer": round(ms * 1e3 / L, 3),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
                      "unit": "TOPS", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm.cu",
-                                                 "w4a4_lr_gemm_prefill_sweep4096.md")
-                     if (M, K, N, r) == (4096, 4096, 4096, 64) else None,
-                     "kernel": "w4a4_lr_gemm_kernel (prefill tiling)",
+                     "traffic": profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm_a8.cu",
+                                                 "w4a4_lr_gemm_a8_sweep4096.md")
+                     if a8 and (M, K, N, r) == (4096, 4096, 4096, 64) else None,
+                     "kernel": "w4a4_lr_gemm_a8_kernel" if a8 else "w4a4_lr_gemm_kernel (prefill tiling)",
                      "gemm_us": round(gemm_ms_avg * 1e3, 2), "peak_source": src,
                      "act_us": round(act_ms_avg * 1e3, 2),
                      "lowrank_flops_per_launch": 2 * M * r * (K + N)},
         "gpu_launches": 2 * L * args.steps,
+        "path": ("tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte), the path "
+                 "tq_w4a4_lr_layer takes" if a8 else "tq_quantize_act + tq_w4a4_lr_gemm"),
+        "packed_code_path_us_per_layer": round(packed_ms * 1e3 / L, 3) if packed_ms else None,
         "clocks": clk.summary(),
     }
     return out

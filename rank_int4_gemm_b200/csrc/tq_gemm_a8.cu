@@ -64,7 +64,10 @@ struct A8Smem {
   static constexpr uint32_t kTokSub = kTk * 128;            // 24 KB
   static constexpr uint32_t kWBytes = kCh * 128;            // 16 KB
   static constexpr uint32_t kStage = 2 * kTokSub + kWBytes;  // 64 KB
-  static constexpr uint32_t kBar = kNS * kStage;
+  // epilogue transpose buffers, one per converter warp: [32 tokens][40 bf16]
+  static constexpr uint32_t kYRow = 80;
+  static constexpr uint32_t kYBuf = kNS * kStage;
+  static constexpr uint32_t kBar = kYBuf + 4 * 32 * kYRow;
   // full[kNS], empty[kNS], a_full[kNA], a_empty[kNA], acc_full, acc_empty
   static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNA + 2;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
@@ -332,26 +335,41 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       }
       it += p.n_lr;  // low-rank stages go to the MMA only
       if (!alive) break;
-      // ---- epilogue: Y[t][c] = s_x[t] s_w[c] (acc >> 4) + lr, bf16
+      // ---- epilogue: Y[t][c] = s_x[t] s_w[c] (acc >> 4) + lr, bf16.  Each
+      //      warp owns 32 channels; per 32 tokens it transposes its block
+      //      through shared memory and stores whole 64-byte row segments.
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)tcount & 1u, p.status, abort_flag)))
         break;
       tc_fence_after();
+      const uint32_t ybuf = base + L::kYBuf + (uint32_t)(warp - 2) * 32u * L::kYRow;
+      const int gc0 = tn * kCh + q * 32;  // first channel of this warp
       for (int j = 0; j < kTk / 32; ++j) {
         uint32_t a[32], l[32];
         tmem_ld32_a8(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
         if (p.r > 0) tmem_ld32_a8(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
+        const int t0 = tm * kTk + 32 * j;
+        const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
         tmem_ld_wait();
-        if (gc < p.N) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int t = tm * kTk + 32 * j + e;
-            if (t < p.M) {
-              float y = __ldg(p.s_x + t) * sw * (float)(((int)a[e]) >> 4);
-              if (p.r > 0) y += __uint_as_float(l[e]);
-              p.Y[(size_t)t * p.N + gc] = __float2bfloat16_rn(y);
-            }
-          }
+        for (int e = 0; e < 32; ++e) {
+          float y = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
+          if (p.r > 0) y += __uint_as_float(l[e]);
+          const __nv_bfloat16 h = __float2bfloat16_rn(y);
+          asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
+                       "h"(*reinterpret_cast<const unsigned short*>(&h))
+                       : "memory");
         }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int idx = lane + 32 * k;      // 32 token rows x 4 16-byte parts
+          const int e = idx >> 2, part = idx & 3;
+          const uint4 v = ld_shared_v4_a8(ybuf + (uint32_t)e * L::kYRow + (uint32_t)part * 16u);
+          const int t = t0 + e, c = gc0 + part * 8;
+          if (t < p.M && c < p.N)
+            *reinterpret_cast<uint4*>(p.Y + (size_t)t * p.N + c) = v;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(acc_empty);

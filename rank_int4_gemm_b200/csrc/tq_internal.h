@@ -11,7 +11,7 @@ namespace tq {
 struct Tuning {
   int split_k = 0;        // decode GEMM: number of K splits
   int pdl = 1;            // launch the GEMM with programmatic dependent launch
-  int layer_a8 = 0;       // tq_w4a4_lr_layer at M > 128: codes one per byte
+  int layer_a8 = 1;       // tq_w4a4_lr_layer at M > 128: codes one per byte
 };
 Tuning& tuning();
 
