@@ -16,7 +16,7 @@
 //           pushed to every CTA of the cluster (distributed shared memory)
 //   pass 2  X tiles again (now from L2), rotation -> codes, packed into the
 //           ABI layout and stored; X.L1 accumulated in TMEM over the slice
-//   then    X.L1 partials pushed to the owner CTA of each column, summed in
+//   then    X.L1 partial rows pushed to the CTA that owns the row, summed in
 //           cluster-rank order (deterministic) and stored.
 //
 // Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-5:
@@ -163,7 +163,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       for (int h = 0; h < 2; ++h) {
         const int k = c * 8 + 2 * e + h;
         uint32_t bits = 0;  // bf16 0
-        if ((j / p.b) == (k / p.b))
+        if (((j ^ k) & ~(p.b - 1)) == 0)  // same b-block
           bits = (__popc((unsigned)(j & k & (p.b - 1))) & 1) ? 0xBF80u : 0x3F80u;
         two |= bits << (16 * h);
       }
@@ -343,41 +343,64 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_arrive(&rot_empty[u]);
     }
 
-    // ---- X L1: partial over the slice -> the column's owner CTA
+    // ---- X L1: partial over the slice -> the row's owner CTA
     bool xl1_ok = true;
     if (r > 0) xl1_ok = __all_sync(kFull, mbar_wait(xl1_full, 0u, nullptr, abort_flag));
     cluster_arrive_rel();  // B2: every CTA is past pass 2 (stages free)
     cluster_wait_acquire();
-    const int cols_max = r > 0 ? (r + (int)csize - 1) / (int)csize : 0;
-    const uint32_t recv = base + L::kStage0;  // [C][128][cols_max] fp32
+    // rows of the tile are split among the cluster: CTA o sums rows
+    // [o rpo, (o+1) rpo); every CTA sends each row's partial to its owner
+    const int rpo = (kTok + (int)csize - 1) / (int)csize;
+    const uint32_t recv = base + L::kStage0;  // [C senders][rpo][r] fp32
     if (r > 0 && xl1_ok) {
       tc_fence_after();
+      const int owner = row / rpo;
+      const uint32_t dst = dsmem_map(recv + (uint32_t)(((int)crank * rpo + row - owner * rpo) * r) * 4u,
+                                     (uint32_t)owner);
       for (int c0 = 0; c0 < r; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_xl1 + (uint32_t)c0 + lane_off, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int col = c0 + e;
-          const int owner = col * (int)csize / r;
-          const int lo = (owner * r + (int)csize - 1) / (int)csize;
-          dsmem_st_f32(dsmem_map(recv + (uint32_t)(((int)crank * kTok + row) * cols_max + col - lo) * 4u,
-                                 (uint32_t)owner),
-                       __uint_as_float(v[e]));
-        }
+        for (int e = 0; e < 16; e += 4)
+          asm volatile("st.shared::cluster.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + (uint32_t)(c0 + e) * 4u),
+                       "r"(v[e]), "r"(v[e + 1]), "r"(v[e + 2]), "r"(v[e + 3])
+                       : "memory");
       }
     }
     cluster_arrive_rel();  // B3: partials delivered
     cluster_wait_acquire();
-    if (r > 0 && grow < p.M && !*abort_flag) {
-      const int lo = ((int)crank * r + (int)csize - 1) / (int)csize;
-      const int hi = (((int)crank + 1) * r + (int)csize - 1) / (int)csize;
-      for (int cc = 0; cc < hi - lo; ++cc) {
-        float s = 0.f;
-        for (uint32_t z = 0; z < csize; ++z)
-          s += ld_shared_f32_tc(recv + (uint32_t)(((int)z * kTok + row) * cols_max + cc) * 4u);
-        if (p.XL1) p.XL1[(size_t)grow * r + lo + cc] = s;
-        if (p.XL1b) p.XL1b[(size_t)grow * r + lo + cc] = __float2bfloat16_rn(s);
+    if (r > 0 && !*abort_flag) {
+      // this CTA's rows: sum the C partials in cluster-rank order
+      const int row0 = (int)crank * rpo;
+      const int nrow = min(rpo, kTok - row0);
+      const int q4 = r / 4;  // 4-column groups per row
+      const int tid = threadIdx.x - kEpiFirstWarp * 32;
+      for (int v4 = tid; v4 < nrow * q4; v4 += kEpiThreadsTc) {
+        const int rr = v4 / q4, c = (v4 - rr * q4) * 4;
+        const int gr = tile * kTok + row0 + rr;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (uint32_t z = 0; z < csize; ++z) {
+          float4 t;
+          asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(t.x), "=f"(t.y), "=f"(t.z), "=f"(t.w)
+                       : "r"(recv + (uint32_t)((((int)z * rpo + rr) * r + c) * 4)));
+          acc.x += t.x;
+          acc.y += t.y;
+          acc.z += t.z;
+          acc.w += t.w;
+        }
+        if (gr < p.M) {
+          if (p.XL1) *reinterpret_cast<float4*>(p.XL1 + (size_t)gr * r + c) = acc;
+          if (p.XL1b) {
+            __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
+            __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
+            uint2 u;
+            u.x = *reinterpret_cast<uint32_t*>(&h0);
+            u.y = *reinterpret_cast<uint32_t*>(&h1);
+            *reinterpret_cast<uint2*>(p.XL1b + (size_t)gr * r + c) = u;
+          }
+        }
       }
     }
   }
@@ -413,11 +436,46 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
   p.kb_total = K / kBlk;
   p.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   const int tiles = (M + kTok - 1) / kTok;
-  // a cluster of C CTAs along K per 128-token tile, about one CTA per SM
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_set >> dev & 1u)) {
+    cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)TcSmem::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  // a cluster of C CTAs along K per 128-token tile: about one CTA per SM,
+  // and no larger than lets every cluster of the grid be resident at once
   int C = std::max(1, std::min(kMaxC, num_sms() / tiles));
   C = std::min(C, p.kb_total);
-  p.nb = (p.kb_total + C - 1) / C;
-  C = (p.kb_total + p.nb - 1) / p.nb;  // every CTA owns at least one block
+  for (;; C /= 2) {
+    p.nb = (p.kb_total + C - 1) / C;
+    const int Ce = (p.kb_total + p.nb - 1) / p.nb;  // every CTA owns at least one block
+    if (C <= 1) {
+      C = Ce;
+      break;
+    }
+    cudaLaunchConfig_t q = {};
+    q.gridDim = dim3(Ce, tiles, 1);
+    q.blockDim = dim3(kThreadsTc, 1, 1);
+    q.dynamicSmemBytes = TcSmem::kAlloc;
+    cudaLaunchAttribute qa[1];
+    qa[0].id = cudaLaunchAttributeClusterDimension;
+    qa[0].val.clusterDim.x = Ce;
+    qa[0].val.clusterDim.y = 1;
+    qa[0].val.clusterDim.z = 1;
+    q.attrs = qa;
+    q.numAttrs = 1;
+    int active = 0;
+    if (cudaOccupancyMaxActiveClusters(&active, quantize_act_tc_kernel, &q) == cudaSuccess &&
+        active >= tiles) {
+      C = Ce;
+      break;
+    }
+    cudaGetLastError();
+  }
   CUtensorMap map_x, map_l1;
   if (!encode_tiled_2d(&map_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
                        (uint64_t)K * 2, 64, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -428,16 +486,6 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
       return cudaErrorInvalidValue;
   } else {
     map_l1 = map_x;  // never read
-  }
-  static uint64_t attr_set = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(attr_set >> dev & 1u)) {
-    cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)TcSmem::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, tiles, 1);

@@ -15,7 +15,7 @@
 //     exactly (|acc| <= 16*49*K < 2^31); the epilogue shifts it back.
 //
 // Tile: 128 channels (MMA M = TMEM lanes) x 192 tokens (MMA N).  TMEM:
-// INT32 accumulator [192] | two 32-column A buffers | fp32 low-rank [192].
+// INT32 accumulator [192] | four 32-column A buffers | fp32 low-rank [192].
 // Persistent CTAs walk the tiles; a 3-stage TMA ring carries two k-blocks of
 // tokens and weights per stage, then the low-rank chunks (64 columns of
 // bf16(XL1) and L2^T per stage, kind::f16 into the low-rank accumulator).
