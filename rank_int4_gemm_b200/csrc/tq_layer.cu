@@ -9,20 +9,21 @@
 //               staged once in shared memory; Sylvester transform (the warp
 //               butterflies of tq_quantize_act, so the codes are the same
 //               bits) and partial absmax, exchanged across the cluster through
-//               distributed shared memory; the rotated values stay in
-//               registers and become the codes, written as int8 (16 * code)
-//               straight into the MMA's B operand.  Only then, off the path
-//               to the integer MMAs, the same warps compute the slice's X.L1
-//               partial on mma.sync (L1^T fragments were fetched into
-//               registers before the kernel waited on its predecessor) and
-//               push it to split 0.  Warps 0-3 run the epilogue.
-//   warps 16-19 expand the streamed int4 weights into int8 operand slots;
-//               the first kNOPS k-blocks are expanded before the token codes
-//               exist, so only the rest wait on the MMA.  In split 0 they also
-//               place the tile's L2^T rows (the low-rank A operand).
-//   warp 20     TMA producer of the packed weights (started before the kernel
-//               waits on its predecessor: weights never depend on it).
-//   warp 21     TMEM allocation and MMA issue: kind::i8 for the codes,
+//               distributed shared memory.  While that exchange completes
+//               the same warps compute the slice's X.L1 partial on mma.sync
+//               (L1^T fragments are fetched into registers while X lands)
+//               and push it to split 0; then the rotated values, kept in
+//               registers, become the codes, written as int8 (16 * code)
+//               straight into the MMA's B operand.  Warps 0-3 run the
+//               epilogue.
+//   warps 16-19 expand the int4 weights into one int8 operand slot per
+//               k-block (the whole slice is requested at CTA start and lands
+//               packed in the odd slots), all before the token codes exist,
+//               so the MMAs run back to back.  In split 0 they also place the
+//               tile's L2^T rows (the low-rank A operand).
+//   warp 16     also issues the weight TMAs in the prologue (before the
+//               kernel waits on its predecessor: weights never depend on it),
+//               allocates TMEM and issues the MMAs: kind::i8 for the codes,
 //               kind::f16 for the low-rank branch (split 0).
 //
 // Cluster barriers, all threads of all CTAs in order: B0 (every CTA is
@@ -50,16 +51,18 @@ constexpr int kBN = 16;            // tokens (MMA N)
 constexpr int kKB = 128;           // codes per k-block
 constexpr int kPackedRow = 64;     // packed bytes per row per k-block
 constexpr int kKBS = 2;            // k-blocks per TMA stage (128-byte swizzled rows)
-constexpr int kNSTG = 4;           // TMA stages: a whole 1024-column slice requested at once
-constexpr int kNOPS = 4;           // int8 operand slots
+constexpr int kNSTG = 4;           // TMA stages (2 k-blocks each): the whole slice at CTA start
 constexpr int kMaxKb = 8;          // k-blocks per CTA (slice <= 1024 columns)
 constexpr int kMaxSplits = 4;      // split-K cluster size limit of this kernel
 constexpr int kMaxR = 32;          // low-rank width handled here
 constexpr int kE = 16;             // values per lane per warp pass
 constexpr int kW = 32 * kE;        // 512 columns per warp pass
 constexpr int kActWarps = 16, kConvWarps = 4;
-constexpr int kProducerWarp = kActWarps + kConvWarps, kMmaWarp = kProducerWarp + 1;
-constexpr int kThreads = (kMmaWarp + 1) * 32;
+// the first converter warp also issues the prologue TMAs, owns the TMEM
+// allocation and issues the MMAs (20 warps: five per SM sub-partition, so each
+// thread may hold up to 96 registers)
+constexpr int kIssueWarp = kActWarps;
+constexpr int kThreads = (kActWarps + kConvWarps) * 32;
 constexpr int kActThreads = kActWarps * 32;
 constexpr int kConvThreads = kConvWarps * 32;
 constexpr int kEpiThreads = 128;
@@ -79,14 +82,16 @@ struct LayerParams {
 
 // Shared-memory map (offsets from the 1024-aligned base).
 struct Smem {
-  static constexpr uint32_t kOp = kBM * 128;                  // one int8 weight k-block
-  static constexpr uint32_t kStg = kBM * 128;                 // one TMA stage (2 k-blocks packed)
-  static constexpr uint32_t kOpBase = 0;                      // also the L2^T tile (split 0)
-  static constexpr uint32_t kStgBase = kOpBase + kNOPS * kOp;
-  static constexpr uint32_t kBBase = kStgBase + kNSTG * kStg;  // token codes [kb][16][128]
+  // kMaxKb int8 weight k-blocks, one slot each; stage s (2 packed k-blocks,
+  // 128-byte swizzled rows) lands in slot 2s+1 and is expanded in place
+  static constexpr uint32_t kOp = kBM * 128;
+  static constexpr uint32_t kStg = kBM * 128;
+  static constexpr uint32_t kOpBase = 0;
+  static constexpr uint32_t kBBase = kOpBase + kMaxKb * kOp;  // token codes [kb][16][128]
   static constexpr uint32_t kBBytes = kMaxKb * kBN * 128;
   static constexpr uint32_t kLrBBase = kBBase + kBBytes;      // bf16(XL1) [16][64], SW128
-  static constexpr uint32_t kXBase = kLrBBase + kBN * 128;    // X slice [16][1024] bf16, swizzled
+  static constexpr uint32_t kLrABase = (kLrBBase + kBN * 128 + 1023u) & ~1023u;  // L2^T [128][64]
+  static constexpr uint32_t kXBase = kLrABase + kBM * 128;    // X slice [16][1024] bf16, swizzled
   static constexpr uint32_t kXRow = kMaxKb * kKB * 2;         // bytes per X row
   static constexpr uint32_t kXBytes = kBN * kXRow;
   // split-K partials [S][16][rows] + low-rank [16][rows]; before the epilogue
@@ -98,8 +103,8 @@ struct Smem {
   static constexpr uint32_t kAmax = kXRecv + kXRecvBytes;     // [S][16] + [16]
   static constexpr uint32_t kScale = kAmax + (kMaxSplits + 1) * kBN * 4;  // s_w [128]
   static constexpr uint32_t kBar = kScale + kBM * 4;
-  // barriers: stg_full, stg_empty, op_full, op_empty, b_ready, lr_ready, acc_full
-  static constexpr uint32_t kNumBars = 2 * kNSTG + 2 * kNOPS + 3;
+  // barriers: stg_full[kNSTG], op_full[kMaxKb], b_ready, lr_ready, acc_full
+  static constexpr uint32_t kNumBars = kNSTG + kMaxKb + 3;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kMisc + 32;
   static constexpr uint32_t kAlloc = kBytes + 1024;
@@ -186,10 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_::kBar);
   uint64_t* stg_full = bars;
-  uint64_t* stg_empty = bars + kNSTG;
-  uint64_t* op_full = bars + 2 * kNSTG;
-  uint64_t* op_empty = bars + 2 * kNSTG + kNOPS;
-  uint64_t* b_ready = bars + 2 * kNSTG + 2 * kNOPS;
+  uint64_t* op_full = bars + kNSTG;
+  uint64_t* b_ready = op_full + kMaxKb;
   uint64_t* lr_ready = b_ready + 1;
   uint64_t* acc_full = b_ready + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S_::kMisc);
@@ -212,15 +215,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   pdl_launch_dependents();  // the next layer may start staging its weights
   // ---------------------------------------------------------------- prologue
-  if (warp == kProducerWarp && lane == 0) {
-    for (int i = 0; i < kNSTG; ++i) {
-      mbar_init(&stg_full[i], 1);
-      mbar_init(&stg_empty[i], kConvThreads);
-    }
-    for (int i = 0; i < kNOPS; ++i) {
-      mbar_init(&op_full[i], kConvThreads);
-      mbar_init(&op_empty[i], 1);
-    }
+  if (warp == kIssueWarp && lane == 0) {
+    for (int i = 0; i < kNSTG; ++i) mbar_init(&stg_full[i], 1);
+    for (int i = 0; i < kMaxKb; ++i) mbar_init(&op_full[i], kConvThreads);
     mbar_init(b_ready, kActThreads);
     mbar_init(lr_ready, kActThreads + kConvThreads);
     mbar_init(acc_full, 1);
@@ -229,13 +226,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
     tma_prefetch_desc(&map_w);
     const uint64_t pol = policy_evict_first();
-    for (int i = 0; i < min(n_st, kNSTG); ++i) {
+    for (int i = 0; i < n_st; ++i) {  // the whole slice, into the odd slots
       mbar_arrive_expect_tx(&stg_full[i], S_::kStg);
-      tma_load_2d(smem + S_::kStgBase + i * S_::kStg, &map_w, &stg_full[i],
+      tma_load_2d(smem + S_::kOpBase + (2 * i + 1) * S_::kOp, &map_w, &stg_full[i],
                   (kb0 + i * kKBS) * kPackedRow, tile * kBM, pol);
     }
   }
-  if (warp == kMmaWarp) {
+  if (warp == kIssueWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -310,7 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane < S)
       dsmem_st_f32(dsmem_map(amax_all + (uint32_t)((split * kBN + warp) * 4), (uint32_t)lane), amax);
     cluster_arrive_release();  // B1: this CTA's absmax partials delivered
-    cluster_wait_acquire();
+    cluster_wait_acquire();  // B1 complete
 
     // ---- codes of token `warp` as the int8 B operand (16 * code: the code's
     //      low nibble in the high nibble)
@@ -345,9 +342,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();
     mbar_arrive(b_ready);
 
-    // ---- X L1 partial over the slice, off the path to the integer MMAs:
-    //      A fragments from the staged X (tokens x 16 columns), B from the
-    //      registers
+    // ---- X L1 partial over the slice (mma.sync, overlapping the integer
+    //      MMAs): A fragments from the staged X, B from the registers
     const uint32_t part = base + S_::kKRecv;  // [KP][16][r] fp32
     if (xl1_warp) {
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -422,30 +418,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     cluster_wait_acquire();    // B0
     cluster_arrive_release();  // B1 (nothing to publish from these warps)
-    bool alive = true, b1_done = false;
-    for (int st = 0; st < n_st && alive; ++st) {
-      const int sg_slot = st % kNSTG;
-      if (!mbar_wait(&stg_full[sg_slot], (uint32_t)(st / kNSTG) & 1u, p.status, abort_flag)) break;
-      const int nsub = min(kKBS, n_kb - st * kKBS);
-      const uint32_t sg = base + S_::kStgBase + sg_slot * S_::kStg;
-      for (int sub = 0; sub < nsub; ++sub) {
-        const int i = st * kKBS + sub;
-        if (i == kNOPS && !b1_done) {  // slots reused from here on: meet B1/B2 first
-          cluster_wait_acquire();
-          cluster_arrive_release();
-          b1_done = true;
-        }
-        if (!mbar_wait(&op_empty[i % kNOPS], ((uint32_t)(i / kNOPS) & 1u) ^ 1u, p.status,
-                       abort_flag)) {
-          alive = false;
-          break;
-        }
-        const uint32_t dst = base + S_::kOpBase + (uint32_t)(i % kNOPS) * S_::kOp + (uint32_t)tid * 128u;
-        const uint32_t x7 = (uint32_t)tid & 7u;
-        const uint32_t src = sg + (uint32_t)tid * 128u;
-        uint4 w[4];
+    // split 0: the tile's L2^T rows -> the low-rank A operand
+    if (do_lr) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(sub * 4 + q) ^ x7) << 4));
+      for (int j = 0; j < 8; ++j)
+        st_shared_v4(base + S_::kLrABase + sw_off((uint32_t)tid, (uint32_t)j),
+                     j < kMaxR / 8 ? l2row[j] : make_uint4(0u, 0u, 0u, 0u));
+      fence_proxy_async_smem();
+    }
+    // int4 -> int8, in place: each thread expands its row of the stage's
+    // first k-block into slot 2s, reads the second, and once all four warps
+    // have read the packed rows, writes the second into slot 2s+1
+    for (int st = 0; st < n_st; ++st) {
+      if (!mbar_wait(&stg_full[st], 0u, p.status, abort_flag)) break;
+      const uint32_t x7 = (uint32_t)tid & 7u;
+      const uint32_t src = base + S_::kOpBase + (uint32_t)(2 * st + 1) * S_::kOp + (uint32_t)tid * 128u;
+      auto expand = [&](const uint4 (&w)[4], int slot) {
+        const uint32_t dst = base + S_::kOpBase + (uint32_t)slot * S_::kOp + (uint32_t)tid * 128u;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint4 lo, hi;
@@ -460,87 +449,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
           st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&op_full[i % kNOPS]);
-      }
-      if (!alive) break;
-      mbar_arrive(&stg_empty[sg_slot]);
-    }
-    if (!b1_done) {
-      cluster_wait_acquire();    // B1
-      cluster_arrive_release();  // B2
-    }
-    // split 0: L2^T rows -> operand slot n_kb % kNOPS, the low-rank A operand
-    if (alive && do_lr) {
-      const int i = n_kb;
-      if (mbar_wait(&op_empty[i % kNOPS], ((uint32_t)(i / kNOPS) & 1u) ^ 1u, p.status, abort_flag)) {
-        const uint32_t dst0 = base + S_::kOpBase + (uint32_t)(i % kNOPS) * S_::kOp;
+      };
+      uint4 w[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          st_shared_v4(dst0 + sw_off((uint32_t)tid, (uint32_t)j),
-                       j < kMaxR / 8 ? l2row[j] : make_uint4(0u, 0u, 0u, 0u));
-        fence_proxy_async_smem();
-      }
-    }
-    if (p.r > 0) mbar_arrive(lr_ready);
-    sw_tile[tid] = sw;         // read by the epilogue after B3
-    cluster_wait_acquire();  // B2
-  } else if (warp == kProducerWarp) {
-    // =========================================================== producer
-    cluster_wait_acquire();    // B0
-    cluster_arrive_release();  // B1
-    const uint64_t pol = policy_evict_first();
-    for (int i = kNSTG; i < n_st; ++i) {
-      const int s = i % kNSTG;
-      if (!mbar_wait(&stg_empty[s], ((uint32_t)(i / kNSTG) & 1u) ^ 1u, p.status, abort_flag)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&stg_full[s], S_::kStg);
-        tma_load_2d(smem + S_::kStgBase + s * S_::kStg, &map_w, &stg_full[s],
-                    (kb0 + i * kKBS) * kPackedRow, tile * kBM, pol);
-      }
-      __syncwarp();
+      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)q ^ x7) << 4));
+      expand(w, 2 * st);  // slot 2s holds nothing yet
+#pragma unroll
+      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(4 + q) ^ x7) << 4));
+      named_bar_sync(2, kConvThreads);  // every row of the packed stage is read
+      expand(w, 2 * st + 1);
+      fence_proxy_async_smem();
+      mbar_arrive(&op_full[2 * st]);
+      mbar_arrive(&op_full[2 * st + 1]);
     }
     cluster_wait_acquire();    // B1
     cluster_arrive_release();  // B2
-    cluster_wait_acquire();
-  } else {
-    // ========================================================== MMA issuer
-    cluster_wait_acquire();    // B0
-    cluster_arrive_release();  // B1
-    cluster_wait_acquire();
-    cluster_arrive_release();  // B2
-    const uint32_t id_i8 = idesc_i8_s32(kBN);
-    const uint32_t id_bf = idesc_bf16_f32(kBN);
-    bool alive = mbar_wait(b_ready, 0u, p.status, abort_flag);
-    for (int i = 0; i < n_kb && alive; ++i) {
-      const int s = i % kNOPS;
-      if (!mbar_wait(&op_full[s], (uint32_t)(i / kNOPS) & 1u, p.status, abort_flag)) {
-        alive = false;
-        break;
-      }
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t da = sdesc_sw128(base + S_::kOpBase + s * S_::kOp);
-        const uint64_t db = sdesc_sw128(base + S_::kBBase + (uint32_t)(i * kBN * 128));
+    if (p.r > 0) mbar_arrive(lr_ready);
+    sw_tile[tid] = sw;         // read by the epilogue after B3
+    if (warp == kIssueWarp) {
+      // ======================================================== MMA issue
+      const uint32_t id_i8 = idesc_i8_s32(kBN);
+      const uint32_t id_bf = idesc_bf16_f32(kBN);
+      bool alive = mbar_wait(b_ready, 0u, p.status, abort_flag);
+      for (int i = 0; i < n_kb && alive; ++i) {
+        if (!mbar_wait(&op_full[i], 0u, p.status, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t da = sdesc_sw128(base + S_::kOpBase + (uint32_t)i * S_::kOp);
+          const uint64_t db = sdesc_sw128(base + S_::kBBase + (uint32_t)(i * kBN * 128));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_i8(tmem_acc, da + 2 * kk, db + 2 * kk, id_i8, (i > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&op_empty[s]);
+          for (int kk = 0; kk < 4; ++kk)
+            mma_i8(tmem_acc, da + 2 * kk, db + 2 * kk, id_i8, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
       }
+      if (alive && do_lr && mbar_wait(lr_ready, 0u, p.status, abort_flag)) {
+        tc_fence_after();
+        if (lane == 0) {
+          const uint64_t da = sdesc_sw128(base + S_::kLrABase);
+          const uint64_t db = sdesc_sw128(base + S_::kLrBBase);
+          for (int kk = 0; kk < p.r / 16; ++kk)
+            mma_bf16(tmem_lr, da + 2 * kk, db + 2 * kk, id_bf, kk > 0 ? 1u : 0u);
+        }
+        __syncwarp();
+      }
+      if (lane == 0) mma_commit(acc_full);
       __syncwarp();
     }
-    if (alive && do_lr && mbar_wait(lr_ready, 0u, p.status, abort_flag)) {
-      tc_fence_after();
-      if (lane == 0) {
-        const uint64_t da = sdesc_sw128(base + S_::kOpBase + (uint32_t)(n_kb % kNOPS) * S_::kOp);
-        const uint64_t db = sdesc_sw128(base + S_::kLrBBase);
-        for (int kk = 0; kk < p.r / 16; ++kk)
-          mma_bf16(tmem_lr, da + 2 * kk, db + 2 * kk, id_bf, kk > 0 ? 1u : 0u);
-      }
-      __syncwarp();
-    }
-    if (lane == 0) mma_commit(acc_full);
-    __syncwarp();
     cluster_wait_acquire();  // B2
   }
 
@@ -595,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == kIssueWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_acc, kTmemCols);
   }
