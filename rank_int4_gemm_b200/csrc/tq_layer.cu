@@ -3,28 +3,35 @@
 //   Y = dequant( Q4(X H) . Q4(H^T R) ) + bf16(X L1) L2
 //
 // Per output tile of 128 channels, a cluster of S CTAs splits K (split-K);
-// CTA z owns k-blocks [z*kbps, ...) of K, at most 1024 columns.  Its warps:
+// CTA z owns k-blocks [z*kbps, ...) of K, at most 8 blocks of 128 columns.
 //
-//   warps 0-15  activation, warp t = token t: the token's slice of X is
-//               staged once in shared memory; Sylvester transform (the warp
-//               butterflies of tq_quantize_act, so the codes are the same
-//               bits) and partial absmax, exchanged across the cluster through
-//               distributed shared memory.  While that exchange completes
-//               the same warps compute the slice's X.L1 partial on mma.sync
-//               (L1^T fragments are fetched into registers while X lands)
-//               and push it to split 0; then the rotated values, kept in
-//               registers, become the codes, written as int8 (16 * code)
-//               straight into the MMA's B operand.  Warps 0-3 run the
+// The rotation runs on the tensor cores.  The slice of X is staged as a
+// 128-row bf16 operand whose row (t, j) = 8 t + j is token t's k-block j
+// (128 columns), so one kind::f16 MMA chain of M = N = K = 128 against the
+// block-diagonal Sylvester matrix (+-1 entries, Hadamard blocks of b <= 128
+// columns, generated in shared memory) gives every rotated value of the
+// slice, exact products accumulated in fp32, in TMEM.  The int4 weights are
+// expanded into TMEM as the integer MMA's A operand, so the expanded weights
+// never pass through shared memory.
+//
+//   warps 0-15  activation: stage X (cp.async), one thread issues the
+//               rotation MMAs; warp w reads TMEM lanes 32 (w % 4) .. (the
+//               rows of tokens 4 (w % 4) .. +3) and columns 32 (w / 4) ..;
+//               partial absmax per token, exchanged across the cluster
+//               through distributed shared memory; the rotated values, kept
+//               in registers, become the codes, written as int8 (16 * code)
+//               into the integer MMA's B operand.  Then the slice's X.L1
+//               partial on mma.sync (L1^T fragments fetched into registers
+//               while X lands), pushed to split 0.  Warps 0-3 run the
 //               epilogue.
-//   warps 16-19 expand the int4 weights into one int8 operand slot per
-//               k-block (the whole slice is requested at CTA start and lands
-//               packed in the odd slots), all before the token codes exist,
-//               so the MMAs run back to back.  In split 0 they also place the
-//               tile's L2^T rows (the low-rank A operand).
+//   warps 16-19 expand the streamed int4 weights (the whole slice is
+//               requested at CTA start) into TMEM; in split 0 they also place
+//               the tile's L2^T rows (the low-rank A operand).
 //   warp 16     also issues the weight TMAs in the prologue (before the
 //               kernel waits on its predecessor: weights never depend on it),
-//               allocates TMEM and issues the MMAs: kind::i8 for the codes,
-//               kind::f16 for the low-rank branch (split 0).
+//               allocates TMEM and issues the integer MMAs (kind::i8, A from
+//               TMEM, tokens as N = 16) and the low-rank MMAs (kind::f16,
+//               split 0).
 //
 // Cluster barriers, all threads of all CTAs in order: B0 (every CTA is
 // running), B1 (absmax partials delivered), B2 (X.L1 partials delivered),
@@ -55,18 +62,25 @@ constexpr int kNSTG = 4;           // TMA stages (2 k-blocks each): the whole sl
 constexpr int kMaxKb = 8;          // k-blocks per CTA (slice <= 1024 columns)
 constexpr int kMaxSplits = 4;      // split-K cluster size limit of this kernel
 constexpr int kMaxR = 32;          // low-rank width handled here
-constexpr int kE = 16;             // values per lane per warp pass
-constexpr int kW = 32 * kE;        // 512 columns per warp pass
+constexpr int kMaxB = 128;         // Hadamard block limit (one MMA row = one block)
+constexpr int kSplitCols = 512;    // a split covers a multiple of 4 k-blocks
 constexpr int kActWarps = 16, kConvWarps = 4;
 // the first converter warp also issues the prologue TMAs, owns the TMEM
-// allocation and issues the MMAs (20 warps: five per SM sub-partition, so each
-// thread may hold up to 96 registers)
+// allocation and issues the integer MMAs (20 warps: five per SM
+// sub-partition, so each thread may hold up to 96 registers)
 constexpr int kIssueWarp = kActWarps;
 constexpr int kThreads = (kActWarps + kConvWarps) * 32;
 constexpr int kActThreads = kActWarps * 32;
 constexpr int kConvThreads = kConvWarps * 32;
 constexpr int kEpiThreads = 128;
 constexpr int kMaxBPair = 8;       // X L1 k-step pairs per warp (B fragments held in registers)
+
+// TMEM columns (512 allocated; one CTA per SM)
+constexpr uint32_t kColRot = 0;    // fp32 rotated slice, [128 rows (t, j)][128]
+constexpr uint32_t kColW = 128;    // int8 weights, 32 columns per k-block
+constexpr uint32_t kColAcc = 384;  // INT32 accumulator [16 tokens]
+constexpr uint32_t kColLr = 400;   // fp32 low-rank accumulator [16 tokens]
+constexpr uint32_t kTmemCols = 512;
 
 struct LayerParams {
   const __nv_bfloat16* X;    // [M][K]
@@ -80,37 +94,41 @@ struct LayerParams {
   float scale_mul;           // 1 / (7 sqrt(b))
 };
 
-// Shared-memory map (offsets from the 1024-aligned base).
+// Shared-memory map (offsets from the 1024-aligned base).  The two K halves
+// (64 columns each) of the 128-column operands are separate 128-byte
+// swizzled tiles.
 struct Smem {
-  // kMaxKb int8 weight k-blocks, one slot each; stage s (2 packed k-blocks,
-  // 128-byte swizzled rows) lands in slot 2s+1 and is expanded in place
-  static constexpr uint32_t kOp = kBM * 128;
-  static constexpr uint32_t kStg = kBM * 128;
-  static constexpr uint32_t kOpBase = 0;
-  static constexpr uint32_t kBBase = kOpBase + kMaxKb * kOp;  // token codes [kb][16][128]
+  static constexpr uint32_t kHalf = 128 * 128;               // [128 rows][128 B]
+  static constexpr uint32_t kXBase = 0;                      // X rows (t, j) [2][128][128 B]
+  // Hadamard tiles P, Q [64 rows][128 B] (Q = -P, used when b = 128)
+  static constexpr uint32_t kHTile = 64 * 128;
+  static constexpr uint32_t kHBase = kXBase + 2 * kHalf;
+  static constexpr uint32_t kStg = kBM * 128;                // one TMA stage (2 packed k-blocks)
+  static constexpr uint32_t kWBase = kHBase + 4 * kHTile;    // packed weights [kNSTG]
+  static constexpr uint32_t kBBase = kWBase + kNSTG * kStg;  // token codes [kb][16][128]
   static constexpr uint32_t kBBytes = kMaxKb * kBN * 128;
-  static constexpr uint32_t kLrBBase = kBBase + kBBytes;      // bf16(XL1) [16][64], SW128
-  static constexpr uint32_t kLrABase = (kLrBBase + kBN * 128 + 1023u) & ~1023u;  // L2^T [128][64]
-  static constexpr uint32_t kXBase = kLrABase + kBM * 128;    // X slice [16][1024] bf16, swizzled
-  static constexpr uint32_t kXRow = kMaxKb * kKB * 2;         // bytes per X row
-  static constexpr uint32_t kXBytes = kBN * kXRow;
+  static constexpr uint32_t kLrABase = kBBase + kBBytes;     // L2^T [128][128 B], SW128
+  static constexpr uint32_t kLrBBase = kLrABase + kBM * 128; // bf16(XL1) [16][128 B], SW128
   // split-K partials [S][16][rows] + low-rank [16][rows]; before the epilogue
   // the X L1 k-part partials [KP][16][r]
-  static constexpr uint32_t kKRecv = kXBase + kXBytes;
+  static constexpr uint32_t kKRecv = kLrBBase + kBN * 128;
   static constexpr uint32_t kKRecvBytes = 2 * kBN * kBM * 4;  // largest at S = 1
   static constexpr uint32_t kXRecv = kKRecv + kKRecvBytes;    // XL1 partials [S][16][r] fp32
   static constexpr uint32_t kXRecvBytes = kMaxSplits * kBN * kMaxR * 4;
-  static constexpr uint32_t kAmax = kXRecv + kXRecvBytes;     // [S][16] + [16]
-  static constexpr uint32_t kScale = kAmax + (kMaxSplits + 1) * kBN * 4;  // s_w [128]
+  static constexpr uint32_t kAmax = kXRecv + kXRecvBytes;     // [S][4][16] + [16]
+  static constexpr uint32_t kScale = kAmax + (kMaxSplits * 4 + 1) * kBN * 4;  // s_w [128]
   static constexpr uint32_t kBar = kScale + kBM * 4;
-  // barriers: stg_full[kNSTG], op_full[kMaxKb], b_ready, lr_ready, acc_full
-  static constexpr uint32_t kNumBars = kNSTG + kMaxKb + 3;
+  // barriers: stg_full[kNSTG], rot_full, w_full, b_ready, lr_ready, acc_full, h_ready
+  static constexpr uint32_t kNumBars = kNSTG + 6;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kMisc + 32;
   static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 static_assert(Smem::kAlloc <= 227 * 1024, "fused layer shared memory");
 static_assert(kActWarps * kBN * 8 * 4 <= Smem::kKRecvBytes, "X L1 k-part partials");
+static_assert(Smem::kWBase % 1024 == 0 && Smem::kBBase % 1024 == 0 &&
+                  Smem::kLrABase % 1024 == 0 && Smem::kLrBBase % 1024 == 0,
+              "1024-byte aligned operand tiles");
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -150,35 +168,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
-__device__ __forceinline__ uint32_t ldg_u32(const __nv_bfloat16* p) {
-  return __ldg(reinterpret_cast<const unsigned int*>(p));
-}
 __device__ __forceinline__ int owned_lo(int o, int S) { return (o * kBM + S - 1) / S; }
 
 // 16-byte chunk j (0..7) of row `row` of a 128-byte-swizzled K-major tile.
 __device__ __forceinline__ uint32_t sw_off(uint32_t row, uint32_t j) {
   return row * 128u + ((j ^ (row & 7u)) << 4);
 }
-// 16-byte chunk c (0..127) of row `row` (0..15) of the staged X slice; the
-// chunk index is XORed with the row so that the 8 rows of an ldmatrix land
-// in different banks.
-__device__ __forceinline__ uint32_t x_off(uint32_t row, uint32_t c) {
-  return row * Smem::kXRow + ((c ^ (row & 7u)) << 4);
-}
-
-// This lane's kE = 16 consecutive values of token `row`, columns
-// col0 .. col0 + 15 of the staged slice, as fp32.
-__device__ __forceinline__ void load_x16(uint32_t xbase, int row, int col0, float (&v)[kE]) {
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint4 u = ld_shared_v4(xbase + x_off((uint32_t)row, (uint32_t)(col0 / 8 + h)));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      v[8 * h + 2 * j] = __uint_as_float(w[j] << 16);
-      v[8 * h + 2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
-    }
-  }
+// 16-byte chunk q (0..127: columns 8q .. 8q+7 of the slice) of token t in
+// the staged X operand: row 8t + q/16 (k-block), K half (q/8) & 1.
+__device__ __forceinline__ uint32_t xa_off(uint32_t t, uint32_t q) {
+  return ((q >> 3) & 1u) * Smem::kHalf + sw_off(t * 8u + (q >> 4), q & 7u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -191,14 +190,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S_::kBar);
   uint64_t* stg_full = bars;
-  uint64_t* op_full = bars + kNSTG;
-  uint64_t* b_ready = op_full + kMaxKb;
-  uint64_t* lr_ready = b_ready + 1;
-  uint64_t* acc_full = b_ready + 2;
+  uint64_t* rot_full = bars + kNSTG;
+  uint64_t* w_full = rot_full + 1;
+  uint64_t* b_ready = rot_full + 2;
+  uint64_t* lr_ready = rot_full + 3;
+  uint64_t* acc_full = rot_full + 4;
+  uint64_t* h_ready = rot_full + 5;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S_::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S_::kMisc + 4);
-  const uint32_t amax_all = base + S_::kAmax;                 // [S][16] fp32
-  const uint32_t amax_row = amax_all + kMaxSplits * kBN * 4;  // [16] fp32
+  const uint32_t amax_all = base + S_::kAmax;                     // [S][4][16] fp32
+  const uint32_t amax_row = amax_all + kMaxSplits * 4 * kBN * 4;  // [16] fp32
   float* sw_tile = reinterpret_cast<float*>(smem + S_::kScale);
 
   const int warp = threadIdx.x >> 5;
@@ -211,24 +212,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int kbase = kb0 * kKB;           // first column of this CTA's slice
   const int slice = n_kb * kKB;          // 512 or 1024 columns
   const bool do_lr = p.r > 0 && split == 0;
-  constexpr uint32_t kTmemCols = 32;     // INT32 [16] + fp32 low-rank [16]
 
   pdl_launch_dependents();  // the next layer may start staging its weights
   // ---------------------------------------------------------------- prologue
   if (warp == kIssueWarp && lane == 0) {
     for (int i = 0; i < kNSTG; ++i) mbar_init(&stg_full[i], 1);
-    for (int i = 0; i < kMaxKb; ++i) mbar_init(&op_full[i], kConvThreads);
+    mbar_init(rot_full, 1);
+    mbar_init(w_full, kConvThreads);
     mbar_init(b_ready, kActThreads);
     mbar_init(lr_ready, kActThreads + kConvThreads);
     mbar_init(acc_full, 1);
+    mbar_init(h_ready, kConvThreads);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
     tma_prefetch_desc(&map_w);
     const uint64_t pol = policy_evict_first();
-    for (int i = 0; i < n_st; ++i) {  // the whole slice, into the odd slots
+    for (int i = 0; i < n_st; ++i) {  // the whole slice
       mbar_arrive_expect_tx(&stg_full[i], S_::kStg);
-      tma_load_2d(smem + S_::kOpBase + (2 * i + 1) * S_::kOp, &map_w, &stg_full[i],
+      tma_load_2d(smem + S_::kWBase + i * S_::kStg, &map_w, &stg_full[i],
                   (kb0 + i * kKBS) * kPackedRow, tile * kBM, pol);
     }
   }
@@ -240,8 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem_acc = *tmem_slot;
-  const uint32_t tmem_lr = tmem_acc + kBN;
+  const uint32_t tmem = *tmem_slot;
 
   if (warp < kActWarps) {
     // =================================================== activation warps
@@ -256,16 +257,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kspp = (slice / 16) / KP;
     pdl_wait();  // X comes from the preceding kernel
 
-    // ---- X slice [16][slice] -> shared memory (rows past M are zero)
+    // ---- X slice -> the rotation's A operand (rows of tokens past M are zero)
     const uint32_t xbase = base + S_::kXBase;
     {
-      const int cpr = slice / 8;  // 16-byte chunks per row
+      const int cpr = slice / 8;  // 16-byte chunks per token
       for (int ch = tid; ch < kBN * cpr; ch += kActThreads) {
-        const int row = ch / cpr, cc = ch - row * cpr;
+        const int row = ch / cpr, q = ch - row * cpr;
         const bool ok = row < p.M;
-        const __nv_bfloat16* src = p.X + (size_t)(ok ? row : 0) * p.K + kbase + cc * 8;
+        const __nv_bfloat16* src = p.X + (size_t)(ok ? row : 0) * p.K + kbase + q * 8;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
-                         xbase + x_off((uint32_t)row, (uint32_t)cc)),
+                         xbase + xa_off((uint32_t)row, (uint32_t)q)),
                      "l"(src), "r"(ok ? 16u : 0u)
                      : "memory");
       }
@@ -285,56 +286,113 @@ __global__ void __launch_bounds__(kThreads, 1)
         bq[i] = __ldg(reinterpret_cast<const uint4*>(
             p.L1t + (size_t)(nt * 8 + g) * p.K + kbase + 32 * (kp * kspp / 2 + i) + 8 * c));
     }
-    cp_async_wait<0>();
-    named_bar_sync(1, kActThreads);
-
-    // ---- transform of token `warp` over the slice (kept in registers),
-    //      partial absmax
-    const int np = slice / kW;  // 1 or 2 warp passes
-    float v[2][kE];
-    float amax = 0.f;
-#pragma unroll
-    for (int ps = 0; ps < 2; ++ps) {
-      if (ps < np) {
-        load_x16(xbase, warp, ps * kW + lane * kE, v[ps]);
-        fwht_warp<kE>(v[ps], p.b);
-#pragma unroll
-        for (int i = 0; i < kE; ++i) amax = fmaxf(amax, fabsf(v[ps][i]));
+    // ---- X rows of k-blocks past a short slice: zero (while X lands)
+    {
+      const int nz = kMaxKb - n_kb;  // k-blocks past the slice, per token
+      for (int ch = tid; ch < kBN * nz * 16; ch += kActThreads) {
+        const int t = ch / (nz * 16), rem = ch - t * nz * 16;
+        const int j = n_kb + (rem >> 4), cc = rem & 15;
+        st_shared_v4(base + S_::kXBase + (uint32_t)(cc >> 3) * S_::kHalf +
+                         sw_off((uint32_t)(t * 8 + j), (uint32_t)(cc & 7)),
+                     make_uint4(0u, 0u, 0u, 0u));
       }
     }
-    amax = warp_max(amax);
-    cluster_wait_acquire();  // B0 complete: every peer is running
-    if (lane < S)
-      dsmem_st_f32(dsmem_map(amax_all + (uint32_t)((split * kBN + warp) * 4), (uint32_t)lane), amax);
-    cluster_arrive_release();  // B1: this CTA's absmax partials delivered
-    cluster_wait_acquire();  // B1 complete
+    cp_async_wait<0>();
+    fence_proxy_async_smem();  // X and zero rows -> tensor core reads
+    named_bar_sync(1, kActThreads);
 
-    // ---- codes of token `warp` as the int8 B operand (16 * code: the code's
-    //      low nibble in the high nibble)
+    // ---- rotation: D[(t, j)][n] = sum_k X[t][128 j + k] H[k][n], in two
+    //      halves of 64 output columns.  For b = 128, H = [[P, P], [P, -P]]
+    //      with P the Sylvester matrix of order 64 (k or n >= 64 sets bit 6,
+    //      which adds 1 to popcount(n & k) only when both do); for b <= 64,
+    //      H = diag(P, P) with P block-diagonal, and the off-diagonal
+    //      quadrants are skipped.
+    if (tid == 0) {
+      mbar_wait(h_ready, 0u, p.status, abort_flag);
+      tc_fence_after();
+      const uint32_t id = idesc_bf16_f32(64);
+      const uint64_t dp = sdesc_sw128(base + S_::kHBase);
+      const uint64_t dq = sdesc_sw128(base + S_::kHBase + S_::kHTile);
+      const bool full = p.b == kMaxB;
+#pragma unroll
+      for (int nh = 0; nh < 2; ++nh) {
+        uint32_t acc = 0u;
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh) {
+          if (!full && kh != nh) continue;
+          const uint64_t da = sdesc_sw128(xbase + (uint32_t)kh * S_::kHalf);
+          const uint64_t db = (full && nh == 1 && kh == 1) ? dq : dp;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_bf16(tmem + kColRot + 64u * (uint32_t)nh, da + 2 * kk, db + 2 * kk, id, acc);
+            acc = 1u;
+          }
+        }
+      }
+      mma_commit(rot_full);
+    }
+    // this thread's row of D: token t, k-block j, columns 32 cq .. 32 cq + 31
+    const int q4 = warp & 3, cq = warp >> 2;
+    const int t = 4 * q4 + (lane >> 3), j = lane & 7;
+    float v[32];
+    {
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(rot_full, 0u, p.status, abort_flag));
+      tc_fence_after();
+      uint32_t u[32];
+      if (ok) {
+        tmem_ld32(tmem + kColRot + 32u * (uint32_t)cq + ((uint32_t)(32 * q4) << 16), u);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[i] = 0u;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]);
+    }
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    // over the token's 8 rows (lanes 8 (t % 4) ..)
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    cluster_wait_acquire();  // B0 complete: every peer is running
+    if (j < S)
+      dsmem_st_f32(dsmem_map(amax_all + (uint32_t)(((split * 4 + cq) * kBN + t) * 4), (uint32_t)j),
+                   amax);
+    cluster_arrive_release();  // B1: this CTA's absmax partials delivered
+    cluster_wait_acquire();    // B1 complete
+
+    // ---- codes of (t, j, columns 32 cq ..) as the int8 B operand (16 * code:
+    //      the code's low nibble in the high nibble)
     {
       float am = 0.f;
 #pragma unroll
       for (int z = 0; z < kMaxSplits; ++z)
-        if (z < S) am = fmaxf(am, ld_shared_f32(amax_all + (uint32_t)((z * kBN + warp) * 4)));
-      if (lane == 0) st_shared_f32(amax_row + (uint32_t)(warp * 4), am);
+        if (z < S)
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4)
+            am = fmaxf(am, ld_shared_f32(amax_all + (uint32_t)(((z * 4 + c4) * kBN + t) * 4)));
+      if (cq == 0 && j == 0) st_shared_f32(amax_row + (uint32_t)(t * 4), am);
       const CodeScale cs = code_scale(am);
+      if (cs.pre != 1.f) {
 #pragma unroll
-      for (int ps = 0; ps < 2; ++ps) {
-        if (ps < np) {
-          if (cs.pre != 1.f) {
+        for (int i = 0; i < 32; ++i) v[i] *= cs.pre;
+      }
+      if (j < n_kb) {
 #pragma unroll
-            for (int i = 0; i < kE; ++i) v[ps][i] *= cs.pre;
-          }
+        for (int h = 0; h < 2; ++h) {
           uint32_t w4[4];
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            w4[q] = (low_bytes4(code_bits(v[ps][4 * q], cs.inv), code_bits(v[ps][4 * q + 1], cs.inv),
-                                code_bits(v[ps][4 * q + 2], cs.inv), code_bits(v[ps][4 * q + 3], cs.inv))
+          for (int q = 0; q < 4; ++q) {
+            const float* x = v + 16 * h + 4 * q;
+            w4[q] = (low_bytes4(code_bits(x[0], cs.inv), code_bits(x[1], cs.inv),
+                                code_bits(x[2], cs.inv), code_bits(x[3], cs.inv))
                      << 4) &
                     0xF0F0F0F0u;
-          const int col = ps * kW + lane * kE;  // within the slice
-          const int kb = col / kKB, j = (col % kKB) / 16;
-          st_shared_v4(base + S_::kBBase + (uint32_t)(kb * kBN * 128) + sw_off((uint32_t)warp, (uint32_t)j),
+          }
+          st_shared_v4(base + S_::kBBase + (uint32_t)(j * kBN * 128) +
+                           sw_off((uint32_t)t, (uint32_t)(2 * cq + h)),
                        make_uint4(w4[0], w4[1], w4[2], w4[3]));
         }
       }
@@ -351,8 +409,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kMaxBPair; ++i) {
         if (2 * i < kspp) {
           const uint32_t q = (uint32_t)(4 * (kp * kspp / 2 + i) + c);  // 16-byte chunk of the slice
-          const uint4 x0 = ld_shared_v4(xbase + x_off((uint32_t)g, q));
-          const uint4 x8 = ld_shared_v4(xbase + x_off((uint32_t)(g + 8), q));
+          const uint4 x0 = ld_shared_v4(xbase + xa_off((uint32_t)g, q));
+          const uint4 x8 = ld_shared_v4(xbase + xa_off((uint32_t)(g + 8), q));
           const uint32_t a0[4] = {x0.x, x8.x, x0.y, x8.y}, b0[2] = {bq[i].x, bq[i].y};
           const uint32_t a1[4] = {x0.z, x8.z, x0.w, x8.w}, b1[2] = {bq[i].z, bq[i].w};
           mma_16816(acc[0], a0, b0);
@@ -382,29 +440,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      into the low-rank B operand [16][64] (columns past r are zero)
     if (do_lr) {
       if (tid < kBN * 8) {
-        const int row = tid >> 3, j = tid & 7;
+        const int row = tid >> 3, jj = tid & 7;
         float f[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) f[e] = 0.f;
-        if (j * 8 < p.r) {
-          const uint32_t xr = base + S_::kXRecv + (uint32_t)((row * p.r + j * 8) * 4);
+        if (jj * 8 < p.r) {
+          const uint32_t xr = base + S_::kXRecv + (uint32_t)((row * p.r + jj * 8) * 4);
           for (int z = 0; z < S; ++z)
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               f[e] += ld_shared_f32(xr + (uint32_t)((z * kBN * p.r + e) * 4));
         }
-        st_shared_v4(base + S_::kLrBBase + sw_off((uint32_t)row, (uint32_t)j),
+        st_shared_v4(base + S_::kLrBBase + sw_off((uint32_t)row, (uint32_t)jj),
                      make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
                                 pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7])));
       }
       fence_proxy_async_smem();
     }
     if (p.r > 0) mbar_arrive(lr_ready);
-  } else if (warp < kActWarps + kConvWarps) {
+  } else {
     // ==================================================== weight converters
-    const int tid = threadIdx.x - kActThreads;  // 0..127
-    // split 0: the tile's L2^T row `tid` ([r] bf16, r <= 32: 4 chunks),
-    // fetched now and placed once its operand slot is free
+    const int tid = threadIdx.x - kActThreads;  // 0..127: channel row = TMEM lane
+    // split 0: the tile's L2^T row `tid` ([r] bf16, r <= 32: 4 chunks)
     uint4 l2row[kMaxR / 8];
     // the scale of channel `tid`, for the epilogue (stored after the loop, so
     // that no thread waits on this load early)
@@ -416,9 +473,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (do_lr && gn < p.N && j * 8 < p.r)
         l2row[j] = __ldg(reinterpret_cast<const uint4*>(p.L2t + (size_t)gn * p.r + j * 8));
     }
+    // the Hadamard tiles of the rotation (idle time: the weights are still
+    // in flight).  P[n][k] (n, k < 64) = (-1)^popcount(n & k & m) inside the
+    // diagonal blocks of min(b, 64) columns, m = min(b, 64) - 1; Q = -P.
+    // One 16-byte chunk (k = k0 .. k0+7, k0 % 8 == 0) at a time: for blocks
+    // of 8 or more columns the chunk lies in one block or none, and the
+    // parity of n & k splits into that of n & k0 and that of n & e
+    // (e = k - k0), read from an 8-entry pattern table indexed by n & 7.
+    {
+      const int bm = min(p.b, 64) - 1;
+      const int n_chunks = (p.b == kMaxB ? 2 : 1) * 64 * 8;
+      constexpr unsigned long long kParity8 = 0x963C5AF066CCAA00ull;  // byte m: bit e = parity(m & e)
+      for (int ch = tid; ch < n_chunks; ch += kConvThreads) {
+        const int q = ch >> 9, n = (ch >> 3) & 63, c8 = ch & 7;
+        const int k0 = c8 * 8;
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        if (bm >= 7) {
+          if (((n ^ k0) & ~bm) == 0) {
+            const uint32_t flip = ((__popc((unsigned)(n & k0 & bm)) & 1) ^ q) ? 0xFFu : 0u;
+            const uint32_t bits = ((uint32_t)(kParity8 >> (8 * (n & 7))) & 0xFFu) ^ flip;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = 0x3F803F80u | (((bits >> (2 * e)) & 1u) << 15) |
+                     (((bits >> (2 * e + 1)) & 1u) << 31);
+          }
+        } else {  // blocks of 1, 2 or 4 columns: element by element
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int k = k0 + e;
+            if (((n ^ k) & ~bm) == 0)
+              w[e >> 1] |= ((__popc((unsigned)(n & k & bm)) & 1) ? 0xBF80u : 0x3F80u) << (16 * (e & 1));
+          }
+        }
+        st_shared_v4(base + S_::kHBase + (uint32_t)q * S_::kHTile + sw_off((uint32_t)n, (uint32_t)c8),
+                     make_uint4(w[0], w[1], w[2], w[3]));
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(h_ready);
+    }
     cluster_wait_acquire();    // B0
     cluster_arrive_release();  // B1 (nothing to publish from these warps)
-    // split 0: the tile's L2^T rows -> the low-rank A operand
     if (do_lr) {
 #pragma unroll
       for (int j = 0; j < 8; ++j)
@@ -426,42 +520,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                      j < kMaxR / 8 ? l2row[j] : make_uint4(0u, 0u, 0u, 0u));
       fence_proxy_async_smem();
     }
-    // int4 -> int8, in place: each thread expands its row of the stage's
-    // first k-block into slot 2s, reads the second, and once all four warps
-    // have read the packed rows, writes the second into slot 2s+1
+    // int4 -> int8 into TMEM: row `tid` of each k-block becomes 32 columns of
+    // lane `tid` (column c holds codes 4c .. 4c+3 as 16 * code; within a
+    // 16-byte packed group, byte i holds code i in its low nibble and code
+    // i + 16 in its high nibble)
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const uint32_t x7 = (uint32_t)tid & 7u;
     for (int st = 0; st < n_st; ++st) {
-      if (!mbar_wait(&stg_full[st], 0u, p.status, abort_flag)) break;
-      const uint32_t x7 = (uint32_t)tid & 7u;
-      const uint32_t src = base + S_::kOpBase + (uint32_t)(2 * st + 1) * S_::kOp + (uint32_t)tid * 128u;
-      auto expand = [&](const uint4 (&w)[4], int slot) {
-        const uint32_t dst = base + S_::kOpBase + (uint32_t)slot * S_::kOp + (uint32_t)tid * 128u;
+      if (!__all_sync(0xffffffffu, mbar_wait(&stg_full[st], 0u, p.status, abort_flag))) break;
+      const uint32_t src = base + S_::kWBase + (uint32_t)st * S_::kStg + (uint32_t)tid * 128u;
+      uint4 w[8];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 lo, hi;
-          lo.x = (w[q].x << 4) & 0xF0F0F0F0u;
-          lo.y = (w[q].y << 4) & 0xF0F0F0F0u;
-          lo.z = (w[q].z << 4) & 0xF0F0F0F0u;
-          lo.w = (w[q].w << 4) & 0xF0F0F0F0u;
-          hi.x = w[q].x & 0xF0F0F0F0u;
-          hi.y = w[q].y & 0xF0F0F0F0u;
-          hi.z = w[q].z & 0xF0F0F0F0u;
-          hi.w = w[q].w & 0xF0F0F0F0u;
-          st_shared_v4(dst + (((uint32_t)(2 * q) ^ x7) << 4), lo);
-          st_shared_v4(dst + (((uint32_t)(2 * q + 1) ^ x7) << 4), hi);
+      for (int q = 0; q < 8; ++q) w[q] = ld_shared_v4(src + (((uint32_t)q ^ x7) << 4));
+#pragma unroll
+      for (int sub = 0; sub < kKBS; ++sub) {
+        if (st * kKBS + sub < n_kb) {
+          uint32_t e32[32];
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint4 ww = w[4 * sub + c4];
+            const uint32_t wv[4] = {ww.x, ww.y, ww.z, ww.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              e32[8 * c4 + e] = (wv[e] << 4) & 0xF0F0F0F0u;
+              e32[8 * c4 + 4 + e] = wv[e] & 0xF0F0F0F0u;
+            }
+          }
+          tmem_st32(tmem + kColW + 32u * (uint32_t)(st * kKBS + sub) + lane_off, e32);
         }
-      };
-      uint4 w[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)q ^ x7) << 4));
-      expand(w, 2 * st);  // slot 2s holds nothing yet
-#pragma unroll
-      for (int q = 0; q < 4; ++q) w[q] = ld_shared_v4(src + (((uint32_t)(4 + q) ^ x7) << 4));
-      named_bar_sync(2, kConvThreads);  // every row of the packed stage is read
-      expand(w, 2 * st + 1);
-      fence_proxy_async_smem();
-      mbar_arrive(&op_full[2 * st]);
-      mbar_arrive(&op_full[2 * st + 1]);
+      }
     }
+    tmem_st_wait();
+    tc_fence_before();
+    mbar_arrive(w_full);
     cluster_wait_acquire();    // B1
     cluster_arrive_release();  // B2
     if (p.r > 0) mbar_arrive(lr_ready);
@@ -470,19 +561,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ======================================================== MMA issue
       const uint32_t id_i8 = idesc_i8_s32(kBN);
       const uint32_t id_bf = idesc_bf16_f32(kBN);
-      bool alive = mbar_wait(b_ready, 0u, p.status, abort_flag);
-      for (int i = 0; i < n_kb && alive; ++i) {
-        if (!mbar_wait(&op_full[i], 0u, p.status, abort_flag)) {
-          alive = false;
-          break;
-        }
+      bool alive = mbar_wait(b_ready, 0u, p.status, abort_flag) &&
+                   mbar_wait(w_full, 0u, p.status, abort_flag) && !*abort_flag;
+      if (alive) {
         tc_fence_after();
         if (lane == 0) {
-          const uint64_t da = sdesc_sw128(base + S_::kOpBase + (uint32_t)i * S_::kOp);
-          const uint64_t db = sdesc_sw128(base + S_::kBBase + (uint32_t)(i * kBN * 128));
+          for (int i = 0; i < n_kb; ++i) {
+            const uint64_t db = sdesc_sw128(base + S_::kBBase + (uint32_t)(i * kBN * 128));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_i8(tmem_acc, da + 2 * kk, db + 2 * kk, id_i8, (i > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              mma_i8_tmem_a(tmem + kColAcc, tmem + kColW + 32u * (uint32_t)i + 8u * (uint32_t)kk,
+                            db + 2 * kk, id_i8, (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         __syncwarp();
       }
@@ -492,7 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t da = sdesc_sw128(base + S_::kLrABase);
           const uint64_t db = sdesc_sw128(base + S_::kLrBBase);
           for (int kk = 0; kk < p.r / 16; ++kk)
-            mma_bf16(tmem_lr, da + 2 * kk, db + 2 * kk, id_bf, kk > 0 ? 1u : 0u);
+            mma_bf16(tmem + kColLr, da + 2 * kk, db + 2 * kk, id_bf, kk > 0 ? 1u : 0u);
         }
         __syncwarp();
       }
@@ -515,8 +605,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if (ok) {
       uint32_t ai[16], af[16];
-      tmem_ld16(tmem_acc + t_row, ai);
-      if (do_lr) tmem_ld16(tmem_lr + t_row, af);
+      tmem_ld16(tmem + kColAcc + t_row, ai);
+      if (do_lr) tmem_ld16(tmem + kColLr + t_row, af);
       tmem_ld_wait();
       const uint32_t ob = dsmem_map(base + S_::kKRecv, (uint32_t)owner);
       const uint32_t dst_i = ob + (uint32_t)((split * kBN * rows_max + (row - lo_o)) * 4);
@@ -555,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kIssueWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem_acc, kTmemCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -563,8 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool layer_decode_supported(int M, int N, int K, int r, int had_block) {
   (void)N;
-  return M >= 1 && M <= kBN && r <= kMaxR && K % kW == 0 && had_block <= kW &&
-         K / kKB <= kMaxKb * kMaxSplits;
+  return M >= 1 && M <= kBN && r <= kMaxR && K % kSplitCols == 0 && had_block >= 1 &&
+         had_block <= kMaxB && K / kKB <= kMaxKb * kMaxSplits;
 }
 
 cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream) {
@@ -584,7 +674,7 @@ cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream) {
   p.kb_total = a.K / kKB;
   const int tiles = (a.N + kBM - 1) / kBM;
   // splits: about one CTA per SM, each split a whole number of 512-column
-  // warp passes (4 k-blocks) and at most kMaxKb k-blocks
+  // groups (4 k-blocks) and at most kMaxKb k-blocks
   int s = tuning().split_k;
   if (s <= 0) s = std::max(1, num_sms() / tiles);
   s = std::max(1, std::min(s, kMaxSplits));

@@ -18,7 +18,7 @@ def tq(cuda_ok):
 
 
 CASES = [
-    # name, M, K, N, r, b      (fused: M<=16, r<=64, K%512==0, K<=4096)
+    # name, M, K, N, r, b      (fused: M<=16, r<=32, K%512==0, K<=4096, b<=128)
     ("decode_m1", 1, 4096, 4096, 32, 128),
     ("decode_m3", 3, 4096, 4096, 32, 128),
     ("decode_m16", 16, 4096, 4096, 32, 128),
@@ -28,6 +28,8 @@ CASES = [
     ("rank64_block256", 16, 4096, 512, 64, 256),
     ("no_rotation", 2, 1024, 128, 32, 1),
     ("block2", 9, 1024, 384, 48, 2),
+    ("block16", 4, 1024, 256, 16, 16),
+    ("block64", 11, 2048, 384, 32, 64),
     # two-kernel path inside the same entry point
     ("fallback_m17", 17, 1024, 256, 32, 128),
     ("fallback_rank128", 8, 1024, 256, 128, 128),
