@@ -139,10 +139,11 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  *
  * i.e. tq_quantize_act followed by tq_w4a4_lr_gemm, with the same codes,
  * scales and tolerances.  At decode sizes (M <= 16, r <= 32, K % 512 == 0,
- * K <= 4096, had_block <= 512) it runs as ONE kernel: each split-K cluster
- * rotates and quantizes its own slice of X, exchanges the absmax and X L1
- * partials in distributed shared memory and feeds the codes straight to the
- * tensor cores, while the weights stream in (TwinQuant notes section 04.C:
+ * K <= 4096, had_block <= 128) it runs as ONE kernel: each split-K cluster
+ * rotates its own slice of X on the tensor cores, quantizes it, exchanges
+ * the absmax and X L1 partials in distributed shared memory and feeds the
+ * codes straight to the integer MMAs, while the weights stream in and are
+ * expanded into tensor memory (TwinQuant notes section 04.C:
  * the residual GEMM quantizes activations concurrently and both paths share
  * one epilogue).  For M > 128 with had_block <= 128 and r <= 128 it runs
  * tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte in the
