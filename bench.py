@@ -10,7 +10,9 @@ over 16 distinct layers, so the 16 x 9.2 MB of operands (147 MB) exceed the
 126 MB L2 and every layer streams its weights from HBM.  The offline weight
 packing is not part of a step.  A step is replayed as one CUDA graph.
 --workload prefill_gateup|prefill_down|large_gateup|large_down|sweep times
-tq_quantize_act + tq_w4a4_lr_gemm on the prefill and sweep shapes instead.
+tq_quantize_act + tq_w4a4_lr_gemm on the prefill and sweep shapes instead;
+--workload sweeps runs the roofline sweeps at K = N = 4096 (M from 1 to 8192
+at rank 64, rank from 0 to 512 at M = 4096) through tq_w4a4_lr_layer.
 
 Metric: algorithmic GB/s of the layer (X + L1^T + Wq + s_w + L2^T + Y bytes
 per layer), the decode roofline quantity; TOPS (2 M N K) is reported beside it.
@@ -57,7 +59,7 @@ def parse():
                     help="replay only the timed step graph (for a profiler); prints one status line")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill_gateup", "prefill_down", "large_gateup",
-                             "large_down", "sweep"],
+                             "large_down", "sweep", "sweeps"],
                     help="decode is the default workload; the others are the prefill "
                          "shapes, scored in TOPS against the dense INT8 peak")
     ap.add_argument("--rank", type=int, default=None, help="low-rank r override (sweep)")
@@ -435,9 +437,9 @@ def run_prefill(args, rank, world, local_rank, dist):
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
             "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev),
         })
-    # codes one per byte when the activation stage runs on tensor cores
-    # (b <= 128, r <= 128): the path tq_w4a4_lr_layer takes for M > 128
-    a8 = b <= 128 and r <= 128
+    # the kernels tq_w4a4_lr_layer runs for this shape (codes one per byte
+    # for M > 128 and b <= 128), timed here call by call
+    a8 = tq.tq_layer_path(M, N, K, r, b) == "codes_i8"
     torch.cuda.synchronize()
 
     def one(lay, ev=None, packed=not a8):
@@ -516,6 +518,95 @@ def run_prefill(args, rank, world, local_rank, dist):
         "clocks": clk.summary(),
     }
     return out
+
+
+SWEEP_M = (1, 4, 16, 64, 256, 1024, 4096, 8192)
+SWEEP_R = (0, 32, 64, 128, 256, 512)
+
+
+def run_sweeps(args, rank, world, local_rank, dist):
+    """The roofline sweeps at K = N = 4096, Hadamard block 128, through the
+    public layer entry tq_w4a4_lr_layer (whichever kernels it routes to): M
+    over SWEEP_M at rank 64 and rank over SWEEP_R at M = 4096.  Each point
+    replays one CUDA graph over enough distinct layers that the step's
+    operands exceed L2 (weights shared between points of the same rank, X
+    and Y per point).  Reports GB/s of algorithmic bytes and TOPS (2 M N K)
+    with their fractions of the measured HBM and INT8 peaks, the
+    memory-to-compute crossover (the smallest M whose INT8 fraction is above
+    its HBM fraction) and each rank's latency against rank 0."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = synth.CONFIGS["sweep"]
+    K, N, b = base.K, base.N, base.had_block
+    hbm, hbm_src = measured_peaks()
+    i8, i8_src = int8_peak(sustained=False)
+    pools = {}
+
+    def weights(r, n):
+        pool = pools.setdefault(r, [])
+        sh = base.with_(r=r)
+        while len(pool) < n:
+            w = synth.make_weights(sh, seed=replica_seed(rank) + 10 * len(pool), device="cuda")
+            Rt = w["Rt"].to(dev)
+            Wq, s_w = tq.tq_pack_weight(Rt, b)
+            del Rt
+            pool.append({"Wq": Wq, "s_w": s_w, "L1t": w["L1t"].to(dev) if r else None,
+                         "L2t": w["L2t"].to(dev) if r else None})
+        return pool[:n]
+
+    def point(M, r):
+        per_layer = layer_bytes(M, K, N, r)
+        L = max(2, min(16, -(-250_000_000 // per_layer)))
+        sh = base.with_(r=r)
+        lays = []
+        for i, w in enumerate(weights(r, L)):
+            lays.append(dict(w, X=synth.make_activations(sh, seed=replica_seed(rank) + 10 * i, M=M).to(dev),
+                             Y=torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                             ws=torch.zeros(tq.tq_layer_workspace_bytes(M, N, K, r),
+                                            dtype=torch.uint8, device=dev)))
+        torch.cuda.synchronize()
+
+        def step():
+            for l in lays:
+                tq.tq_w4a4_lr_layer(l["X"], l["L1t"], l["Wq"], l["s_w"], l["L2t"], b, Y=l["Y"],
+                                    workspace=l["ws"])
+        g = capture(torch, step)
+        ms = time_graph(torch, g, max(5, min(args.steps, 50)), max(3, args.warmup))
+        del g, lays
+        us = ms * 1e3 / L
+        gbs = per_layer / (us * 1e-6) / 1e9
+        tops = 2 * M * N * K / (us * 1e-6) / 1e12
+        return {"M": M, "r": r, "path": tq.tq_layer_path(M, N, K, r, b), "layers": L,
+                "us_per_layer": round(us, 3), "GB/s": round(gbs, 1), "TOPS": round(tops, 2),
+                "frac_hbm": round(gbs / hbm, 4), "frac_int8": round(tops / i8, 4)}
+
+    with ClockSampler(local_rank) as clk:
+        pts_m = [point(M, 64) for M in SWEEP_M]
+        pts_r = [p for p in pts_m if p["M"] == 4096] + [point(4096, r) for r in SWEEP_R if r != 64]
+    pts_r.sort(key=lambda p: p["r"])
+    r0 = next(p for p in pts_r if p["r"] == 0)["us_per_layer"]
+    for p in pts_r:
+        p["vs_rank0"] = round(p["us_per_layer"] / r0, 4)
+    cross = next((p["M"] for p in pts_m if p["frac_int8"] > p["frac_hbm"]), None)
+    ref = next(p for p in pts_m if p["M"] == 4096)
+    return {
+        "metric": METRIC, "value": ref["TOPS"], "unit": "TOPS", "n_gpus": world,
+        "steps": max(5, min(args.steps, 50)), "warmup": max(3, args.warmup),
+        "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int4", "data": "synthetic",
+        "config": {"workload": f"roofline sweeps: K = N = {K}, Hadamard block {b}; M over "
+                               f"{list(SWEEP_M)} at rank 64, rank over {list(SWEEP_R)} at M = 4096",
+                   "l2": "each point: distinct layers whose operands exceed L2"},
+        "sweep_m": pts_m, "sweep_r": pts_r, "crossover_M": cross,
+        "rank64_vs_rank0": next(p for p in pts_r if p["r"] == 64)["vs_rank0"],
+        "peaks": {"hbm_gbs": hbm, "hbm_source": hbm_src, "int8_tops": i8, "int8_source": i8_src},
+        "clocks": clk.summary(),
+    }
 
 
 # ------------------------------------------------------------ oracle (CPU)
@@ -612,6 +703,8 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     if args.workload == "decode":
         out = run_tq(args, rank, world, local_rank, dist)
+    elif args.workload == "sweeps":
+        out = run_sweeps(args, rank, world, local_rank, dist)
     else:
         out = run_prefill(args, rank, world, local_rank, dist)
     if rank == 0:

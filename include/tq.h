@@ -145,7 +145,7 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  * codes straight to the integer MMAs, while the weights stream in and are
  * expanded into tensor memory (TwinQuant notes section 04.C:
  * the residual GEMM quantizes activations concurrently and both paths share
- * one epilogue).  For M > 128 with had_block <= 128 and r <= 128 it runs
+ * one epilogue).  For M > 128 with had_block <= 128 it runs
  * tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte in the
  * workspace).  Other shapes run tq_quantize_act + tq_w4a4_lr_gemm, keeping
  * Xq, s_x and XL1 in the workspace.
@@ -164,6 +164,17 @@ TQ_API int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t,
                             void* stream);
 
 /*
+ * tq_layer_path -- which kernels tq_w4a4_lr_layer runs for a shape.  A host
+ * query: no device work, no CUDA call.  Returns TQ_PATH_FUSED (the one-kernel
+ * decode layer), TQ_PATH_CODES_I8 (tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8),
+ * TQ_PATH_CODES_PACKED (tq_quantize_act + tq_w4a4_lr_gemm), or the negative
+ * of the tq_status tq_w4a4_lr_layer would return for the shape's arguments
+ * (TQ_ERR_INVALID_VALUE, TQ_ERR_UNSUPPORTED_SHAPE).
+ */
+enum { TQ_PATH_FUSED = 0, TQ_PATH_CODES_I8 = 1, TQ_PATH_CODES_PACKED = 2 };
+TQ_API int tq_layer_path(int M, int N, int K, int r, int had_block);
+
+/*
  * tq_quantize_act_i8 -- tq_quantize_act for many tokens, with the codes one
  * per byte: the same rotation (CoQuant Eq. (3), block Hadamard), per-token
  * scale and RoundClip codes (CoQuant Eq. (1)) and the same X L1
@@ -178,7 +189,9 @@ TQ_API int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t,
  *   s_x  [M] fp32      out : per-token scales
  *   XL1b [M][r] bf16   out : bf16(X L1) (round to nearest even), the
  *                            low-rank GEMM operand; NULL iff r == 0
- * Limits: had_block <= 128, r <= 128 (else TQ_ERR_UNSUPPORTED_SHAPE).
+ * Limits: had_block <= 128 (else TQ_ERR_UNSUPPORTED_SHAPE).  Ranks above 128
+ * run the codes and X L1 as separate launches (X L1 in launches of at most
+ * 256 columns) on the same stream.
  */
 TQ_API int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block,
                               const uint16_t* L1t, int r,

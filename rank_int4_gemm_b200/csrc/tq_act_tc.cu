@@ -38,7 +38,8 @@ constexpr int kTok = 128;          // tokens per tile (MMA M)
 constexpr int kBlk = 128;          // columns per block (MMA N of the rotation, MMA K)
 constexpr int kNS = 2;             // X / L1^T stages
 constexpr int kMaxC = 8;           // CTAs per cluster along K
-constexpr int kMaxRtc = 128;       // X L1 width handled here
+constexpr int kMaxRtc = 128;       // X L1 width computed beside the codes
+constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
 constexpr int kThreadsTc = 192;
 constexpr int kEpiFirstWarp = 2;
 constexpr int kEpiThreadsTc = 128;
@@ -49,31 +50,40 @@ struct TcParams {
   float* s_x;        // [M]
   float* XL1;        // [M][r] fp32, or null
   __nv_bfloat16* XL1b;  // [M][r] rounded to bf16, or null
-  int M, K, b, r;
-  int kb_total, nb;  // 128-column blocks in K, blocks per CTA
-  float scale_mul;   // 1 / (7 sqrt(b))
+  int M, K, b, r;     // r: X L1 columns of this launch
+  int r_ld, r_off;    // row stride of XL1 / XL1b, first column (and L1^T row) of this launch
+  int xl1_only;       // X L1 only: no rotation, no codes, no s_x
+  int kb_total, nb;   // 128-column blocks in K, blocks per CTA
+  float scale_mul;    // 1 / (7 sqrt(b))
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Atoms are 128-byte
-// swizzled K-major tiles of 64 bf16 columns.
-struct TcSmem {
-  static constexpr uint32_t kH = 0;                         // Hd^T: 2 atoms x 128 rows
-  static constexpr uint32_t kHBytes = 2 * kBlk * 128;
-  static constexpr uint32_t kStage0 = kH + kHBytes;
-  static constexpr uint32_t kXBytes = 2 * kTok * 128;       // X block: 2 atoms x 128 rows
-  static constexpr uint32_t kL1Max = 2 * kMaxRtc * 128;     // L1^T block: 2 atoms x r rows
-  static constexpr uint32_t kStage = kXBytes + kL1Max;
-  static constexpr uint32_t kAmax = kStage0 + kNS * kStage; // [C][128] fp32
-  static constexpr uint32_t kBar = kAmax + kMaxC * kTok * 4;
-  // full[kNS], empty[kNS], rot_full[2], rot_empty[2], xl1_full
-  static constexpr uint32_t kNumBars = 2 * kNS + 5;
-  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
-  static constexpr uint32_t kBytes = kMisc + 16;
-  static constexpr uint32_t kAlloc = kBytes + 1024;
+// swizzled K-major tiles of 64 bf16 columns.  A stage holds one X block and,
+// when X L1 is computed, the matching L1^T block (2 atoms x r rows); an
+// X-L1-only launch has no Hadamard operand.
+constexpr int kNumBarsTc = 2 * kNS + 5;  // full[kNS], empty[kNS], rot_full[2], rot_empty[2], xl1_full
+struct TcLayout {
+  uint32_t h, stage0, stage, amax, bar, misc, bytes;
 };
-static_assert(TcSmem::kAlloc <= 227 * 1024, "activation tile shared memory");
-// the X L1 receive area [C][128][ceil(r/C)] reuses the stages after pass 2
-static_assert(kTok * (kMaxRtc + kMaxC) * 4 <= kNS * TcSmem::kStage, "X L1 receive area");
+__host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
+  TcLayout L;
+  L.h = 0;                                             // Hd^T: 2 atoms x 128 rows
+  L.stage0 = xl1_only ? 0u : 2u * kBlk * 128u;
+  L.stage = 2u * kTok * 128u + (uint32_t)r * 256u;     // X block + L1^T block
+  L.amax = L.stage0 + kNS * L.stage;                   // [C][128] fp32
+  L.bar = L.amax + kMaxC * kTok * 4u;
+  L.misc = L.bar + kNumBarsTc * 8u;
+  L.bytes = L.misc + 16u;
+  return L;
+}
+static_assert(2u * kBlk * 128u + kNS * (2u * kTok * 128u + kMaxRtc * 256u) + kMaxC * kTok * 4u +
+                      kNumBarsTc * 8u + 16u + 1024u <= 227u * 1024u,
+              "activation tile shared memory (codes)");
+static_assert(kNS * (2u * kTok * 128u + kMaxRx * 256u) + kMaxC * kTok * 4u + kNumBarsTc * 8u +
+                      16u + 1024u <= 227u * 1024u,
+              "activation tile shared memory (X L1 only)");
+// the X L1 receive area [C][128][ceil(r/C)] reuses the stages after pass 2:
+// 512 (r + C) bytes <= 2 (32 KB + 256 r) for every C <= 128
 
 __device__ __forceinline__ void st_shared_v4_tc(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y),
@@ -101,16 +111,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw_addr);
-  using L = TcSmem;
+  const TcLayout L = tc_layout(p.xl1_only != 0, p.r);
+  const bool xo = p.xl1_only != 0;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kNS;
   uint64_t* rot_full = bars + 2 * kNS;
   uint64_t* rot_empty = rot_full + 2;
   uint64_t* xl1_full = rot_full + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -140,7 +151,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   }
   // Hd^T as the B operand of the rotation: row j (output column), column k;
   // Hd is symmetric.  +-1 (or 0 off the diagonal blocks), unnormalised.
-  for (int ch = threadIdx.x; ch < kBlk * 16; ch += kThreadsTc) {
+  for (int ch = threadIdx.x; ch < (xo ? 0 : kBlk * 16); ch += kThreadsTc) {
     const int j = ch >> 4, c = ch & 15;
     uint32_t w[4];
 #pragma unroll
@@ -156,7 +167,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       }
       w[e] = two;
     }
-    st_shared_v4_tc(base + L::kH + atom_off((uint32_t)j, (uint32_t)c, kBlk),
+    st_shared_v4_tc(base + L.h + atom_off((uint32_t)j, (uint32_t)c, kBlk),
                     make_uint4(w[0], w[1], w[2], w[3]));
   }
   fence_proxy_async_smem();
@@ -181,21 +192,22 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       pdl_wait();  // X comes from the preceding kernel
       const uint64_t pol_x = policy_evict_last();    // read again in pass 2
       const uint64_t pol_w = policy_evict_first();
-      for (int i = 0; i < 2 * nb; ++i) {
+      const int n_loads = xo ? nb : 2 * nb;  // X-L1-only: one pass
+      for (int i = 0; i < n_loads; ++i) {
         const int s = i % kNS;
-        const bool second = i >= nb;
-        const int j = second ? i - nb : i;
+        const bool second = xo || i >= nb;
+        const int j = (xo || i < nb) ? i : i - nb;
         if (!mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, nullptr, abort_flag)) break;
-        const uint32_t st = base + L::kStage0 + (uint32_t)s * L::kStage;
+        const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
         const bool with_l1 = second && r > 0;
-        mbar_arrive_expect_tx(&full[s], L::kXBytes + (with_l1 ? l1_bytes : 0u));
+        mbar_arrive_expect_tx(&full[s], 2u * kTok * 128u + (with_l1 ? l1_bytes : 0u));
         const int x = (kb0 + j) * kBlk;
         tma_load_2d(smem + (st - base), &map_x, &full[s], x, tile * kTok, pol_x);
         tma_load_2d(smem + (st - base) + kTok * 128, &map_x, &full[s], x + 64, tile * kTok, pol_x);
         if (with_l1) {
-          tma_load_2d(smem + (st - base) + L::kXBytes, &map_l1, &full[s], x, 0, pol_w);
-          tma_load_2d(smem + (st - base) + L::kXBytes + (uint32_t)r * 128u, &map_l1, &full[s],
-                      x + 64, 0, pol_w);
+          const uint32_t l1 = (st - base) + 2u * kTok * 128u;
+          tma_load_2d(smem + l1, &map_l1, &full[s], x, p.r_off, pol_w);
+          tma_load_2d(smem + l1 + (uint32_t)r * 128u, &map_l1, &full[s], x + 64, p.r_off, pol_w);
         }
       }
     }
@@ -211,28 +223,33 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     cluster_arrive_rel();      // B1
     const uint32_t id_rot = idesc_bf16_f32(kBlk);
     const uint32_t id_xl1 = idesc_bf16_f32(r > 0 ? r : 16);
-    for (int i = 0; i < 2 * nb; ++i) {
+    const int n_loads = xo ? nb : 2 * nb;
+    for (int i = 0; i < n_loads; ++i) {
       const int s = i % kNS, u = i & 1;
-      const bool second = i >= nb;
-      const int j = second ? i - nb : i;
+      const bool second = xo || i >= nb;
+      const int j = (xo || i < nb) ? i : i - nb;
       if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, nullptr, abort_flag)) break;
-      if (!mbar_wait(&rot_empty[u], ((uint32_t)(i / 2) & 1u) ^ 1u, nullptr, abort_flag)) break;
+      if (!xo && !mbar_wait(&rot_empty[u], ((uint32_t)(i / 2) & 1u) ^ 1u, nullptr, abort_flag))
+        break;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t st = base + L::kStage0 + (uint32_t)s * L::kStage;
+        const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
           const uint32_t atom = (uint32_t)kk >> 2, ko = ((uint32_t)kk & 3u) * 2u;  // 32 B steps
           const uint64_t da = sdesc_sw128(st + atom * (kTok * 128u)) + ko;
-          const uint64_t dh = sdesc_sw128(base + L::kH + atom * (kBlk * 128u)) + ko;
-          mma_bf16(tmem_rot + (uint32_t)u * kBlk, da, dh, id_rot, kk > 0 ? 1u : 0u);
+          if (!xo) {
+            const uint64_t dh = sdesc_sw128(base + L.h + atom * (kBlk * 128u)) + ko;
+            mma_bf16(tmem_rot + (uint32_t)u * kBlk, da, dh, id_rot, kk > 0 ? 1u : 0u);
+          }
           if (second && r > 0) {
-            const uint64_t dl = sdesc_sw128(st + L::kXBytes + atom * ((uint32_t)r * 128u)) + ko;
+            const uint64_t dl =
+                sdesc_sw128(st + 2u * kTok * 128u + atom * ((uint32_t)r * 128u)) + ko;
             mma_bf16(tmem_xl1, da, dl, id_xl1, (j > 0 || kk > 0) ? 1u : 0u);
           }
         }
         mma_commit(&empty[s]);
-        mma_commit(&rot_full[u]);
+        if (!xo) mma_commit(&rot_full[u]);
       }
       __syncwarp();
     }
@@ -253,7 +270,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
     // ---- pass 1: partial absmax of this token over the CTA's slice
     float amax = 0.f;
-    for (int i = 0; i < nb; ++i) {
+    for (int i = 0; i < (xo ? 0 : nb); ++i) {
       const int u = i & 1;
       const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
                                                   abort_flag));
@@ -271,19 +288,20 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tc_fence_before();
       mbar_arrive(&rot_empty[u]);
     }
-    for (uint32_t z = 0; z < csize; ++z)
-      dsmem_st_f32(dsmem_map(base + L::kAmax + (crank * kTok + (uint32_t)row) * 4u, z), amax);
+    if (!xo)
+      for (uint32_t z = 0; z < csize; ++z)
+        dsmem_st_f32(dsmem_map(base + L.amax + (crank * kTok + (uint32_t)row) * 4u, z), amax);
     cluster_arrive_rel();  // B1: partial absmax delivered
     cluster_wait_acquire();
     float am = 0.f;
     for (uint32_t z = 0; z < csize; ++z)
-      am = fmaxf(am, ld_shared_f32_tc(base + L::kAmax + (z * kTok + (uint32_t)row) * 4u));
-    if (crank == 0 && grow < p.M) p.s_x[grow] = am * p.scale_mul;
+      am = fmaxf(am, ld_shared_f32_tc(base + L.amax + (z * kTok + (uint32_t)row) * 4u));
+    if (!xo && crank == 0 && grow < p.M) p.s_x[grow] = am * p.scale_mul;
     const CodeScale cs = code_scale(am);
 
     // ---- pass 2: the same rotation again -> codes in the packed layout
     //      (inside each 32-code group byte i = code i | code i+16 << 4)
-    for (int i = nb; i < 2 * nb; ++i) {
+    for (int i = nb; i < (xo ? nb : 2 * nb); ++i) {
       const int u = i & 1;
       const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
                                                   abort_flag));
@@ -338,7 +356,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // rows of the tile are split among the cluster: CTA o sums rows
     // [o rpo, (o+1) rpo); every CTA sends each row's partial to its owner
     const int rpo = (kTok + (int)csize - 1) / (int)csize;
-    const uint32_t recv = base + L::kStage0;  // [C senders][rpo][r] fp32
+    const uint32_t recv = base + L.stage0;  // [C senders][rpo][r] fp32
     if (r > 0 && xl1_ok) {
       tc_fence_after();
       const int owner = row / rpo;
@@ -378,14 +396,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           acc.w += t.w;
         }
         if (gr < p.M) {
-          if (p.XL1) *reinterpret_cast<float4*>(p.XL1 + (size_t)gr * r + c) = acc;
+          const size_t o = (size_t)gr * p.r_ld + p.r_off + c;
+          if (p.XL1) *reinterpret_cast<float4*>(p.XL1 + o) = acc;
           if (p.XL1b) {
             __nv_bfloat162 h0 = __floats2bfloat162_rn(acc.x, acc.y);
             __nv_bfloat162 h1 = __floats2bfloat162_rn(acc.z, acc.w);
             uint2 u;
             u.x = *reinterpret_cast<uint32_t*>(&h0);
             u.y = *reinterpret_cast<uint32_t*>(&h1);
-            *reinterpret_cast<uint2*>(p.XL1b + (size_t)gr * r + c) = u;
+            *reinterpret_cast<uint2*>(p.XL1b + o) = u;
           }
         }
       }
@@ -404,32 +423,42 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
 bool act_tc_supported(int M, int K, int had_block, int r) {
   (void)K;
-  return M >= 64 && had_block <= kBlk && r <= kMaxRtc;
+  return M >= 64 && had_block <= kBlk && r <= 2 * kMaxRx;
 }
 
-cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
-                          int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
-                          cudaStream_t stream) {
+namespace {
+
+// One launch: codes (+ X L1 columns [0, r) when r > 0), or, with xl1_only,
+// X L1 columns [r_off, r_off + r) alone.
+cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
+                              int r_total, int r_off, int r, bool xl1_only, uint8_t* Xq,
+                              int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
+                              cudaStream_t stream) {
   TcParams p{};
-  p.Xq = Xq;
-  p.Xq8 = Xq8;
+  p.Xq = xl1_only ? nullptr : Xq;
+  p.Xq8 = xl1_only ? nullptr : Xq8;
   p.s_x = s_x;
-  p.XL1 = XL1;
-  p.XL1b = reinterpret_cast<__nv_bfloat16*>(XL1b);
+  p.XL1 = r > 0 ? XL1 : nullptr;
+  p.XL1b = r > 0 ? reinterpret_cast<__nv_bfloat16*>(XL1b) : nullptr;
   p.M = M;
   p.K = K;
   p.b = had_block;
   p.r = r;
+  p.r_ld = r_total;
+  p.r_off = r_off;
+  p.xl1_only = xl1_only ? 1 : 0;
   p.kb_total = K / kBlk;
   p.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   const int tiles = (M + kTok - 1) / kTok;
+  const uint32_t smem_bytes = tc_layout(xl1_only, r).bytes + 1024u;
   static uint64_t attr_set = 0;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set >> dev & 1u)) {
+    const uint32_t most = std::max(tc_layout(false, kMaxRtc).bytes, tc_layout(true, kMaxRx).bytes) +
+                          1024u;
     cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)TcSmem::kAlloc);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
@@ -447,7 +476,7 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(Ce, tiles, 1);
     q.blockDim = dim3(kThreadsTc, 1, 1);
-    q.dynamicSmemBytes = TcSmem::kAlloc;
+    q.dynamicSmemBytes = smem_bytes;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
     qa[0].val.clusterDim.x = Ce;
@@ -468,8 +497,10 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
                        (uint64_t)K * 2, 64, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (r > 0) {
-    if (!encode_tiled_2d(&map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, (uint64_t)K, (uint64_t)r,
-                         (uint64_t)K * 2, 64, (uint32_t)r, CU_TENSOR_MAP_SWIZZLE_128B))
+    // all r_total rows of L1^T; a launch reads rows [r_off, r_off + r)
+    if (!encode_tiled_2d(&map_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L1t, (uint64_t)K,
+                         (uint64_t)r_total, (uint64_t)K * 2, 64, (uint32_t)r,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   } else {
     map_l1 = map_x;  // never read
@@ -477,7 +508,7 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, tiles, 1);
   cfg.blockDim = dim3(kThreadsTc, 1, 1);
-  cfg.dynamicSmemBytes = TcSmem::kAlloc;
+  cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -487,6 +518,30 @@ cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, quantize_act_tc_kernel, map_x, map_l1, p);
+}
+
+}  // namespace
+
+// Up to kMaxRtc X L1 columns are computed beside the codes, from the same
+// staged X.  Wider ranks (the tensor memory holds the rotation's two buffers
+// and 256 accumulator columns) run the codes alone, then X L1 in launches of
+// at most kMaxRx columns that skip the rotation.
+cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
+                          int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
+                          cudaStream_t stream) {
+  if (r <= kMaxRtc)
+    return launch_act_tc_one(X, M, K, had_block, L1t, r, 0, r, false, Xq, Xq8, s_x, XL1, XL1b,
+                             stream);
+  if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, nullptr, r, 0, 0, false, Xq, Xq8, s_x,
+                                        nullptr, nullptr, stream))
+    return e;
+  for (int off = 0; off < r; off += kMaxRx) {
+    const int w = std::min(kMaxRx, r - off);
+    if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, L1t, r, off, w, true, Xq, Xq8, s_x,
+                                          XL1, XL1b, stream))
+      return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace tq

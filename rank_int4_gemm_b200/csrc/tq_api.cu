@@ -146,7 +146,7 @@ int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block, const uin
   if (!X || !Xq8 || !s_x || M <= 0) return TQ_ERR_INVALID_VALUE;
   if (int s = check_k(K, had_block)) return s;
   if (int s = check_r(r)) return s;
-  if (had_block > 128 || r > 128) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if (had_block > 128) return TQ_ERR_UNSUPPORTED_SHAPE;
   if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1b != nullptr)) return TQ_ERR_INVALID_VALUE;
   if (!aligned16(X) || !aligned16(Xq8) || !aligned16(s_x) || (r > 0 && !aligned16(L1t)) ||
       (r > 0 && !aligned16(XL1b)))
@@ -191,7 +191,18 @@ int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x, const uint8_t* Wq, c
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static bool layer_uses_a8(int M, int r, int had_block) {
-  return tq::tuning().layer_a8 && M > 128 && had_block <= 128 && r <= 128;
+  (void)r;
+  return tq::tuning().layer_a8 && M > 128 && had_block <= 128;
+}
+
+int tq_layer_path(int M, int N, int K, int r, int had_block) {
+  if (M <= 0 || N <= 0) return -TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return -s;
+  if (int s = check_r(r)) return -s;
+  if (N < 8 || N % 8 != 0) return -TQ_ERR_UNSUPPORTED_SHAPE;
+  if (tq::layer_decode_supported(M, N, K, r, had_block)) return TQ_PATH_FUSED;
+  if (layer_uses_a8(M, r, had_block)) return TQ_PATH_CODES_I8;
+  return TQ_PATH_CODES_PACKED;
 }
 
 size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {

@@ -17,7 +17,7 @@ _LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 if not os.path.exists(_LIB_PATH):
     raise ImportError(
-        f"{_LIB_PATH} is missing: build it with `python -m rank_int4_gemm_b200.build_lib` "
+        f"{_LIB_PATH} is missing: build it with `python rank_int4_gemm_b200/build_lib.py` "
         "(there is no fallback implementation)")
 
 _lib = ctypes.CDLL(_LIB_PATH)
@@ -42,6 +42,8 @@ _lib.tq_w4a4_lr_gemm_noalloc.restype = _I
 _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
 _lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.tq_layer_path.restype = _I
+_lib.tq_layer_path.argtypes = [_I, _I, _I, _I, _I]
 _lib.tq_w4a4_lr_layer.restype = _I
 _lib.tq_w4a4_lr_layer.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
                                   ctypes.c_size_t, _P]
@@ -251,6 +253,18 @@ def tq_query_device_status(workspace, stream=None) -> int:
 
 def tq_layer_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
     return int(_lib.tq_layer_workspace_bytes(M, N, K, r))
+
+
+LAYER_PATHS = {0: "fused", 1: "codes_i8", 2: "codes_packed"}
+
+
+def tq_layer_path(M: int, N: int, K: int, r: int, had_block: int) -> str:
+    """Which kernels tq_w4a4_lr_layer runs for this shape (host query):
+    "fused", "codes_i8" or "codes_packed"; raises on a shape it rejects."""
+    v = int(_lib.tq_layer_path(M, N, K, r, had_block))
+    if v < 0:
+        raise TQError(-v, "tq_layer_path")
+    return LAYER_PATHS[v]
 
 
 def tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None, stream=None):

@@ -90,3 +90,30 @@ def test_no_device_is_reported(lib):
     # Valid-looking arguments pass validation, then the device check fails
     # (this container has no GPU), so nothing is launched.
     assert lib.tq_pack_weight(P(FAKE), 8, 256, 128, P(FAKE), P(FAKE), None) == 7
+
+
+def test_layer_path_routing():
+    """tq_layer_path is a host query (runs without a GPU): the one-kernel
+    decode layer where its limits hold (M <= 16, r <= 32, K % 512 == 0,
+    K <= 4096, Hadamard block <= 128), int8 codes for M > 128 with block
+    <= 128, packed codes otherwise; rejected shapes raise."""
+    import rank_int4_gemm_b200 as tq
+    p = tq.tq_layer_path
+    assert p(16, 4096, 4096, 32, 128) == "fused"
+    assert p(1, 4096, 4096, 0, 128) == "fused"
+    assert p(16, 4096, 4096, 32, 1) == "fused"
+    assert p(17, 4096, 4096, 32, 128) == "codes_packed"
+    assert p(16, 4096, 4096, 64, 128) == "codes_packed"
+    assert p(16, 8192, 4096, 32, 128) == "fused"        # N does not limit it
+    assert p(16, 4096, 4608, 32, 128) == "codes_packed"  # K > 4096
+    assert p(16, 4096, 384, 16, 128) == "codes_packed"   # K % 512 != 0
+    assert p(16, 4096, 4096, 32, 256) == "codes_packed"  # block > 128
+    assert p(128, 4096, 4096, 64, 128) == "codes_packed"
+    assert p(129, 4096, 4096, 64, 128) == "codes_i8"
+    assert p(4096, 4096, 4096, 128, 128) == "codes_i8"
+    assert p(4096, 4096, 4096, 512, 128) == "codes_i8"
+    assert p(4096, 4096, 4096, 64, 256) == "codes_packed"
+    for bad in [(0, 4096, 4096, 32, 128), (16, 4096, 4000, 32, 128), (16, 4096, 4096, 24, 128),
+                (16, 12, 4096, 32, 128)]:
+        with pytest.raises(tq.TQError):
+            p(*bad)

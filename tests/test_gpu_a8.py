@@ -29,6 +29,10 @@ SHAPES = [
     ("block2", 129, 256, 16, 16, 2),
     ("tiny_n", 150, 256, 8, 0, 128),
     ("no_rotation", 700, 640, 392, 32, 1),
+    # ranks above 128: codes, then X L1 in launches of at most 256 columns
+    ("rank144", 130, 512, 256, 144, 128),
+    ("rank400", 257, 768, 512, 400, 64),
+    ("rank512", 150, 1024, 640, 512, 128),
 ]
 
 
@@ -98,9 +102,9 @@ def test_layer_entry_prefill(tq):
 
 def test_a8_argument_errors(tq):
     X = torch.zeros(256, 512, dtype=torch.bfloat16, device="cuda")
-    L1t = torch.zeros(256, 512, dtype=torch.bfloat16, device="cuda")
+    L1t = torch.zeros(528, 512, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(tq.TQError) as e:
-        tq.tq_quantize_act_i8(X, 128, L1t)  # r = 256 > 128
+        tq.tq_quantize_act_i8(X, 128, L1t)  # r = 528 > 512
     assert e.value.status == 2
     with pytest.raises(tq.TQError) as e:
         tq.tq_quantize_act_i8(X, 256)  # had_block 256 > 128

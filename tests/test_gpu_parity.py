@@ -62,8 +62,9 @@ SHAPES = [
 ]
 
 
-# tq_quantize_act on tensor cores (M >= 64, b <= 128, r <= 128): 128-token
-# tiles, ragged last tile, one and several CTAs along K, every block size
+# tq_quantize_act on tensor cores (M >= 64, b <= 128): 128-token tiles,
+# ragged last tile, one and several CTAs along K, every block size; ranks
+# above 128 (codes, then X L1 in launches of at most 256 columns)
 TC_SHAPES = [
     ("tc_min_m", 64, 256, 128, 16, 128),
     ("tc_ragged", 129, 1024, 136, 32, 128),
@@ -74,6 +75,8 @@ TC_SHAPES = [
     ("tc_block64", 70, 768, 128, 64, 64),
     ("tc_no_rotation", 65, 384, 64, 16, 1),
     ("tc_many_tiles", 1100, 1536, 256, 64, 128),
+    ("tc_rank256", 130, 1024, 384, 256, 128),
+    ("tc_rank304", 200, 512, 384, 304, 32),
 ]
 
 
