@@ -37,7 +37,7 @@ namespace {
 constexpr int kTok = 128;          // tokens per tile (MMA M)
 constexpr int kBlk = 128;          // columns per block (MMA N of the rotation, MMA K)
 constexpr int kNS = 2;             // X / L1^T stages
-constexpr int kMaxC = 8;           // CTAs per cluster along K
+constexpr int kMaxC = 16;          // CTAs per cluster along K (above 8: non-portable size)
 constexpr int kMaxRtc = 128;       // X L1 width computed beside the codes
 constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
 constexpr int kThreadsTc = 192;
@@ -133,6 +133,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const int r = p.r;
   const uint32_t l1_bytes = (uint32_t)r * 256u;         // one L1^T block, 2 atoms
 
+  // X (and L1^T) loads: one pass over the slice for X-L1-only launches and
+  // for CTAs of at most two blocks (whose rotations stay in the two TMEM
+  // buffers until the codes are written), two passes (absmax, then codes)
+  // otherwise
+  const bool resident = !xo && nb <= 2;
+  const int n_loads = (xo || resident) ? nb : 2 * nb;
+  auto issue_load = [&](int i, uint64_t pol_x, uint64_t pol_w) {
+    const int s = i % kNS;
+    const bool second = xo || resident || i >= nb;
+    const int j = i < nb ? i : i - nb;
+    const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
+    const bool with_l1 = second && r > 0;
+    mbar_arrive_expect_tx(&full[s], 2u * kTok * 128u + (with_l1 ? l1_bytes : 0u));
+    const int x = (kb0 + j) * kBlk;
+    tma_load_2d(smem + (st - base), &map_x, &full[s], x, tile * kTok, pol_x);
+    tma_load_2d(smem + (st - base) + kTok * 128, &map_x, &full[s], x + 64, tile * kTok, pol_x);
+    if (with_l1) {
+      const uint32_t l1 = (st - base) + 2u * kTok * 128u;
+      tma_load_2d(smem + l1, &map_l1, &full[s], x, p.r_off, pol_w);
+      tma_load_2d(smem + l1 + (uint32_t)r * 128u, &map_l1, &full[s], x + 64, p.r_off, pol_w);
+    }
+  };
+  const int n_pre = min(kNS, n_loads);  // stages requested in the prologue
+
   // ---------------------------------------------------------------- prologue
   if (warp == 0 && lane == 0) {
     for (int i = 0; i < kNS; ++i) {
@@ -148,27 +172,44 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     fence_barrier_init();
     tma_prefetch_desc(&map_x);
     if (r > 0) tma_prefetch_desc(&map_l1);
+    pdl_wait();  // X comes from the preceding kernel
+    // the first stages go out now, before the operand set-up below (their
+    // slots are free: nothing has used them yet)
+    for (int i = 0; i < n_pre; ++i) issue_load(i, policy_evict_last(), policy_evict_first());
   }
   // Hd^T as the B operand of the rotation: row j (output column), column k;
-  // Hd is symmetric.  +-1 (or 0 off the diagonal blocks), unnormalised.
-  for (int ch = threadIdx.x; ch < (xo ? 0 : kBlk * 16); ch += kThreadsTc) {
-    const int j = ch >> 4, c = ch & 15;
-    uint32_t w[4];
+  // Hd is symmetric.  +-1 (or 0 off the diagonal blocks), unnormalised.  One
+  // 16-byte chunk (k = k0 .. k0+7, k0 % 8 == 0) at a time: for b >= 8 the
+  // chunk lies in one block or none, and the parity of j & k splits into
+  // that of j & k0 and that of j & e (e = k - k0), read from an 8-entry
+  // pattern table indexed by j & 7.
+  {
+    const int bm = p.b - 1;
+    constexpr unsigned long long kParity8 = 0x963C5AF066CCAA00ull;  // byte m: bit e = parity(m & e)
+    for (int ch = threadIdx.x - 32; warp > 0 && ch < (xo ? 0 : kBlk * 16); ch += kThreadsTc - 32) {
+      const int j = ch >> 4, c = ch & 15;
+      const int k0 = c * 8;
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if (bm >= 7) {
+        if (((j ^ k0) & ~bm) == 0) {
+          const uint32_t flip = (__popc((unsigned)(j & k0 & bm)) & 1) ? 0xFFu : 0u;
+          const uint32_t bits = ((uint32_t)(kParity8 >> (8 * (j & 7))) & 0xFFu) ^ flip;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      uint32_t two = 0;
+          for (int e = 0; e < 4; ++e)
+            w[e] = 0x3F803F80u | (((bits >> (2 * e)) & 1u) << 15) |
+                   (((bits >> (2 * e + 1)) & 1u) << 31);
+        }
+      } else {  // blocks of 1, 2 or 4 columns: element by element
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int k = c * 8 + 2 * e + h;
-        uint32_t bits = 0;  // bf16 0
-        if (((j ^ k) & ~(p.b - 1)) == 0)  // same b-block
-          bits = (__popc((unsigned)(j & k & (p.b - 1))) & 1) ? 0xBF80u : 0x3F80u;
-        two |= bits << (16 * h);
+        for (int e = 0; e < 8; ++e) {
+          const int k = k0 + e;
+          if (((j ^ k) & ~bm) == 0)
+            w[e >> 1] |= ((__popc((unsigned)(j & k & bm)) & 1) ? 0xBF80u : 0x3F80u) << (16 * (e & 1));
+        }
       }
-      w[e] = two;
+      st_shared_v4_tc(base + L.h + atom_off((uint32_t)j, (uint32_t)c, kBlk),
+                      make_uint4(w[0], w[1], w[2], w[3]));
     }
-    st_shared_v4_tc(base + L.h + atom_off((uint32_t)j, (uint32_t)c, kBlk),
-                    make_uint4(w[0], w[1], w[2], w[3]));
   }
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -189,26 +230,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     cluster_wait_acquire();    // B0
     cluster_arrive_rel();      // B1 (nothing to publish)
     if (lane == 0) {
-      pdl_wait();  // X comes from the preceding kernel
       const uint64_t pol_x = policy_evict_last();    // read again in pass 2
       const uint64_t pol_w = policy_evict_first();
-      const int n_loads = xo ? nb : 2 * nb;  // X-L1-only: one pass
-      for (int i = 0; i < n_loads; ++i) {
-        const int s = i % kNS;
-        const bool second = xo || i >= nb;
-        const int j = (xo || i < nb) ? i : i - nb;
-        if (!mbar_wait(&empty[s], ((uint32_t)(i / kNS) & 1u) ^ 1u, nullptr, abort_flag)) break;
-        const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
-        const bool with_l1 = second && r > 0;
-        mbar_arrive_expect_tx(&full[s], 2u * kTok * 128u + (with_l1 ? l1_bytes : 0u));
-        const int x = (kb0 + j) * kBlk;
-        tma_load_2d(smem + (st - base), &map_x, &full[s], x, tile * kTok, pol_x);
-        tma_load_2d(smem + (st - base) + kTok * 128, &map_x, &full[s], x + 64, tile * kTok, pol_x);
-        if (with_l1) {
-          const uint32_t l1 = (st - base) + 2u * kTok * 128u;
-          tma_load_2d(smem + l1, &map_l1, &full[s], x, p.r_off, pol_w);
-          tma_load_2d(smem + l1 + (uint32_t)r * 128u, &map_l1, &full[s], x + 64, p.r_off, pol_w);
-        }
+      for (int i = n_pre; i < n_loads; ++i) {
+        if (!mbar_wait(&empty[i % kNS], ((uint32_t)(i / kNS) & 1u) ^ 1u, nullptr, abort_flag))
+          break;
+        issue_load(i, pol_x, pol_w);
       }
     }
     __syncwarp();
@@ -223,11 +250,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     cluster_arrive_rel();      // B1
     const uint32_t id_rot = idesc_bf16_f32(kBlk);
     const uint32_t id_xl1 = idesc_bf16_f32(r > 0 ? r : 16);
-    const int n_loads = xo ? nb : 2 * nb;
     for (int i = 0; i < n_loads; ++i) {
       const int s = i % kNS, u = i & 1;
-      const bool second = xo || i >= nb;
-      const int j = (xo || i < nb) ? i : i - nb;
+      const bool second = xo || resident || i >= nb;
+      const int j = i < nb ? i : i - nb;
       if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, nullptr, abort_flag)) break;
       if (!xo && !mbar_wait(&rot_empty[u], ((uint32_t)(i / 2) & 1u) ^ 1u, nullptr, abort_flag))
         break;
@@ -302,9 +328,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     // ---- pass 2: the same rotation again -> codes in the packed layout
     //      (inside each 32-code group byte i = code i | code i+16 << 4)
     for (int i = nb; i < (xo ? nb : 2 * nb); ++i) {
-      const int u = i & 1;
-      const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
-                                                  abort_flag));
+      // resident: block i - nb is still in its buffer from pass 1
+      const int u = resident ? i - nb : (i & 1);
+      const bool ok = resident ? !*abort_flag
+                               : __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u,
+                                                             nullptr, abort_flag));
       tc_fence_after();
       if (ok) {
         const size_t blk = (size_t)(kb0 + i - nb);
@@ -459,6 +487,9 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
                           1024u;
     cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(quantize_act_tc_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
     attr_set |= uint64_t(1) << dev;
   }
