@@ -20,9 +20,10 @@
 // tokens and weights per stage, then the low-rank chunks (64 columns of
 // bf16(XL1) and L2^T per stage, kind::f16 into the low-rank accumulator).
 //
-// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-5:
+// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-9:
 // weight expansion into TMEM, then the epilogue of the tile (warp w owns
-// lanes 32*(w%4)..: channel rows).  No TMA multicast.
+// lanes 32*(w%4)..: channel rows; warps w and w+4 split the k-blocks and the
+// epilogue's token chunks).  No TMA multicast.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -36,15 +37,27 @@ namespace tq {
 namespace {
 
 constexpr int kCh = 128;           // channels per tile (MMA M)
-constexpr int kTk = 192;           // tokens per tile (MMA N)
+constexpr int kTkMax = 192;        // tokens per tile (MMA N)
 constexpr int kKb = 128;           // codes per k-block
 constexpr int kNS = 3;             // stages
-constexpr int kThreadsA8 = 192;
-constexpr int kConvThreadsA8 = 128;
-constexpr uint32_t kColAcc = 0;    // INT32 accumulator, kTk columns
-constexpr int kNA = 4;             // int8 weight k-blocks in TMEM (A operand buffers)
-constexpr uint32_t kColA = 192;    // kNA x 32 columns: one int8 weight k-block each
-constexpr uint32_t kColLr = 320;   // fp32 low-rank accumulator, kTk columns
+// warps 2-9 expand the weights and run the epilogue, two per TMEM lane
+// quarter: warps 2-5 take the first k-block of each stage, warps 6-9 the
+// second, and the two halves split the epilogue's token chunks
+constexpr int kConvWarpsA8 = 8;
+constexpr int kConvThreadsA8 = kConvWarpsA8 * 32;
+constexpr int kThreadsA8 = 64 + kConvThreadsA8;
+constexpr int kQuarterThreads = 128;  // one warp per lane quarter: the writers of a k-block
+constexpr uint32_t kColAcc = 0;    // INT32 accumulator, TK columns
+// TMEM (512 columns): INT32 accumulator [TK] | A operand buffers, 32 columns
+// each (one int8 weight k-block) | fp32 low-rank accumulator [TK]; a narrower
+// token tile leaves room for more weight buffers in flight.
+template <int TK>
+struct A8Tmem {
+  static constexpr int kNA = (512 - 2 * TK) / 32;  // 4, 6 or 8
+  static constexpr uint32_t kColA = TK;
+  static constexpr uint32_t kColLr = TK + 32 * kNA;
+  static_assert(kColLr + TK <= 512, "TMEM columns");
+};
 
 struct A8Params {
   const float* s_x;    // [M]
@@ -57,25 +70,25 @@ struct A8Params {
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
-// [2 k-blocks][192 rows][128 B] then packed weights [128 rows][128 B]
-// (2 k-blocks).  A low-rank stage holds bf16(XL1) [192][64] in the first token
+// [2 k-blocks][TK rows][128 B] then packed weights [128 rows][128 B]
+// (2 k-blocks).  A low-rank stage holds bf16(XL1) [TK][64] in the first token
 // sub-tile and L2^T [128][64] in the weight part.
+template <int TK>
 struct A8Smem {
-  static constexpr uint32_t kTokSub = kTk * 128;            // 24 KB
+  static constexpr uint32_t kTokSub = TK * 128;             // 24 KB at TK = 192
   static constexpr uint32_t kWBytes = kCh * 128;            // 16 KB
   static constexpr uint32_t kStage = 2 * kTokSub + kWBytes;  // 64 KB
   // epilogue transpose buffers, one per converter warp: [32 tokens][40 bf16]
   static constexpr uint32_t kYRow = 80;
   static constexpr uint32_t kYBuf = kNS * kStage;
-  static constexpr uint32_t kBar = kYBuf + 4 * 32 * kYRow;
+  static constexpr uint32_t kBar = kYBuf + kConvWarpsA8 * 32 * kYRow;
   // full[kNS], empty[kNS], a_full[kNA], a_empty[kNA], acc_full, acc_empty
-  static constexpr uint32_t kNumBars = 2 * kNS + 2 * kNA + 2;
+  static constexpr uint32_t kNumBars = 2 * kNS + 2 * A8Tmem<TK>::kNA + 2;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
 };
-static_assert(A8Smem::kAlloc <= 227 * 1024, "a8 GEMM shared memory");
-static_assert(A8Smem::kTokSub % 1024 == 0 && A8Smem::kStage % 1024 == 0, "1024-B aligned atoms");
+static_assert(A8Smem<kTkMax>::kAlloc <= 227 * 1024, "a8 GEMM shared memory");
 
 __device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
   uint4 v;
@@ -85,6 +98,7 @@ __device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
   return v;
 }
 
+template <int TK>
 __global__ void __launch_bounds__(kThreadsA8, 1)
     w4a4_lr_gemm_a8_kernel(const __grid_constant__ CUtensorMap map_t,   // tokens int8 [M][K]
                            const __grid_constant__ CUtensorMap map_w,   // weights [N][K/2]
@@ -95,7 +109,12 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw_addr);
-  using L = A8Smem;
+  using L = A8Smem<TK>;
+  constexpr int kNA = A8Tmem<TK>::kNA;
+  constexpr uint32_t kColA = A8Tmem<TK>::kColA;
+  constexpr uint32_t kColLr = A8Tmem<TK>::kColLr;
+  static_assert(TK % 32 == 0 && TK >= 128 && TK <= kTkMax, "token tile (the epilogue takes 32 tokens at a time)");
+  static_assert(L::kTokSub % 1024 == 0 && L::kStage % 1024 == 0, "1024-B aligned atoms");
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* full = bars;
@@ -116,7 +135,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       mbar_init(&empty[i], 1);
     }
     for (int i = 0; i < kNA; ++i) {
-      mbar_init(&a_full[i], kConvThreadsA8);
+      mbar_init(&a_full[i], kQuarterThreads);
       mbar_init(&a_empty[i], 1);
     }
     mbar_init(acc_full, 1);
@@ -161,8 +180,8 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
               pdl_wait();  // token codes come from the preceding kernel
               waited = true;
             }
-            tma_load_2d(sp, &map_t, &full[s], kb * kKb, tm * kTk, pol_t);
-            if (two) tma_load_2d(sp + L::kTokSub, &map_t, &full[s], (kb + 1) * kKb, tm * kTk, pol_t);
+            tma_load_2d(sp, &map_t, &full[s], kb * kKb, tm * TK, pol_t);
+            if (two) tma_load_2d(sp + L::kTokSub, &map_t, &full[s], (kb + 1) * kKb, tm * TK, pol_t);
           } else {
             const int c = st - p.n_st;  // 64-column low-rank chunk
             mbar_arrive_expect_tx(&full[s], L::kWBytes + L::kTokSub);
@@ -171,7 +190,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
               waited = true;
             }
             tma_load_2d(sp + 2 * L::kTokSub, &map_l2, &full[s], c * 64, tn * kCh, pol_w);
-            tma_load_2d(sp, &map_xb, &full[s], c * 64, tm * kTk, pol_t);
+            tma_load_2d(sp, &map_xb, &full[s], c * 64, tm * TK, pol_t);
           }
         }
       }
@@ -179,8 +198,8 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ========================================================== MMA issuer
-    const uint32_t id_i8 = idesc_i8_s32(kTk);
-    const uint32_t id_bf = idesc_bf16_f32(kTk);
+    const uint32_t id_i8 = idesc_i8_s32(TK);
+    const uint32_t id_bf = idesc_bf16_f32(TK);
     int it = 0, ab = 0, tcount = 0;
     bool alive = true;
     for (int tile = blockIdx.x; tile < p.tiles && alive && !*abort_flag;
@@ -234,6 +253,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
   } else {
     // =============================== weight expansion into TMEM, epilogue
     const int q = warp & 3;                          // TMEM lane quarter
+    const int half = (warp - 2) >> 2;                // which k-block of a stage
     const int row = q * 32 + lane;                   // channel row of the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t x7 = (uint32_t)row & 7u;
@@ -256,34 +276,30 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         }
         const uint32_t wrow = base + (uint32_t)s * L::kStage + 2 * L::kTokSub + (uint32_t)row * 128u;
         const int nsub = (2 * st + 1 < p.kb_total) ? 2 : 1;
-        uint4 w[2][4];
+        const bool mine = half < nsub;  // this half's k-block exists in the stage
+        uint4 w[4];
 #pragma unroll
-        for (int sub = 0; sub < 2; ++sub)
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4)
-            if (sub < nsub) w[sub][c4] = ld_shared_v4_a8(wrow + ((((uint32_t)(sub * 4 + c4)) ^ x7) << 4));
+        for (int c4 = 0; c4 < 4; ++c4)
+          if (mine) w[c4] = ld_shared_v4_a8(wrow + ((((uint32_t)(half * 4 + c4)) ^ x7) << 4));
         bool ok = true;
+        if (mine) {
+          uint32_t v[32];
 #pragma unroll
-        for (int sub = 0; sub < 2; ++sub) {
-          if (sub < nsub) {
-            uint32_t v[32];
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const uint32_t ww[4] = {w[c4].x, w[c4].y, w[c4].z, w[c4].w};
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-              const uint32_t ww[4] = {w[sub][c4].x, w[sub][c4].y, w[sub][c4].z, w[sub][c4].w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[8 * c4 + e] = (ww[e] << 4) & 0xF0F0F0F0u;
-                v[8 * c4 + 4 + e] = ww[e] & 0xF0F0F0F0u;
-              }
+            for (int e = 0; e < 4; ++e) {
+              v[8 * c4 + e] = (ww[e] << 4) & 0xF0F0F0F0u;
+              v[8 * c4 + 4 + e] = ww[e] & 0xF0F0F0F0u;
             }
-            const int u = (ab + sub) % kNA;
-            ok = ok && __all_sync(0xffffffffu, mbar_wait(&a_empty[u],
-                                                         ((uint32_t)((ab + sub) / kNA) & 1u) ^ 1u,
-                                                         p.status, abort_flag));
-            if (ok) {
-              tc_fence_after();
-              tmem_st32(tmem + kColA + 32u * (uint32_t)u + lane_off, v);
-            }
+          }
+          const int u = (ab + half) % kNA;
+          ok = __all_sync(0xffffffffu, mbar_wait(&a_empty[u],
+                                                 ((uint32_t)((ab + half) / kNA) & 1u) ^ 1u,
+                                                 p.status, abort_flag));
+          if (ok) {
+            tc_fence_after();
+            tmem_st32(tmem + kColA + 32u * (uint32_t)u + lane_off, v);
           }
         }
         if (!ok) {
@@ -292,7 +308,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        for (int sub = 0; sub < nsub; ++sub) mbar_arrive(&a_full[(ab + sub) % kNA]);
+        if (mine) mbar_arrive(&a_full[(ab + half) % kNA]);
         ab += nsub;
       }
       it += p.n_lr;  // low-rank stages go to the MMA only
@@ -305,11 +321,11 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       tc_fence_after();
       const uint32_t ybuf = base + L::kYBuf + (uint32_t)(warp - 2) * 32u * L::kYRow;
       const int gc0 = tn * kCh + q * 32;  // first channel of this warp
-      for (int j = 0; j < kTk / 32; ++j) {
+      for (int j = half; j < TK / 32; j += 2) {
         uint32_t a[32], l[32];
         tmem_ld32(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
         if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
-        const int t0 = tm * kTk + 32 * j;
+        const int t0 = tm * TK + 32 * j;
         const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
         tmem_ld_wait();
 #pragma unroll
@@ -348,6 +364,53 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 
 }  // namespace
 
+namespace {
+
+template <int TK>
+cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stream) {
+  p.tiles_m = (a.M + TK - 1) / TK;
+  p.tiles = p.tiles_m * ((a.N + kCh - 1) / kCh);
+  CUtensorMap map_t, map_w, map_xb, map_l2;
+  if (!encode_tiled_2d(&map_t, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq8, (uint64_t)a.K, (uint64_t)a.M,
+                       (uint64_t)a.K, 128, TK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tiled_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, (uint64_t)(a.K / 2),
+                       (uint64_t)a.N, (uint64_t)(a.K / 2), 128, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  if (a.r > 0) {
+    if (!encode_tiled_2d(&map_xb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.XL1b, (uint64_t)a.r,
+                         (uint64_t)a.M, (uint64_t)a.r * 2, 64, TK, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_tiled_2d(&map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L2t, (uint64_t)a.r,
+                         (uint64_t)a.N, (uint64_t)a.r * 2, 64, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  } else {
+    map_xb = map_t;  // never read
+    map_l2 = map_t;
+  }
+  static uint64_t attr_set = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(attr_set >> dev & 1u)) {
+    cudaError_t e = cudaFuncSetAttribute(w4a4_lr_gemm_a8_kernel<TK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)A8Smem<TK>::kAlloc);
+    if (e != cudaSuccess) return e;
+    attr_set |= uint64_t(1) << dev;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(std::min(p.tiles, num_sms()), 1, 1);
+  cfg.blockDim = dim3(kThreadsA8, 1, 1);
+  cfg.dynamicSmemBytes = A8Smem<TK>::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = tuning().pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel<TK>, map_t, map_w, map_xb, map_l2, p);
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   A8Params p{};
   p.s_x = a.s_x;
@@ -361,45 +424,10 @@ cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   p.kb_total = a.K / kKb;
   p.n_st = (p.kb_total + 1) / 2;
   p.n_lr = (a.r + 63) / 64;
-  p.tiles_m = (a.M + kTk - 1) / kTk;
-  p.tiles = p.tiles_m * ((a.N + kCh - 1) / kCh);
-  CUtensorMap map_t, map_w, map_xb, map_l2;
-  if (!encode_tiled_2d(&map_t, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Xq8, (uint64_t)a.K, (uint64_t)a.M,
-                       (uint64_t)a.K, 128, kTk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tiled_2d(&map_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wq, (uint64_t)(a.K / 2),
-                       (uint64_t)a.N, (uint64_t)(a.K / 2), 128, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
-  if (a.r > 0) {
-    if (!encode_tiled_2d(&map_xb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.XL1b, (uint64_t)a.r,
-                         (uint64_t)a.M, (uint64_t)a.r * 2, 64, kTk, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_tiled_2d(&map_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.L2t, (uint64_t)a.r,
-                         (uint64_t)a.N, (uint64_t)a.r * 2, 64, kCh, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
-  } else {
-    map_xb = map_t;  // never read
-    map_l2 = map_t;
-  }
-  static uint64_t attr_set = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(attr_set >> dev & 1u)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_lr_gemm_a8_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)A8Smem::kAlloc);
-    if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(p.tiles, num_sms()), 1, 1);
-  cfg.blockDim = dim3(kThreadsA8, 1, 1);
-  cfg.dynamicSmemBytes = A8Smem::kAlloc;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = tuning().pdl ? 1 : 0;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel, map_t, map_w, map_xb, map_l2, p);
+  // 128 x 192 tiles: narrower token tiles (160, 128; more TMEM left for
+  // weight buffers) were measured slower on every prefill shape but one,
+  // where they won by under 1 %
+  return launch_gemm_a8_tk<kTkMax>(a, p, stream);
 }
 
 }  // namespace tq
