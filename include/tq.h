@@ -175,6 +175,39 @@ enum { TQ_PATH_FUSED = 0, TQ_PATH_CODES_I8 = 1, TQ_PATH_CODES_PACKED = 2 };
 TQ_API int tq_layer_path(int M, int N, int K, int r, int had_block);
 
 /*
+ * Shared input, gate / up pair with a SwiGLU epilogue (the MLP's gate and
+ * up projections read the same X, so its rotation, codes and X L1 are
+ * computed once for both; TwinQuant notes section 04.C: one shared epilogue).
+ *
+ * tq_pack_gate_up -- offline: the two projections' packed operands (each as
+ * tq_pack_weight makes them, with rank r) as one layer of 2N channels:
+ *   Wq2  [2N][K/2] u8   row 2i = gate row i, row 2i+1 = up row i
+ *   s_w2 [2N] fp32      interleaved the same way
+ *   L1t2 [2r][K] bf16   gate L1^T rows, then up L1^T rows
+ *   L2t2 [2N][2r] bf16  row 2i = [gate L2^T row i, 0], row 2i+1 = [0, up row i]
+ * L1t_* / L2t_* / L1t2 / L2t2 are NULL iff r == 0; 2r <= 512.
+ *
+ * tq_w4a4_lr_gate_up -- Y[t][i] = bf16( silu(g) * u ), silu(g) = g / (1 + e^-g),
+ * with g and u the fp32 layer outputs (s_x s_w acc + lr, before any rounding)
+ * of gate channel i and up channel i.  One activation pass (codes one per
+ * byte, X L1 of rank r2 = 2r) and one int8-code GEMM over the 2N channels,
+ * whose epilogue pairs the two rows of each channel.
+ *   X [M][K] bf16, the pair from tq_pack_gate_up, Y [M][N] bf16 (out);
+ *   workspace >= tq_gate_up_workspace_bytes(M, N, K, r2), zero-filled before
+ *   first use.  Limits: had_block <= 128, N % 8 == 0, r2 % 32 == 0, r2 <= 512.
+ */
+TQ_API int tq_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
+                           const uint16_t* L2t_g, const uint8_t* Wq_u, const float* s_w_u,
+                           const uint16_t* L1t_u, const uint16_t* L2t_u, int N, int K, int r,
+                           uint8_t* Wq2, float* s_w2, uint16_t* L1t2, uint16_t* L2t2,
+                           void* stream);
+TQ_API size_t tq_gate_up_workspace_bytes(int M, int N, int K, int r2);
+TQ_API int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uint8_t* Wq2,
+                              const float* s_w2, const uint16_t* L2t2, int M, int N, int K,
+                              int r2, int had_block, uint16_t* Y, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/*
  * tq_quantize_act_i8 -- tq_quantize_act for many tokens, with the codes one
  * per byte: the same rotation (CoQuant Eq. (3), block Hadamard), per-token
  * scale and RoundClip codes (CoQuant Eq. (1)) and the same X L1

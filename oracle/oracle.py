@@ -178,3 +178,10 @@ def layer(X, L1t, L2t, Rt, b: int, round_mid: bool = True) -> dict:
     out.update(w)
     out.update({"acc": acc, "XL1": XL1, "lr": lr, "Y64": Y64, "Ybf16": round_bf16(Y64)})
     return out
+
+
+def swiglu(g, u) -> np.ndarray:
+    """silu(g) * u = g / (1 + exp(-g)) * u, elementwise in fp64: the gate /
+    up pair's output from the two layers' fp64 outputs."""
+    g, u = _f64(g), _f64(u)
+    return g / (1.0 + np.exp(-g)) * u

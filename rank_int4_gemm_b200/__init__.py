@@ -9,5 +9,6 @@ from .tq import (  # noqa: F401
     TQError, lib_path, tq_status_string, tq_version, tq_pack_weight, tq_quantize_act,
     tq_gemm_workspace_bytes, tq_w4a4_lr_gemm, tq_w4a4_lr_gemm_noalloc, tq_debug_w4a4_gemm_acc,
     tq_query_device_status, Workspace, layer_forward, tq_layer_workspace_bytes, tq_w4a4_lr_layer,
-    tq_quantize_act_i8, tq_w4a4_lr_gemm_a8, tq_layer_path,
+    tq_quantize_act_i8, tq_w4a4_lr_gemm_a8, tq_layer_path, tq_pack_gate_up,
+    tq_gate_up_workspace_bytes, tq_w4a4_lr_gate_up,
 )

@@ -407,6 +407,33 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
+// Gate / up pair as one layer (offline): row 2i of the pair is gate channel
+// i, row 2i+1 up channel i (packed codes and scales); the low-rank factors
+// stack along r, L1^T as [gate; up] (two copies) and L2^T block-diagonally:
+// row 2i = [gate L2^T row i, 0], row 2i+1 = [0, up L2^T row i].  One CTA per
+// row of the pair.
+__global__ void pack_gate_up_kernel(const uint8_t* __restrict__ Wq_g, const float* __restrict__ s_w_g,
+                                    const uint16_t* __restrict__ L2t_g,
+                                    const uint8_t* __restrict__ Wq_u, const float* __restrict__ s_w_u,
+                                    const uint16_t* __restrict__ L2t_u, int K, int r,
+                                    uint8_t* __restrict__ Wq2, float* __restrict__ s_w2,
+                                    uint16_t* __restrict__ L2t2) {
+  const int o = blockIdx.x, i = o >> 1;
+  const bool up = o & 1;
+  const uint4* src = reinterpret_cast<const uint4*>((up ? Wq_u : Wq_g) + (size_t)i * (K / 2));
+  uint4* dst = reinterpret_cast<uint4*>(Wq2 + (size_t)o * (K / 2));
+  for (int c = threadIdx.x; c < K / 32; c += blockDim.x) dst[c] = src[c];
+  if (threadIdx.x == 0) s_w2[o] = (up ? s_w_u : s_w_g)[i];
+  if (r > 0) {
+    const uint4* l2 = reinterpret_cast<const uint4*>((up ? L2t_u : L2t_g) + (size_t)i * r);
+    uint4* d2 = reinterpret_cast<uint4*>(L2t2 + (size_t)o * 2 * r);
+    for (int c = threadIdx.x; c < r / 4; c += blockDim.x) {  // 2r bf16 = r/4 chunks
+      const bool mine = up ? c >= r / 8 : c < r / 8;
+      d2[c] = mine ? l2[up ? c - r / 8 : c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
@@ -443,6 +470,24 @@ cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uin
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   pack_weight_kernel<<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
+                                const uint16_t* L2t_g, const uint8_t* Wq_u, const float* s_w_u,
+                                const uint16_t* L1t_u, const uint16_t* L2t_u, int N, int K, int r,
+                                uint8_t* Wq2, float* s_w2, uint16_t* L1t2, uint16_t* L2t2,
+                                cudaStream_t stream) {
+  if (r > 0) {
+    const size_t bytes = (size_t)r * K * 2;
+    if (cudaError_t e = cudaMemcpyAsync(L1t2, L1t_g, bytes, cudaMemcpyDeviceToDevice, stream))
+      return e;
+    if (cudaError_t e = cudaMemcpyAsync(L1t2 + (size_t)r * K, L1t_u, bytes,
+                                        cudaMemcpyDeviceToDevice, stream))
+      return e;
+  }
+  pack_gate_up_kernel<<<2 * N, 128, 0, stream>>>(Wq_g, s_w_g, L2t_g, Wq_u, s_w_u, L2t_u, K, r, Wq2,
+                                                  s_w2, L2t2);
   return cudaGetLastError();
 }
 

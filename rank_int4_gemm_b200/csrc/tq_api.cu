@@ -311,4 +311,76 @@ int tq_query_device_status(void* workspace, void* stream) {
   return TQ_OK;
 }
 
+// ------------------------------------------------------------- gate / up
+// Workspace of tq_w4a4_lr_gate_up: [status 256][Xq8 M*K][s_x 4M][XL1b 2M r2],
+// 256-aligned parts.
+size_t tq_gate_up_workspace_bytes(int M, int N, int K, int r2) {
+  (void)N;
+  if (M <= 0 || K <= 0 || r2 < 0) return 256;
+  return 256 + align256((size_t)M * K) + align256((size_t)M * 4) + align256((size_t)M * r2 * 2);
+}
+
+int tq_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
+                    const uint16_t* L2t_g, const uint8_t* Wq_u, const float* s_w_u,
+                    const uint16_t* L1t_u, const uint16_t* L2t_u, int N, int K, int r, uint8_t* Wq2,
+                    float* s_w2, uint16_t* L1t2, uint16_t* L2t2, void* stream) {
+  if (!Wq_g || !s_w_g || !Wq_u || !s_w_u || !Wq2 || !s_w2 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (2 * r > 512) return TQ_ERR_UNSUPPORTED_SHAPE;
+  const bool lr = r > 0;
+  if (lr != (L1t_g && L2t_g && L1t_u && L2t_u && L1t2 && L2t2) ||
+      (!lr && (L1t_g || L2t_g || L1t_u || L2t_u || L1t2 || L2t2)))
+    return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Wq_g) || !aligned16(Wq_u) || !aligned16(Wq2) ||
+      (lr && (!aligned16(L2t_g) || !aligned16(L2t_u) || !aligned16(L2t2) || !aligned16(L1t2))))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_pack_gate_up(Wq_g, s_w_g, L1t_g, L2t_g, Wq_u, s_w_u, L1t_u, L2t_u, N,
+                                           K, r, Wq2, s_w2, L1t2, L2t2,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uint8_t* Wq2,
+                       const float* s_w2, const uint16_t* L2t2, int M, int N, int K, int r2,
+                       int had_block, uint16_t* Y, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  if (!X || !Wq2 || !s_w2 || !Y || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r2)) return s;
+  if (had_block > 128 || N % 8 != 0 || r2 % 32 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r2 > 0) != (L1t2 != nullptr) || (r2 > 0) != (L2t2 != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Wq2) || !aligned16(s_w2) || !aligned16(Y) ||
+      (L1t2 && !aligned16(L1t2)) || (L2t2 && !aligned16(L2t2)) ||
+      (workspace && !aligned16(workspace)))
+    return TQ_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < tq_gate_up_workspace_bytes(M, N, K, r2))
+    return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int8_t* Xq8 = reinterpret_cast<int8_t*>(ws + 256);
+  float* s_x = reinterpret_cast<float*>(ws + 256 + align256((size_t)M * K));
+  uint16_t* XL1b = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(s_x) + align256((size_t)M * 4));
+  if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, L1t2, r2, nullptr, Xq8, s_x, nullptr,
+                                        r2 > 0 ? XL1b : nullptr, st))
+    return from_cuda(e);
+  tq::GemmA8Args a{};
+  a.Xq8 = Xq8;
+  a.s_x = s_x;
+  a.Wq = Wq2;
+  a.s_w = s_w2;
+  a.XL1b = r2 > 0 ? XL1b : nullptr;
+  a.L2t = L2t2;
+  a.M = M;
+  a.N = 2 * N;
+  a.K = K;
+  a.r = r2;
+  a.Y = Y;
+  a.ws = workspace;
+  a.swiglu = 1;
+  return from_cuda(tq::launch_gemm_a8(a, st));
+}
+
 }  // extern "C"
+

@@ -67,6 +67,7 @@ struct A8Params {
   int M, N, K, r;
   int kb_total, n_st, n_lr;  // k-blocks, k-block stages, low-rank stages per tile
   int tiles_m, tiles;        // token tiles, all tiles
+  int swiglu;                // Y[t][c] = silu(y[t][2c]) * y[t][2c+1], Y is [M][N/2]
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
@@ -328,24 +329,52 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         const int t0 = tm * TK + 32 * j;
         const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
         tmem_ld_wait();
+        if (!p.swiglu) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float y = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
-          if (p.r > 0) y += __uint_as_float(l[e]);
-          const __nv_bfloat16 h = __float2bfloat16_rn(y);
-          asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
-                       "h"(*reinterpret_cast<const unsigned short*>(&h))
-                       : "memory");
-        }
-        __syncwarp();
+          for (int e = 0; e < 32; ++e) {
+            float y = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
+            if (p.r > 0) y += __uint_as_float(l[e]);
+            const __nv_bfloat16 h = __float2bfloat16_rn(y);
+            asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
+                         "h"(*reinterpret_cast<const unsigned short*>(&h))
+                         : "memory");
+          }
+          __syncwarp();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int idx = lane + 32 * k;      // 32 token rows x 4 16-byte parts
-          const int e = idx >> 2, part = idx & 3;
-          const uint4 v = ld_shared_v4_a8(ybuf + (uint32_t)e * L::kYRow + (uint32_t)part * 16u);
-          const int t = t0 + e, c = gc0 + part * 8;
-          if (t < p.M && c < p.N)
-            *reinterpret_cast<uint4*>(p.Y + (size_t)t * p.N + c) = v;
+          for (int k = 0; k < 4; ++k) {
+            const int idx = lane + 32 * k;      // 32 token rows x 4 16-byte parts
+            const int e = idx >> 2, part = idx & 3;
+            const uint4 v = ld_shared_v4_a8(ybuf + (uint32_t)e * L::kYRow + (uint32_t)part * 16u);
+            const int t = t0 + e, c = gc0 + part * 8;
+            if (t < p.M && c < p.N)
+              *reinterpret_cast<uint4*>(p.Y + (size_t)t * p.N + c) = v;
+          }
+        } else {
+          // channel rows alternate gate (even lane) and up (odd lane): one
+          // shuffle pairs them; 16 output channels per warp, from gc0 / 2
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            float y = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
+            if (p.r > 0) y += __uint_as_float(l[e]);
+            const float up = __shfl_xor_sync(0xffffffffu, y, 1);
+            if (!(lane & 1)) {
+              const __nv_bfloat16 h = __float2bfloat16_rn(y / (1.f + expf(-y)) * up);
+              asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + (uint32_t)lane),
+                           "h"(*reinterpret_cast<const unsigned short*>(&h))
+                           : "memory");
+            }
+          }
+          __syncwarp();
+          const int n_out = p.N / 2;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int idx = lane + 32 * k;      // 32 token rows x 2 16-byte parts
+            const int e = idx >> 1, part = idx & 1;
+            const uint4 v = ld_shared_v4_a8(ybuf + (uint32_t)e * L::kYRow + (uint32_t)part * 16u);
+            const int t = t0 + e, c = gc0 / 2 + part * 8;
+            if (t < p.M && c < n_out)
+              *reinterpret_cast<uint4*>(p.Y + (size_t)t * n_out + c) = v;
+          }
         }
         __syncwarp();
       }
@@ -424,6 +453,7 @@ cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   p.kb_total = a.K / kKb;
   p.n_st = (p.kb_total + 1) / 2;
   p.n_lr = (a.r + 63) / 64;
+  p.swiglu = a.swiglu;
   // 128 x 192 tiles: narrower token tiles (160, 128; more TMEM left for
   // weight buffers) were measured slower on every prefill shape but one,
   // where they won by under 1 %

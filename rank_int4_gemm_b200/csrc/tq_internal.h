@@ -39,10 +39,16 @@ struct GemmA8Args {
   const uint16_t* XL1b;   // [M][r] bf16
   const uint16_t* L2t;    // [N][r] bf16
   int M, N, K, r;
-  uint16_t* Y;
+  uint16_t* Y;            // [M][N], or [M][N/2] with swiglu
   void* ws;               // status word at offset 0
+  int swiglu = 0;         // rows alternate gate / up: Y = silu(gate) * up
 };
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
+cudaError_t launch_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
+                                const uint16_t* L2t_g, const uint8_t* Wq_u, const float* s_w_u,
+                                const uint16_t* L1t_u, const uint16_t* L2t_u, int N, int K, int r,
+                                uint8_t* Wq2, float* s_w2, uint16_t* L1t2, uint16_t* L2t2,
+                                cudaStream_t stream);
 
 struct GemmArgs {
   const uint8_t* Xq;

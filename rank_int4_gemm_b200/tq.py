@@ -43,6 +43,13 @@ _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
 _lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_layer_path.restype = _I
+_lib.tq_pack_gate_up.restype = _I
+_lib.tq_pack_gate_up.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]
+_lib.tq_gate_up_workspace_bytes.restype = ctypes.c_size_t
+_lib.tq_gate_up_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.tq_w4a4_lr_gate_up.restype = _I
+_lib.tq_w4a4_lr_gate_up.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                                    ctypes.c_size_t, _P]
 _lib.tq_layer_path.argtypes = [_I, _I, _I, _I, _I]
 _lib.tq_w4a4_lr_layer.restype = _I
 _lib.tq_w4a4_lr_layer.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
@@ -281,6 +288,47 @@ def tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None, st
     _check(_lib.tq_w4a4_lr_layer(_ptr(X), _ptr(L1t) if r else None, _ptr(Wq), _ptr(s_w),
                                  _ptr(L2t) if r else None, M, N, K, r, int(had_block), _ptr(Y),
                                  _ptr(ws), ws.numel(), _stream(stream)), "tq_w4a4_lr_layer")
+    return Y
+
+
+def tq_pack_gate_up(Wq_g, s_w_g, L1t_g, L2t_g, Wq_u, s_w_u, L1t_u, L2t_u, stream=None):
+    """Gate and up projections (each packed by tq_pack_weight, rank r) as one
+    layer of 2N interleaved channels: returns (Wq2, s_w2, L1t2, L2t2)."""
+    N, Kh = Wq_g.shape
+    K = 2 * Kh
+    r = 0 if L1t_g is None else L1t_g.shape[0]
+    dev = Wq_g.device
+    Wq2 = torch.empty(2 * N, Kh, dtype=torch.uint8, device=dev)
+    s_w2 = torch.empty(2 * N, dtype=torch.float32, device=dev)
+    L1t2 = torch.empty(2 * r, K, dtype=torch.bfloat16, device=dev) if r else None
+    L2t2 = torch.empty(2 * N, 2 * r, dtype=torch.bfloat16, device=dev) if r else None
+    opt = lambda t: _ptr(t) if t is not None else None  # noqa: E731
+    _check(_lib.tq_pack_gate_up(_ptr(Wq_g), _ptr(s_w_g), opt(L1t_g), opt(L2t_g), _ptr(Wq_u),
+                                _ptr(s_w_u), opt(L1t_u), opt(L2t_u), N, K, r, _ptr(Wq2),
+                                _ptr(s_w2), opt(L1t2), opt(L2t2), _stream(stream)),
+           "tq_pack_gate_up")
+    return Wq2, s_w2, L1t2, L2t2
+
+
+def tq_gate_up_workspace_bytes(M: int, N: int, K: int, r2: int) -> int:
+    return int(_lib.tq_gate_up_workspace_bytes(M, N, K, r2))
+
+
+def tq_w4a4_lr_gate_up(X, L1t2, Wq2, s_w2, L2t2, had_block, Y=None, workspace=None, stream=None):
+    """silu(gate) * up from one pass over X: Y [M][N] bf16, N = Wq2 rows / 2."""
+    M, K = X.shape
+    N = Wq2.shape[0] // 2
+    r2 = 0 if L1t2 is None else L1t2.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=X.device)
+    if workspace is None:
+        workspace = Workspace(X.device)
+    need = tq_gate_up_workspace_bytes(M, N, K, r2)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_gate_up(_ptr(X), _ptr(L1t2) if r2 else None, _ptr(Wq2), _ptr(s_w2),
+                                   _ptr(L2t2) if r2 else None, M, N, K, r2, int(had_block),
+                                   _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
+           "tq_w4a4_lr_gate_up")
     return Y
 
 
