@@ -12,7 +12,10 @@ packing is not part of a step.  A step is replayed as one CUDA graph.
 --workload prefill_gateup|prefill_down|large_gateup|large_down|sweep times
 tq_quantize_act + tq_w4a4_lr_gemm on the prefill and sweep shapes instead;
 --workload sweeps runs the roofline sweeps at K = N = 4096 (M from 1 to 8192
-at rank 64, rank from 0 to 512 at M = 4096) through tq_w4a4_lr_layer.
+at rank 64, rank from 0 to 512 at M = 4096) through tq_w4a4_lr_layer;
+--workload gateup_swiglu times the MLP's gate and up projections as one
+shared-input pair with the SwiGLU epilogue (tq_w4a4_lr_gate_up) against the
+two projections as separate tq_w4a4_lr_layer calls.
 
 Metric: algorithmic GB/s of the layer (X + L1^T + Wq + s_w + L2^T + Y bytes
 per layer), the decode roofline quantity; TOPS (2 M N K) is reported beside it.
@@ -59,7 +62,7 @@ def parse():
                     help="replay only the timed step graph (for a profiler); prints one status line")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill_gateup", "prefill_down", "large_gateup",
-                             "large_down", "sweep", "sweeps"],
+                             "large_down", "sweep", "sweeps", "gateup_swiglu"],
                     help="decode is the default workload; the others are the prefill "
                          "shapes, scored in TOPS against the dense INT8 peak")
     ap.add_argument("--rank", type=int, default=None, help="low-rank r override (sweep)")
@@ -609,6 +612,80 @@ def run_sweeps(args, rank, world, local_rank, dist):
     }
 
 
+def run_gateup(args, rank, world, local_rank, dist):
+    """Gate and up projections of the prefill MLP shape (M = 2048, K = 4096,
+    N = 14336 each, rank 64 each) as one shared-input pair: one activation
+    pass and one GEMM over the 2N interleaved channels with the SwiGLU
+    epilogue.  TOPS counts both projections (2 x 2 M N K); the comparison is
+    the two projections as separate layer calls (without the SwiGLU)."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    sh = synth.CONFIGS["prefill_gateup"]
+    M = args.m if args.m != 16 else sh.M
+    K, N, r, b = sh.K, sh.N, sh.r, sh.had_block
+    per_pair = 2 * M * K + K * N + 2 * M * N
+    L = max(2, min(args.layers, -(-200_000_000 // per_pair)))
+    pairs = []
+    for i in range(L):
+        seed = replica_seed(rank) + 10 * i
+        ws = [synth.make_weights(sh, seed=seed + k, device="cuda") for k in (0, 5)]
+        packed = []
+        for w in ws:
+            Wq, s_w = tq.tq_pack_weight(w["Rt"].to(dev), b)
+            packed.append((Wq, s_w, w["L1t"].to(dev), w["L2t"].to(dev)))
+        (Wg, sg, L1g, L2g), (Wu, su, L1u, L2u) = packed
+        Wq2, s_w2, L1t2, L2t2 = tq.tq_pack_gate_up(Wg, sg, L1g, L2g, Wu, su, L1u, L2u)
+        pairs.append({"X": synth.make_activations(sh, seed=seed, M=M).to(dev), "g": packed[0],
+                      "u": packed[1], "Wq2": Wq2, "s_w2": s_w2, "L1t2": L1t2, "L2t2": L2t2,
+                      "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                      "Yg": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                      "Yu": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                      "ws": tq.Workspace(dev), "wsg": tq.Workspace(dev), "wsu": tq.Workspace(dev)})
+        del ws
+    torch.cuda.synchronize()
+
+    def fused():
+        for p in pairs:
+            tq.tq_w4a4_lr_gate_up(p["X"], p["L1t2"], p["Wq2"], p["s_w2"], p["L2t2"], b, Y=p["Y"],
+                                  workspace=p["ws"])
+
+    def separate():
+        for p in pairs:
+            for (Wq, s_w, L1t, L2t), Y, w in ((p["g"], p["Yg"], p["wsg"]), (p["u"], p["Yu"], p["wsu"])):
+                tq.tq_w4a4_lr_layer(p["X"], L1t, Wq, s_w, L2t, b, Y=Y, workspace=w)
+
+    g1 = capture(torch, fused)
+    g2 = capture(torch, separate)
+    steps, warm = max(5, min(args.steps, 50)), max(3, args.warmup)
+    with ClockSampler(local_rank) as clk:
+        ms = time_graph(torch, g1, steps, warm, dist if world > 1 else None)
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
+    ms2 = time_graph(torch, g2, steps, warm)
+    ops = 2 * (2 * M * N * K)
+    peak, src = int8_peak(sustained=False)
+    return {
+        "metric": METRIC, "value": round(whole_job(L * ops, world, ms) / 1e12, 2), "unit": "TOPS",
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic",
+        "config": {"workload": f"gate/up pair with SwiGLU: M={M}, K={K}, N={N} per projection, "
+                               f"rank {r} each, Hadamard block {b}; {L} distinct pairs per step",
+                   "M": M, "K": K, "N": N, "r": r, "had_block": b, "pairs_per_step": L,
+                   "l2": "inputs larger than L2" if L * per_pair > 126e6 else "L2-resident"},
+        "us_per_pair": round(ms * 1e3 / L, 3),
+        "frac_int8": round(ops / (ms * 1e3 / L * 1e-6) / 1e12 / peak, 4), "peak_source": src,
+        "separate_layers_us": round(ms2 * 1e3 / L, 3),
+        "speedup_vs_separate": round(ms2 / ms, 3),
+        "gpu_launches": 2 * L * steps,
+        "clocks": clk.summary(),
+    }
+
+
 # ------------------------------------------------------------ oracle (CPU)
 
 def cpu_baseline(M, budget_s=12.0):
@@ -705,6 +782,8 @@ def main():
         out = run_tq(args, rank, world, local_rank, dist)
     elif args.workload == "sweeps":
         out = run_sweeps(args, rank, world, local_rank, dist)
+    elif args.workload == "gateup_swiglu":
+        out = run_gateup(args, rank, world, local_rank, dist)
     else:
         out = run_prefill(args, rank, world, local_rank, dist)
     if rank == 0:
