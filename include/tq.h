@@ -208,6 +208,33 @@ TQ_API int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uin
                               size_t workspace_bytes, void* stream);
 
 /*
+ * Per-token asymmetric activations (CoQuant Eq. (1) with a zero-point; the
+ * protocol CoQuant follows quantizes activations per token asymmetrically):
+ * for each token's rotated row v, z = min(v), s = (max(v) - min(v)) / 15,
+ * q = RoundClip((v - z) / s) in [0, 15] (ties to even), Q(v) = s q + z.  A
+ * constant row gets s = 0 and codes 0.
+ *
+ * tq_quantize_act_asym_i8 -- as tq_quantize_act_i8, with Xq8 = q - 8 (int8
+ * in [-8, 7]), s_x [M] = s and z_x [M] = z of the normalised rotation.
+ * tq_weight_code_sums -- offline: wsum [N] int32 = sum_k of each channel's
+ * weight codes (from Wq as tq_pack_weight makes it).
+ * tq_w4a4_lr_gemm_a8_asym -- as tq_w4a4_lr_gemm_a8 with
+ *   Y = bf16( s_w (s_x (acc + 8 wsum) + z_x wsum) + bf16(X L1) L2 ),
+ *   acc = sum_k (q - 8) qw, so that acc + 8 wsum = sum_k q qw exactly.
+ * Limits as tq_quantize_act_i8 / tq_w4a4_lr_gemm_a8; z_x and wsum 16-byte
+ * aligned.
+ */
+TQ_API int tq_quantize_act_asym_i8(const uint16_t* X, int M, int K, int had_block,
+                                   const uint16_t* L1t, int r, int8_t* Xq8, float* s_x,
+                                   float* z_x, uint16_t* XL1b, void* stream);
+TQ_API int tq_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum, void* stream);
+TQ_API int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const float* z_x,
+                                   const uint8_t* Wq, const float* s_w, const int32_t* wsum,
+                                   const uint16_t* XL1b, const uint16_t* L2t, int M, int N,
+                                   int K, int r, uint16_t* Y, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * tq_quantize_act_i8 -- tq_quantize_act for many tokens, with the codes one
  * per byte: the same rotation (CoQuant Eq. (3), block Hadamard), per-token
  * scale and RoundClip codes (CoQuant Eq. (1)) and the same X L1

@@ -22,6 +22,7 @@ def _load():
         lib.orc_hadamard_entry.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         lib.orc_rotate.argtypes = [_P, _L, _L, ctypes.c_int, _P]
         lib.orc_quantize_sym.argtypes = [_P, _L, _L, ctypes.c_int, _P, _P, _P]
+        lib.orc_quantize_asym.argtypes = [_P, _L, _L, ctypes.c_int, _P, _P, _P, _P]
         lib.orc_pack_int4.argtypes = [_P, _L, _L, _P]
         lib.orc_unpack_int4.argtypes = [_P, _L, _L, _P]
         lib.orc_int_gemm.restype = ctypes.c_long
@@ -185,3 +186,35 @@ def swiglu(g, u) -> np.ndarray:
     up pair's output from the two layers' fp64 outputs."""
     g, u = _f64(g), _f64(u)
     return g / (1.0 + np.exp(-g)) * u
+
+
+def quantize_asym(v, qmax: int = 15):
+    """Per-row asymmetric RoundClip (CoQuant Eq. (1), zero-point = row min):
+    returns (codes uint8 in [0, qmax], scales, zero-points, (v - z)/s), fp64."""
+    v = _f64(v)
+    rows, K = v.shape
+    q = np.empty((rows, K), dtype=np.uint8)
+    s = np.empty(rows, dtype=np.float64)
+    z = np.empty(rows, dtype=np.float64)
+    t = np.empty((rows, K), dtype=np.float64)
+    _load().orc_quantize_asym(_ptr(v), rows, K, int(qmax), _ptr(q), _ptr(s), _ptr(z), _ptr(t))
+    return q, s, z, t
+
+
+def layer_asym(X, L1t, L2t, Rt, b: int) -> dict:
+    """The layer with per-token asymmetric activations: the rotated X
+    quantized as Q(x) = s_x q + z_x (q in [0, 15]), the weights as in layer():
+    Y = s_x s_w (q . qw) + z_x s_w (sum_k qw) + bf16(X L1) L2, in fp64."""
+    q, s_x, z_x, t = quantize_asym(rotate(_f64(X), b))
+    w = pack_weight(Rt, b)
+    qw = w["qw"].astype(np.int64)
+    acc = q.astype(np.int64) @ qw.T                     # exact in int64
+    wsum = qw.sum(axis=1)
+    XL1, lr = lowrank(X, L1t, L2t)
+    Y64 = (s_x[:, None] * acc + z_x[:, None] * wsum[None, :]) * w["s_w"][None, :]
+    if _f64(L1t).shape[0] > 0:
+        Y64 = Y64 + lr
+    out = {"qa": q, "s_x": s_x, "z_x": z_x, "t_x": t, "acc": acc, "wsum": wsum,
+           "XL1": XL1, "lr": lr, "Y64": Y64}
+    out.update(w)
+    return out

@@ -89,6 +89,44 @@ void orc_rotate(const double* in, long rows, long K, int b, double* out) {
   }
 }
 
+/* Asymmetric per-row quantizer of CoQuant Eq. (1) with a real zero-point
+ * chosen from the row's range (the protocol's per-token asymmetric
+ * activations): z = min(v), s = (max(v) - min(v)) / qmax,
+ * q = RoundClip((v - z) / s) in [0, qmax], so that Q(v) = q s + z.
+ * Round-to-nearest is half-to-even.  A constant row gets s = 0, all codes 0
+ * and Q(v) = z exactly.  If t_out is not NULL it receives (v - z) / s. */
+void orc_quantize_asym(const double* v, long rows, long K, int qmax,
+                       uint8_t* q, double* s, double* z, double* t_out) {
+#pragma omp parallel for schedule(static)
+  for (long m = 0; m < rows; ++m) {
+    const double* x = v + m * K;
+    double lo = x[0], hi = x[0];
+    for (long k = 1; k < K; ++k) {
+      if (x[k] < lo) lo = x[k];
+      if (x[k] > hi) hi = x[k];
+    }
+    z[m] = lo;
+    if (hi == lo) {
+      s[m] = 0.0;
+      for (long k = 0; k < K; ++k) {
+        q[m * K + k] = 0;
+        if (t_out) t_out[m * K + k] = 0.0;
+      }
+      continue;
+    }
+    double scale = (hi - lo) / (double)qmax;
+    s[m] = scale;
+    for (long k = 0; k < K; ++k) {
+      double t = (x[k] - lo) / scale;
+      double r = nearbyint(t);
+      if (r > qmax) r = qmax;
+      if (r < 0) r = 0;
+      q[m * K + k] = (uint8_t)r;
+      if (t_out) t_out[m * K + k] = t;
+    }
+  }
+}
+
 /* Symmetric per-row quantizer of CoQuant Eq. (1) with zero-point 0:
  *   s = max|v| / qmax,  q = RoundClip(v / s) in [-qmax, qmax].
  * Round-to-nearest is half-to-even (nearbyint in the default rounding mode).

@@ -10,5 +10,6 @@ from .tq import (  # noqa: F401
     tq_gemm_workspace_bytes, tq_w4a4_lr_gemm, tq_w4a4_lr_gemm_noalloc, tq_debug_w4a4_gemm_acc,
     tq_query_device_status, Workspace, layer_forward, tq_layer_workspace_bytes, tq_w4a4_lr_layer,
     tq_quantize_act_i8, tq_w4a4_lr_gemm_a8, tq_layer_path, tq_pack_gate_up,
-    tq_gate_up_workspace_bytes, tq_w4a4_lr_gate_up,
+    tq_gate_up_workspace_bytes, tq_w4a4_lr_gate_up, tq_quantize_act_asym_i8, tq_weight_code_sums,
+    tq_w4a4_lr_gemm_a8_asym,
 )

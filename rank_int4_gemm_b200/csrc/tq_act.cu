@@ -407,6 +407,25 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
+// Sum of each channel's weight codes (offline; the zero-point term of
+// asymmetric activation codes): one warp per row of Wq, signed nibbles.
+__global__ void weight_code_sums_kernel(const uint8_t* __restrict__ Wq, int N, int K,
+                                        int32_t* __restrict__ wsum) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(Wq + (size_t)row * (K / 2));
+  int sum = 0;
+  for (int i = lane; i < K / 8; i += 32) {
+    const uint32_t v = __ldg(w + i);
+#pragma unroll
+    for (int n = 0; n < 8; ++n) sum += (int)(v << (28 - 4 * n)) >> 28;  // sign-extended nibble n
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) wsum[row] = sum;
+}
+
 // Gate / up pair as one layer (offline): row 2i of the pair is gate channel
 // i, row 2i+1 up channel i (packed codes and scales); the low-rank factors
 // stack along r, L1^T as [gate; up] (two copies) and L2^T block-diagonally:
@@ -470,6 +489,12 @@ cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uin
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   pack_weight_kernel<<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum,
+                                     cudaStream_t stream) {
+  weight_code_sums_kernel<<<(N + 7) / 8, 256, 0, stream>>>(Wq, N, K, wsum);
   return cudaGetLastError();
 }
 

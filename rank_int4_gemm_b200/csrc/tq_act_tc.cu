@@ -53,8 +53,10 @@ struct TcParams {
   int M, K, b, r;     // r: X L1 columns of this launch
   int r_ld, r_off;    // row stride of XL1 / XL1b, first column (and L1^T row) of this launch
   int xl1_only;       // X L1 only: no rotation, no codes, no s_x
+  float* z_x;         // asymmetric codes: [M] zero-points (row minimum), or null
+  float zmul;         // 1 / sqrt(b): the zero-point of the unnormalised transform
   int kb_total, nb;   // 128-column blocks in K, blocks per CTA
-  float scale_mul;    // 1 / (7 sqrt(b))
+  float scale_mul;    // 1 / (7 sqrt(b)); asymmetric: 1 / (15 sqrt(b))
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Atoms are 128-byte
@@ -63,23 +65,24 @@ struct TcParams {
 // X-L1-only launch has no Hadamard operand.
 constexpr int kNumBarsTc = 2 * kNS + 5;  // full[kNS], empty[kNS], rot_full[2], rot_empty[2], xl1_full
 struct TcLayout {
-  uint32_t h, stage0, stage, amax, bar, misc, bytes;
+  uint32_t h, stage0, stage, amax, amin, bar, misc, bytes;
 };
 __host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
   TcLayout L;
   L.h = 0;                                             // Hd^T: 2 atoms x 128 rows
   L.stage0 = xl1_only ? 0u : 2u * kBlk * 128u;
   L.stage = 2u * kTok * 128u + (uint32_t)r * 256u;     // X block + L1^T block
-  L.amax = L.stage0 + kNS * L.stage;                   // [C][128] fp32
-  L.bar = L.amax + kMaxC * kTok * 4u;
+  L.amax = L.stage0 + kNS * L.stage;                   // [C][128] fp32: absmax, or max
+  L.amin = L.amax + kMaxC * kTok * 4u;                 // [C][128] fp32: min (asymmetric)
+  L.bar = L.amin + kMaxC * kTok * 4u;
   L.misc = L.bar + kNumBarsTc * 8u;
   L.bytes = L.misc + 16u;
   return L;
 }
-static_assert(2u * kBlk * 128u + kNS * (2u * kTok * 128u + kMaxRtc * 256u) + kMaxC * kTok * 4u +
+static_assert(2u * kBlk * 128u + kNS * (2u * kTok * 128u + kMaxRtc * 256u) + 2u * kMaxC * kTok * 4u +
                       kNumBarsTc * 8u + 16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (codes)");
-static_assert(kNS * (2u * kTok * 128u + kMaxRx * 256u) + kMaxC * kTok * 4u + kNumBarsTc * 8u +
+static_assert(kNS * (2u * kTok * 128u + kMaxRx * 256u) + 2u * kMaxC * kTok * 4u + kNumBarsTc * 8u +
                       16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (X L1 only)");
 // the X L1 receive area [C][128][ceil(r/C)] reuses the stages after pass 2:
@@ -294,8 +297,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     cluster_wait_acquire();  // B0: peers are running before they are written to
 
-    // ---- pass 1: partial absmax of this token over the CTA's slice
-    float amax = 0.f;
+    // ---- pass 1: partial absmax (asymmetric: min and max) of this token
+    //      over the CTA's slice
+    const bool asym = p.z_x != nullptr;
+    float amax = 0.f, lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
     for (int i = 0; i < (xo ? 0 : nb); ++i) {
       const int u = i & 1;
       const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
@@ -308,22 +313,40 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
           tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
           tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(v[e])));
+          for (int e = 0; e < 32; ++e) {
+            const float f = __uint_as_float(v[e]);
+            amax = fmaxf(amax, fabsf(f));
+            lo = fminf(lo, f);
+            hi = fmaxf(hi, f);
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&rot_empty[u]);
     }
     if (!xo)
-      for (uint32_t z = 0; z < csize; ++z)
-        dsmem_st_f32(dsmem_map(base + L.amax + (crank * kTok + (uint32_t)row) * 4u, z), amax);
+      for (uint32_t z = 0; z < csize; ++z) {
+        const uint32_t off = (crank * kTok + (uint32_t)row) * 4u;
+        dsmem_st_f32(dsmem_map(base + L.amax + off, z), asym ? hi : amax);
+        if (asym) dsmem_st_f32(dsmem_map(base + L.amin + off, z), lo);
+      }
     cluster_arrive_rel();  // B1: partial absmax delivered
     cluster_wait_acquire();
-    float am = 0.f;
-    for (uint32_t z = 0; z < csize; ++z)
+    float am = asym ? -__int_as_float(0x7f800000) : 0.f;
+    float mn = __int_as_float(0x7f800000);
+    for (uint32_t z = 0; z < csize; ++z) {
       am = fmaxf(am, ld_shared_f32_tc(base + L.amax + (z * kTok + (uint32_t)row) * 4u));
-    if (!xo && crank == 0 && grow < p.M) p.s_x[grow] = am * p.scale_mul;
-    const CodeScale cs = code_scale(am);
+      if (asym) mn = fminf(mn, ld_shared_f32_tc(base + L.amin + (z * kTok + (uint32_t)row) * 4u));
+    }
+    // asymmetric: codes of (x - min) over the range max - min, in [0, 15]
+    // (stored as code - 8), scale range / 15, zero-point min
+    const float range = asym ? am - mn : am;
+    if (!xo && crank == 0 && grow < p.M) {
+      p.s_x[grow] = range * p.scale_mul;
+      if (asym) p.z_x[grow] = mn * p.zmul;
+    }
+    CodeScale cs = code_scale(range);  // pre (2^64 for a tiny range) and 7 / (range pre)
+    if (asym && range > 0.f) cs.inv = 15.f / (range * cs.pre);
 
     // ---- pass 2: the same rotation again -> codes in the packed layout
     //      (inside each 32-code group byte i = code i | code i+16 << 4)
@@ -345,8 +368,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             float f = __uint_as_float(v[e]);
-            if (cs.pre != 1.f) f *= cs.pre;
-            cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
+            if (asym) {
+              // RoundClip((x - min) / s) to [0, 15] with ties to even, as
+              // code - 8 in the byte (one fp32 subtraction, one product)
+              float y = (f * cs.pre - mn * cs.pre) * cs.inv;
+              y = fminf(fmaxf(y, 0.f), 15.f);
+              cb[e] = __float_as_uint(__fadd_rn(y, 12582912.f)) - 8u;
+            } else {
+              if (cs.pre != 1.f) f *= cs.pre;
+              cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
+            }
           }
           if (grow < p.M) {
             if (p.Xq8) {  // one code per byte, in column order
@@ -460,7 +491,7 @@ namespace {
 // X L1 columns [r_off, r_off + r) alone.
 cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                               int r_total, int r_off, int r, bool xl1_only, uint8_t* Xq,
-                              int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
+                              int8_t* Xq8, float* s_x, float* z_x, float* XL1, uint16_t* XL1b,
                               cudaStream_t stream) {
   TcParams p{};
   p.Xq = xl1_only ? nullptr : Xq;
@@ -475,8 +506,10 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
   p.r_ld = r_total;
   p.r_off = r_off;
   p.xl1_only = xl1_only ? 1 : 0;
+  p.z_x = xl1_only ? nullptr : z_x;
   p.kb_total = K / kBlk;
-  p.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  p.scale_mul = (float)(1.0 / ((p.z_x ? 15.0 : 7.0) * sqrt((double)had_block)));
+  p.zmul = (float)(1.0 / sqrt((double)had_block));
   const int tiles = (M + kTok - 1) / kTok;
   const uint32_t smem_bytes = tc_layout(xl1_only, r).bytes + 1024u;
   static uint64_t attr_set = 0;
@@ -559,17 +592,17 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
 // at most kMaxRx columns that skip the rotation.
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                           int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, float* z_x) {
   if (r <= kMaxRtc)
-    return launch_act_tc_one(X, M, K, had_block, L1t, r, 0, r, false, Xq, Xq8, s_x, XL1, XL1b,
-                             stream);
+    return launch_act_tc_one(X, M, K, had_block, L1t, r, 0, r, false, Xq, Xq8, s_x, z_x, XL1,
+                             XL1b, stream);
   if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, nullptr, r, 0, 0, false, Xq, Xq8, s_x,
-                                        nullptr, nullptr, stream))
+                                        z_x, nullptr, nullptr, stream))
     return e;
   for (int off = 0; off < r; off += kMaxRx) {
     const int w = std::min(kMaxRx, r - off);
     if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, L1t, r, off, w, true, Xq, Xq8, s_x,
-                                          XL1, XL1b, stream))
+                                          nullptr, XL1, XL1b, stream))
       return e;
   }
   return cudaSuccess;

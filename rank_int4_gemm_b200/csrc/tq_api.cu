@@ -382,5 +382,64 @@ int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uint8_t* W
   return from_cuda(tq::launch_gemm_a8(a, st));
 }
 
+// ------------------------------------------------ asymmetric activations
+int tq_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum, void* stream) {
+  if (!Wq || !wsum || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (!aligned16(Wq)) return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_weight_code_sums(Wq, N, K, wsum, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_quantize_act_asym_i8(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
+                            int r, int8_t* Xq8, float* s_x, float* z_x, uint16_t* XL1b,
+                            void* stream) {
+  if (!X || !Xq8 || !s_x || !z_x || M <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (had_block > 128) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1b != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Xq8) || !aligned16(s_x) || !aligned16(z_x) ||
+      (r > 0 && !aligned16(L1t)) || (r > 0 && !aligned16(XL1b)))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x, nullptr, XL1b,
+                                     static_cast<cudaStream_t>(stream), z_x));
+}
+
+int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const float* z_x,
+                            const uint8_t* Wq, const float* s_w, const int32_t* wsum,
+                            const uint16_t* XL1b, const uint16_t* L2t, int M, int N, int K, int r,
+                            uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!Xq8 || !s_x || !z_x || !Wq || !s_w || !wsum || !Y || M <= 0 || N <= 0)
+    return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (XL1b != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Xq8) || !aligned16(s_x) || !aligned16(z_x) || !aligned16(Wq) ||
+      !aligned16(s_w) || !aligned16(wsum) || !aligned16(Y) || (XL1b && !aligned16(XL1b)) ||
+      (L2t && !aligned16(L2t)) || (ws && !aligned16(ws)))
+    return TQ_ERR_MISALIGNED;
+  if (!ws || ws_bytes < tq::gemm_workspace_bytes(M, N, K, r)) return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  tq::GemmA8Args a{};
+  a.Xq8 = Xq8;
+  a.s_x = s_x;
+  a.Wq = Wq;
+  a.s_w = s_w;
+  a.XL1b = XL1b;
+  a.L2t = L2t;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.Y = Y;
+  a.ws = ws;
+  a.z_x = z_x;
+  a.wsum = wsum;
+  return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 

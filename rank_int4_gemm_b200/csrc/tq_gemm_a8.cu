@@ -68,6 +68,8 @@ struct A8Params {
   int kb_total, n_st, n_lr;  // k-blocks, k-block stages, low-rank stages per tile
   int tiles_m, tiles;        // token tiles, all tiles
   int swiglu;                // Y[t][c] = silu(y[t][2c]) * y[t][2c+1], Y is [M][N/2]
+  const float* z_x;          // asymmetric codes (code - 8): [M] zero-points, or null
+  const int32_t* wsum;       //   [N] sums of each channel's weight codes
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
@@ -99,7 +101,11 @@ __device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
   return v;
 }
 
-template <int TK>
+// Epilogue variants, one instantiation each (the plain one carries no code
+// or registers of the others)
+enum { kEpiPlain = 0, kEpiSwiglu = 1, kEpiAsym = 2 };
+
+template <int TK, int EPI>
 __global__ void __launch_bounds__(kThreadsA8, 1)
     w4a4_lr_gemm_a8_kernel(const __grid_constant__ CUtensorMap map_t,   // tokens int8 [M][K]
                            const __grid_constant__ CUtensorMap map_w,   // weights [N][K/2]
@@ -266,6 +272,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int gc = tn * kCh + row;
       const float sw = gc < p.N ? __ldg(p.s_w + gc) : 0.f;
+      const int ws = (EPI == kEpiAsym && gc < p.N) ? __ldg(p.wsum + gc) : 0;
       // int4 -> int8 (16 * code) for this thread's channel row, one k-block
       // (32 TMEM columns) at a time; inside each 16-byte packed chunk the low
       // nibbles are codes 0-15 and the high nibbles codes 16-31 of the group
@@ -328,11 +335,21 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
         const int t0 = tm * TK + 32 * j;
         const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
+        const float zx_l = (EPI == kEpiAsym && t0 + lane < p.M) ? __ldg(p.z_x + t0 + lane) : 0.f;
+        // y = s_x s_w acc; asymmetric codes c = q - 8 with zero-point z:
+        // sum q qw = acc + 8 wsum (exact), y = s_w (s_x (acc + 8 wsum) + z wsum)
+        auto dequant = [&](int e) -> float {
+          const int acc = ((int)a[e]) >> 4;
+          const float sx = __shfl_sync(0xffffffffu, sx_l, e);
+          if constexpr (EPI != kEpiAsym) return sx * sw * (float)acc;
+          const float zx = __shfl_sync(0xffffffffu, zx_l, e);
+          return sw * (sx * (float)(acc + 8 * ws) + zx * (float)ws);
+        };
         tmem_ld_wait();
-        if (!p.swiglu) {
+        if constexpr (EPI != kEpiSwiglu) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            float y = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
+            float y = dequant(e);
             if (p.r > 0) y += __uint_as_float(l[e]);
             const __nv_bfloat16 h = __float2bfloat16_rn(y);
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
@@ -359,7 +376,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
           float y[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            y[e] = __shfl_sync(0xffffffffu, sx_l, e) * sw * (float)(((int)a[e]) >> 4);
+            y[e] = dequant(e);
             if (p.r > 0) y[e] += __uint_as_float(l[e]);
           }
           const bool odd = lane & 1;
@@ -405,7 +422,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 
 namespace {
 
-template <int TK>
+template <int TK, int EPI>
 cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stream) {
   p.tiles_m = (a.M + TK - 1) / TK;
   p.tiles = p.tiles_m * ((a.N + kCh - 1) / kCh);
@@ -429,7 +446,7 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set >> dev & 1u)) {
-    cudaError_t e = cudaFuncSetAttribute(w4a4_lr_gemm_a8_kernel<TK>,
+    cudaError_t e = cudaFuncSetAttribute(w4a4_lr_gemm_a8_kernel<TK, EPI>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)A8Smem<TK>::kAlloc);
     if (e != cudaSuccess) return e;
@@ -445,7 +462,7 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
   attr[0].val.programmaticStreamSerializationAllowed = tuning().pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel<TK>, map_t, map_w, map_xb, map_l2, p);
+  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel<TK, EPI>, map_t, map_w, map_xb, map_l2, p);
 }
 
 }  // namespace
@@ -464,10 +481,14 @@ cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   p.n_st = (p.kb_total + 1) / 2;
   p.n_lr = (a.r + 63) / 64;
   p.swiglu = a.swiglu;
+  p.z_x = a.z_x;
+  p.wsum = a.wsum;
   // 128 x 192 tiles: narrower token tiles (160, 128; more TMEM left for
   // weight buffers) were measured slower on every prefill shape but one,
   // where they won by under 1 %
-  return launch_gemm_a8_tk<kTkMax>(a, p, stream);
+  if (a.swiglu) return launch_gemm_a8_tk<kTkMax, kEpiSwiglu>(a, p, stream);
+  if (a.z_x) return launch_gemm_a8_tk<kTkMax, kEpiAsym>(a, p, stream);
+  return launch_gemm_a8_tk<kTkMax, kEpiPlain>(a, p, stream);
 }
 
 }  // namespace tq

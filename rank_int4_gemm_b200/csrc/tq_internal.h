@@ -26,9 +26,11 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
 // Codes packed (Xq, [M][K/2]) or one int8 per code (Xq8, [M][K]); X L1 as
 // fp32 (XL1) and / or rounded to bf16 (XL1b), either may be null.
 bool act_tc_supported(int M, int K, int had_block, int r);
+// z_x non-null: asymmetric codes (zero-point = row minimum, codes 0..15
+// stored as code - 8), s_x = range / 15
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                           int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
-                          cudaStream_t stream);
+                          cudaStream_t stream, float* z_x = nullptr);
 
 // GEMM with one int8 per activation code (weights expanded into TMEM).
 struct GemmA8Args {
@@ -42,8 +44,12 @@ struct GemmA8Args {
   uint16_t* Y;            // [M][N], or [M][N/2] with swiglu
   void* ws;               // status word at offset 0
   int swiglu = 0;         // rows alternate gate / up: Y = silu(gate) * up
+  const float* z_x = nullptr;     // asymmetric activation codes: [M] zero-points
+  const int32_t* wsum = nullptr;  //   and [N] weight code sums
 };
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
+cudaError_t launch_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum,
+                                     cudaStream_t stream);
 cudaError_t launch_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
                                 const uint16_t* L2t_g, const uint8_t* Wq_u, const float* s_w_u,
                                 const uint16_t* L1t_u, const uint16_t* L2t_u, int N, int K, int r,

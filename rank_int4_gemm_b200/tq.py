@@ -43,6 +43,13 @@ _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
 _lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_layer_path.restype = _I
+_lib.tq_quantize_act_asym_i8.restype = _I
+_lib.tq_quantize_act_asym_i8.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P]
+_lib.tq_weight_code_sums.restype = _I
+_lib.tq_weight_code_sums.argtypes = [_P, _I, _I, _P, _P]
+_lib.tq_w4a4_lr_gemm_a8_asym.restype = _I
+_lib.tq_w4a4_lr_gemm_a8_asym.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P,
+                                         _P, ctypes.c_size_t, _P]
 _lib.tq_pack_gate_up.restype = _I
 _lib.tq_pack_gate_up.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P, _P, _P]
 _lib.tq_gate_up_workspace_bytes.restype = ctypes.c_size_t
@@ -216,6 +223,55 @@ def tq_w4a4_lr_gemm_a8(Xq8, s_x, Wq, s_w, XL1b=None, L2t=None, Y=None, workspace
                                    _ptr(XL1b) if r else None, _ptr(L2t) if r else None,
                                    M, N, K, r, _ptr(Y), _ptr(ws), ws.numel(), _stream(stream)),
            "tq_w4a4_lr_gemm_a8")
+    return Y
+
+
+def tq_quantize_act_asym_i8(X: torch.Tensor, had_block: int, L1t=None, stream=None):
+    """Per-token asymmetric codes: X [M][K] bf16 (+ L1^T) -> (Xq8 [M][K] int8
+    = code - 8, s_x [M], z_x [M] f32, XL1b [M][r] bf16)."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, (M, K), "X")
+    r = 0 if L1t is None else L1t.shape[0]
+    if r:
+        _need(L1t, torch.bfloat16, (r, K), "L1t")
+    dev = X.device
+    Xq8 = torch.empty(M, K, dtype=torch.int8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    z_x = torch.empty(M, dtype=torch.float32, device=dev)
+    XL1b = torch.empty(M, r, dtype=torch.bfloat16, device=dev) if r else None
+    _check(_lib.tq_quantize_act_asym_i8(_ptr(X), M, K, int(had_block), _ptr(L1t) if r else None,
+                                        r, _ptr(Xq8), _ptr(s_x), _ptr(z_x),
+                                        _ptr(XL1b) if r else None, _stream(stream)),
+           "tq_quantize_act_asym_i8")
+    return Xq8, s_x, z_x, XL1b
+
+
+def tq_weight_code_sums(Wq, stream=None):
+    """wsum [N] int32: the sum of each channel's weight codes."""
+    N, K2 = Wq.shape
+    wsum = torch.empty(N, dtype=torch.int32, device=Wq.device)
+    _check(_lib.tq_weight_code_sums(_ptr(Wq), N, 2 * K2, _ptr(wsum), _stream(stream)),
+           "tq_weight_code_sums")
+    return wsum
+
+
+def tq_w4a4_lr_gemm_a8_asym(Xq8, s_x, z_x, Wq, s_w, wsum, XL1b=None, L2t=None, Y=None,
+                            workspace=None, stream=None):
+    """Y [M][N] bf16 = s_w (s_x (acc + 8 wsum) + z_x wsum) + XL1b L2^T."""
+    M, K = Xq8.shape
+    N = Wq.shape[0]
+    r = 0 if XL1b is None else XL1b.shape[1]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
+    if workspace is None:
+        workspace = Workspace(Xq8.device)
+    need = tq_gemm_workspace_bytes(M, N, K, r)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_gemm_a8_asym(_ptr(Xq8), _ptr(s_x), _ptr(z_x), _ptr(Wq), _ptr(s_w),
+                                        _ptr(wsum), _ptr(XL1b) if r else None,
+                                        _ptr(L2t) if r else None, M, N, K, r, _ptr(Y), _ptr(ws),
+                                        ws.numel(), _stream(stream)),
+           "tq_w4a4_lr_gemm_a8_asym")
     return Y
 
 
