@@ -218,3 +218,27 @@ def layer_asym(X, L1t, L2t, Rt, b: int) -> dict:
            "XL1": XL1, "lr": lr, "Y64": Y64}
     out.update(w)
     return out
+
+
+def layer_qlr(X, L1t, L2t, Rt, b: int) -> dict:
+    """The layer with the INT4 low-rank branch (TwinQuant Figure 4): X L1 from
+    the same rotated activation codes and INT4 codes of H^T L1 (per column),
+    dequantized, requantized per token to INT4, times INT4 codes of L2 (per
+    output channel); Y = s_x s_w (qx . qw) + s_xl1 s_L2 (q_xl1 . q_L2), fp64."""
+    a = quantize_act(X, b)
+    w = pack_weight(Rt, b)
+    l1 = pack_weight(L1t, b)                 # rows of L1^T rotated like weight rows
+    acc1 = int_gemm(a["qx"], l1["qw"])       # [M][r], exact
+    xl1 = a["s_x"][:, None] * l1["s_w"][None, :] * acc1
+    qxl1, s_xl1, t_xl1 = quantize_sym(xl1)
+    ql2, s_l2, t_l2 = quantize_sym(_f64(L2t))  # per output channel over r, no rotation
+    acc = int_gemm(a["qx"], w["qw"])
+    acc2 = int_gemm(qxl1, ql2)
+    Y64 = (a["s_x"][:, None] * w["s_w"][None, :] * acc
+           + s_xl1[:, None] * s_l2[None, :] * acc2)
+    out = dict(a)
+    out.update(w)
+    out.update({"qL1": l1["qw"], "s_L1": l1["s_w"], "acc1": acc1, "xl1": xl1, "qxl1": qxl1,
+                "s_xl1": s_xl1, "t_xl1": t_xl1, "qL2": ql2, "s_L2": s_l2, "t_L2": t_l2,
+                "acc": acc, "acc2": acc2, "Y64": Y64})
+    return out

@@ -313,16 +313,26 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
 
 constexpr int kPackThreads = 256;
 
-__global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const float* __restrict__ Rt,
+// Rows of fp32 R^T (the residual), or of bf16 L1^T (the low-rank down
+// projection, quantized per column of H^T L1 for the INT4 low-rank branch).
+__device__ __forceinline__ float4 load4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __restrict__ Rt,
                                                                    int K, int b, float scale_mul,
                                                                    uint8_t* __restrict__ Wq,
                                                                    float* __restrict__ s_w) {
   extern __shared__ __align__(16) float row[];
   __shared__ float red[kPackThreads / 32];
   const int n = blockIdx.x;
-  const float* src = Rt + (size_t)n * K;
+  const T* src = Rt + (size_t)n * K;
   for (int k = threadIdx.x * 4; k < K; k += kPackThreads * 4)
-    *reinterpret_cast<float4*>(row + k) = *reinterpret_cast<const float4*>(src + k);
+    *reinterpret_cast<float4*>(row + k) = load4(src + k);
   __syncthreads();
   // in-place Sylvester butterflies, level by level (pairs never cross blocks)
   for (int h = 1; h < b; h <<= 1) {
@@ -407,6 +417,46 @@ cudaError_t launch_act_e(const ActParams& prm_in, int max_cluster, cudaStream_t 
   return cudaLaunchKernelEx(&cfg, kern, prm);
 }
 
+// Symmetric per-row INT4 codes of r values, written as bf16 integers (exact:
+// |code| <= 7), one warp per row: either rows of bf16 L2^T (offline, the
+// low-rank up projection per output channel), or the dequantized INT32
+// X L1 of the INT4 low-rank branch, xl1[t][j] = s_x[t] s_L1[j] acc[t][j]
+// (per token).  Scale = absmax / 7, codes RoundClip(v * 7 / absmax) with ties
+// to even; an all-zero row gets scale 0 and codes 0.
+__global__ void lowrank_codes_kernel(const __nv_bfloat16* __restrict__ src_bf16,
+                                     const int32_t* __restrict__ acc,
+                                     const float* __restrict__ s_x, const float* __restrict__ s_L1,
+                                     int rows, int r, __nv_bfloat16* __restrict__ codes,
+                                     float* __restrict__ scale) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int kMaxPerLane = 16;  // r <= 512
+  float v[kMaxPerLane];
+  float amax = 0.f;
+  const float sx = acc ? __ldg(s_x + row) : 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int j = lane + 32 * i;
+    v[i] = 0.f;
+    if (j < r) {
+      if (acc)
+        v[i] = sx * __ldg(s_L1 + j) * (float)__ldg(acc + (size_t)row * r + j);
+      else
+        v[i] = __bfloat162float(src_bf16[(size_t)row * r + j]);
+      amax = fmaxf(amax, fabsf(v[i]));
+    }
+  }
+  amax = warp_max(amax);
+  const float inv = amax > 0.f ? 7.f / amax : 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxPerLane; ++i) {
+    const int j = lane + 32 * i;
+    if (j < r) codes[(size_t)row * r + j] = __float2bfloat16_rn((float)quant_code(v[i], inv));
+  }
+  if (lane == 0) scale[row] = amax / 7.f;
+}
+
 // Sum of each channel's weight codes (offline; the zero-point term of
 // asymmetric activation codes): one warp per row of Wq, signed nibbles.
 __global__ void weight_code_sums_kernel(const uint8_t* __restrict__ Wq, int N, int K,
@@ -484,11 +534,35 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
 cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
                                float* s_w, cudaStream_t stream) {
   const size_t smem = (size_t)K * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel,
+  cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel<float>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  pack_weight_kernel<<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  pack_weight_kernel<float><<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
+                                   int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2,
+                                   float* s_L2, cudaStream_t stream) {
+  const size_t smem = (size_t)K * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel<__nv_bfloat16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  pack_weight_kernel<__nv_bfloat16><<<r, kPackThreads, smem, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(L1t), K, had_block, scale_mul, qL1, s_L1);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  lowrank_codes_kernel<<<(N + 7) / 8, 256, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(L2t), nullptr, nullptr, nullptr, N, r,
+      reinterpret_cast<__nv_bfloat16*>(qL2), s_L2);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_requant_xl1(const int32_t* acc, const float* s_x, const float* s_L1, int M,
+                               int r, uint16_t* XL1q, float* s_xl1, cudaStream_t stream) {
+  lowrank_codes_kernel<<<(M + 7) / 8, 256, 0, stream>>>(
+      nullptr, acc, s_x, s_L1, M, r, reinterpret_cast<__nv_bfloat16*>(XL1q), s_xl1);
   return cudaGetLastError();
 }
 

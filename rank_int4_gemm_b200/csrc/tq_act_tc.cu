@@ -388,7 +388,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               int8_t* dst = p.Xq8 + (size_t)grow * (size_t)p.K + blk * kBlk + 32 * g;
               reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
               reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-            } else {
+            }
+            if (p.Xq) {  // packed (both formats when both are asked for)
               uint32_t w[4];
 #pragma unroll
               for (int h = 0; h < 4; ++h)

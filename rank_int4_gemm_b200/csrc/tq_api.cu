@@ -441,5 +441,100 @@ int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const float* z_
   return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
 }
 
+// ----------------------------------------------- INT4 low-rank branch
+int tq_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
+                       int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2, float* s_L2,
+                       void* stream) {
+  if (!L1t || !L2t || !qL1 || !s_L1 || !qL2 || !s_L2 || N <= 0 || r <= 0)
+    return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (!aligned16(L1t) || !aligned16(qL1)) return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_pack_lowrank_q4(L1t, L2t, N, K, r, had_block, qL1, s_L1, qL2, s_L2,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+// Workspace of tq_quantize_act_qlr_i8: [status 256][packed codes M*K/2]
+// [X L1 INT32 4Mr][the X L1 GEMM's own workspace], 256-aligned parts.
+size_t tq_quantize_act_qlr_workspace_bytes(int M, int K, int r) {
+  if (M <= 0 || K <= 0 || r <= 0) return 256;
+  return 256 + align256((size_t)M * K / 2) + align256((size_t)M * r * 4) +
+         align256(tq::gemm_workspace_bytes(M, r, K, 0));
+}
+
+int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block, const uint8_t* qL1,
+                           const float* s_L1, int r, int8_t* Xq8, float* s_x, uint16_t* XL1q,
+                           float* s_xl1, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!X || !qL1 || !s_L1 || !Xq8 || !s_x || !XL1q || !s_xl1 || M <= 0 || r <= 0)
+    return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (had_block > 128) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(qL1) || !aligned16(Xq8) || !aligned16(s_x) ||
+      !aligned16(XL1q) || (workspace && !aligned16(workspace)))
+    return TQ_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < tq_quantize_act_qlr_workspace_bytes(M, K, r))
+    return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint8_t* Xq = ws + 256;
+  int32_t* acc = reinterpret_cast<int32_t*>(Xq + align256((size_t)M * K / 2));
+  uint8_t* gws = reinterpret_cast<uint8_t*>(acc) + align256((size_t)M * r * 4);
+  // the codes, in both layouts: one per byte (the main GEMM) and packed (X L1)
+  if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, nullptr, 0, Xq, Xq8, s_x, nullptr,
+                                        nullptr, st))
+    return from_cuda(e);
+  // X L1 in INT32 from the same codes and the INT4 L1 (H^T L1 per column)
+  tq::GemmArgs g{};
+  g.Xq = Xq;
+  g.Wq = qL1;
+  g.M = M;
+  g.N = r;
+  g.K = K;
+  g.r = 0;
+  g.acc_out = acc;
+  g.ws = gws;
+  g.ws_bytes = tq::gemm_workspace_bytes(M, r, K, 0);
+  if (cudaError_t e = tq::launch_gemm(g, st)) return from_cuda(e);
+  // dequantized with s_x s_L1 and requantized per token to INT4
+  return from_cuda(tq::launch_requant_xl1(acc, s_x, s_L1, M, r, XL1q, s_xl1, st));
+}
+
+int tq_w4a4_lr_gemm_a8_qlr(const int8_t* Xq8, const float* s_x, const uint8_t* Wq,
+                           const float* s_w, const uint16_t* XL1q, const float* s_xl1,
+                           const uint16_t* qL2, const float* s_L2, int M, int N, int K, int r,
+                           uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
+  if (!Xq8 || !s_x || !Wq || !s_w || !XL1q || !s_xl1 || !qL2 || !s_L2 || !Y || M <= 0 ||
+      N <= 0 || r <= 0)
+    return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(Xq8) || !aligned16(s_x) || !aligned16(Wq) || !aligned16(s_w) ||
+      !aligned16(XL1q) || !aligned16(s_xl1) || !aligned16(qL2) || !aligned16(s_L2) ||
+      !aligned16(Y) || (ws && !aligned16(ws)))
+    return TQ_ERR_MISALIGNED;
+  if (!ws || ws_bytes < tq::gemm_workspace_bytes(M, N, K, r)) return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  tq::GemmA8Args a{};
+  a.Xq8 = Xq8;
+  a.s_x = s_x;
+  a.Wq = Wq;
+  a.s_w = s_w;
+  a.XL1b = XL1q;
+  a.L2t = qL2;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.Y = Y;
+  a.ws = ws;
+  a.s_xl1 = s_xl1;
+  a.s_l2 = s_L2;
+  return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"
 

@@ -70,6 +70,8 @@ struct A8Params {
   int swiglu;                // Y[t][c] = silu(y[t][2c]) * y[t][2c+1], Y is [M][N/2]
   const float* z_x;          // asymmetric codes (code - 8): [M] zero-points, or null
   const int32_t* wsum;       //   [N] sums of each channel's weight codes
+  const float* s_xl1;        // INT4 low-rank branch: [M] scales of the requantized X L1
+  const float* s_l2;         //   and [N] of L2; the low-rank accumulator holds integers
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
@@ -103,7 +105,7 @@ __device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
 
 // Epilogue variants, one instantiation each (the plain one carries no code
 // or registers of the others)
-enum { kEpiPlain = 0, kEpiSwiglu = 1, kEpiAsym = 2 };
+enum { kEpiPlain = 0, kEpiSwiglu = 1, kEpiAsym = 2, kEpiQlr = 3 };
 
 template <int TK, int EPI>
 __global__ void __launch_bounds__(kThreadsA8, 1)
@@ -273,6 +275,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       const int gc = tn * kCh + row;
       const float sw = gc < p.N ? __ldg(p.s_w + gc) : 0.f;
       const int ws = (EPI == kEpiAsym && gc < p.N) ? __ldg(p.wsum + gc) : 0;
+      const float sl2 = (EPI == kEpiQlr && gc < p.N) ? __ldg(p.s_l2 + gc) : 0.f;
       // int4 -> int8 (16 * code) for this thread's channel row, one k-block
       // (32 TMEM columns) at a time; inside each 16-byte packed chunk the low
       // nibbles are codes 0-15 and the high nibbles codes 16-31 of the group
@@ -335,7 +338,16 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
         const int t0 = tm * TK + 32 * j;
         const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
-        const float zx_l = (EPI == kEpiAsym && t0 + lane < p.M) ? __ldg(p.z_x + t0 + lane) : 0.f;
+        const float zx_l = (EPI == kEpiAsym && t0 + lane < p.M) ? __ldg(p.z_x + t0 + lane)
+                           : (EPI == kEpiQlr && t0 + lane < p.M) ? __ldg(p.s_xl1 + t0 + lane)
+                                                                 : 0.f;
+        // the low-rank term: fp32 (bf16 branch), or s_xl1 s_L2 times the
+        // exact integer sum of the INT4 branch
+        auto lowrank = [&](int e) -> float {
+          const float v = __uint_as_float(l[e]);
+          if constexpr (EPI != kEpiQlr) return v;
+          return __shfl_sync(0xffffffffu, zx_l, e) * sl2 * v;
+        };
         // y = s_x s_w acc; asymmetric codes c = q - 8 with zero-point z:
         // sum q qw = acc + 8 wsum (exact), y = s_w (s_x (acc + 8 wsum) + z wsum)
         auto dequant = [&](int e) -> float {
@@ -350,7 +362,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             float y = dequant(e);
-            if (p.r > 0) y += __uint_as_float(l[e]);
+            if (p.r > 0) y += lowrank(e);
             const __nv_bfloat16 h = __float2bfloat16_rn(y);
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
                          "h"(*reinterpret_cast<const unsigned short*>(&h))
@@ -377,7 +389,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             y[e] = dequant(e);
-            if (p.r > 0) y[e] += __uint_as_float(l[e]);
+            if (p.r > 0) y[e] += lowrank(e);
           }
           const bool odd = lane & 1;
 #pragma unroll
@@ -483,11 +495,14 @@ cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   p.swiglu = a.swiglu;
   p.z_x = a.z_x;
   p.wsum = a.wsum;
+  p.s_xl1 = a.s_xl1;
+  p.s_l2 = a.s_l2;
   // 128 x 192 tiles: narrower token tiles (160, 128; more TMEM left for
   // weight buffers) were measured slower on every prefill shape but one,
   // where they won by under 1 %
   if (a.swiglu) return launch_gemm_a8_tk<kTkMax, kEpiSwiglu>(a, p, stream);
   if (a.z_x) return launch_gemm_a8_tk<kTkMax, kEpiAsym>(a, p, stream);
+  if (a.s_xl1) return launch_gemm_a8_tk<kTkMax, kEpiQlr>(a, p, stream);
   return launch_gemm_a8_tk<kTkMax, kEpiPlain>(a, p, stream);
 }
 

@@ -46,8 +46,15 @@ struct GemmA8Args {
   int swiglu = 0;         // rows alternate gate / up: Y = silu(gate) * up
   const float* z_x = nullptr;     // asymmetric activation codes: [M] zero-points
   const int32_t* wsum = nullptr;  //   and [N] weight code sums
+  const float* s_xl1 = nullptr;   // INT4 low-rank branch: [M] and [N] scales (XL1b and
+  const float* s_l2 = nullptr;    //   L2t then hold integer codes in bf16)
 };
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
+cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
+                                   int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2,
+                                   float* s_L2, cudaStream_t stream);
+cudaError_t launch_requant_xl1(const int32_t* acc, const float* s_x, const float* s_L1, int M,
+                               int r, uint16_t* XL1q, float* s_xl1, cudaStream_t stream);
 cudaError_t launch_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum,
                                      cudaStream_t stream);
 cudaError_t launch_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
@@ -65,7 +72,7 @@ struct GemmArgs {
   const uint16_t* L2t;
   int M, N, K, r;
   uint16_t* Y;          // bf16 output (null in accumulator-debug mode)
-  int32_t* acc_out;     // raw accumulators (debug mode only)
+  int32_t* acc_out;     // raw accumulators (debug mode; the INT4 low-rank branch's X L1)
   void* ws;
   size_t ws_bytes;
 };

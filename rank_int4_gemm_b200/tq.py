@@ -43,6 +43,16 @@ _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
 _lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_layer_path.restype = _I
+_lib.tq_pack_lowrank_q4.restype = _I
+_lib.tq_pack_lowrank_q4.argtypes = [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P]
+_lib.tq_quantize_act_qlr_workspace_bytes.restype = ctypes.c_size_t
+_lib.tq_quantize_act_qlr_workspace_bytes.argtypes = [_I, _I, _I]
+_lib.tq_quantize_act_qlr_i8.restype = _I
+_lib.tq_quantize_act_qlr_i8.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P, _P,
+                                        ctypes.c_size_t, _P]
+_lib.tq_w4a4_lr_gemm_a8_qlr.restype = _I
+_lib.tq_w4a4_lr_gemm_a8_qlr.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P,
+                                        _P, ctypes.c_size_t, _P]
 _lib.tq_quantize_act_asym_i8.restype = _I
 _lib.tq_quantize_act_asym_i8.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P]
 _lib.tq_weight_code_sums.restype = _I
@@ -272,6 +282,61 @@ def tq_w4a4_lr_gemm_a8_asym(Xq8, s_x, z_x, Wq, s_w, wsum, XL1b=None, L2t=None, Y
                                         _ptr(L2t) if r else None, M, N, K, r, _ptr(Y), _ptr(ws),
                                         ws.numel(), _stream(stream)),
            "tq_w4a4_lr_gemm_a8_asym")
+    return Y
+
+
+def tq_pack_lowrank_q4(L1t, L2t, had_block, stream=None):
+    """INT4 low-rank factors: (qL1 [r][K/2] u8, s_L1 [r], qL2 [N][r] bf16
+    integer codes, s_L2 [N])."""
+    r, K = L1t.shape
+    N = L2t.shape[0]
+    dev = L1t.device
+    qL1 = torch.empty(r, K // 2, dtype=torch.uint8, device=dev)
+    s_L1 = torch.empty(r, dtype=torch.float32, device=dev)
+    qL2 = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
+    s_L2 = torch.empty(N, dtype=torch.float32, device=dev)
+    _check(_lib.tq_pack_lowrank_q4(_ptr(L1t), _ptr(L2t), N, K, r, int(had_block), _ptr(qL1),
+                                   _ptr(s_L1), _ptr(qL2), _ptr(s_L2), _stream(stream)),
+           "tq_pack_lowrank_q4")
+    return qL1, s_L1, qL2, s_L2
+
+
+def tq_quantize_act_qlr_i8(X, had_block, qL1, s_L1, workspace=None, stream=None):
+    """(Xq8 [M][K] s8, s_x [M], XL1q [M][r] bf16 integer codes, s_xl1 [M])."""
+    M, K = X.shape
+    r = qL1.shape[0]
+    dev = X.device
+    Xq8 = torch.empty(M, K, dtype=torch.int8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    XL1q = torch.empty(M, r, dtype=torch.bfloat16, device=dev)
+    s_xl1 = torch.empty(M, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = Workspace(dev)
+    need = int(_lib.tq_quantize_act_qlr_workspace_bytes(M, K, r))
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_quantize_act_qlr_i8(_ptr(X), M, K, int(had_block), _ptr(qL1), _ptr(s_L1), r,
+                                       _ptr(Xq8), _ptr(s_x), _ptr(XL1q), _ptr(s_xl1), _ptr(ws),
+                                       ws.numel(), _stream(stream)),
+           "tq_quantize_act_qlr_i8")
+    return Xq8, s_x, XL1q, s_xl1
+
+
+def tq_w4a4_lr_gemm_a8_qlr(Xq8, s_x, Wq, s_w, XL1q, s_xl1, qL2, s_L2, Y=None, workspace=None,
+                           stream=None):
+    """Y [M][N] bf16 = s_x s_w (Xq8 . Wq) + s_xl1 s_L2 (XL1q . qL2)."""
+    M, K = Xq8.shape
+    N = Wq.shape[0]
+    r = XL1q.shape[1]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
+    if workspace is None:
+        workspace = Workspace(Xq8.device)
+    need = tq_gemm_workspace_bytes(M, N, K, r)
+    ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_w4a4_lr_gemm_a8_qlr(_ptr(Xq8), _ptr(s_x), _ptr(Wq), _ptr(s_w), _ptr(XL1q),
+                                       _ptr(s_xl1), _ptr(qL2), _ptr(s_L2), M, N, K, r, _ptr(Y),
+                                       _ptr(ws), ws.numel(), _stream(stream)),
+           "tq_w4a4_lr_gemm_a8_qlr")
     return Y
 
 
