@@ -15,7 +15,9 @@ tq_quantize_act + tq_w4a4_lr_gemm on the prefill and sweep shapes instead;
 at rank 64, rank from 0 to 512 at M = 4096) through tq_w4a4_lr_layer;
 --workload gateup_swiglu times the MLP's gate and up projections as one
 shared-input pair with the SwiGLU epilogue (tq_w4a4_lr_gate_up) against the
-two projections as separate tq_w4a4_lr_layer calls.
+two projections as separate tq_w4a4_lr_layer calls; --workload qlr times the
+layer with the INT4 low-rank branch against the same layer with the bf16
+branch (prefill gate/up shape).
 
 Metric: algorithmic GB/s of the layer (X + L1^T + Wq + s_w + L2^T + Y bytes
 per layer), the decode roofline quantity; TOPS (2 M N K) is reported beside it.
@@ -62,7 +64,7 @@ def parse():
                     help="replay only the timed step graph (for a profiler); prints one status line")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill_gateup", "prefill_down", "large_gateup",
-                             "large_down", "sweep", "sweeps", "gateup_swiglu"],
+                             "large_down", "sweep", "sweeps", "gateup_swiglu", "qlr"],
                     help="decode is the default workload; the others are the prefill "
                          "shapes, scored in TOPS against the dense INT8 peak")
     ap.add_argument("--rank", type=int, default=None, help="low-rank r override (sweep)")
@@ -686,6 +688,72 @@ def run_gateup(args, rank, world, local_rank, dist):
     }
 
 
+def run_qlr(args, rank, world, local_rank, dist):
+    """The prefill gate/up layer (M = 2048, K = 4096, N = 14336, rank 64) with
+    the INT4 low-rank branch (activation codes, X L1 in INT32, requantized,
+    second integer product) against the same layer with the bf16 branch;
+    TOPS = 2 M N K per layer."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    sh = synth.CONFIGS["prefill_gateup"]
+    M = args.m if args.m != 16 else sh.M
+    K, N, r, b = sh.K, sh.N, sh.r, sh.had_block
+    per_layer = 2 * M * K + K * N // 2 + 2 * M * N
+    L = max(2, min(args.layers, -(-200_000_000 // per_layer)))
+    lays = []
+    for i in range(L):
+        seed = replica_seed(rank) + 10 * i
+        w = synth.make_weights(sh, seed=seed, device="cuda")
+        Wq, s_w = tq.tq_pack_weight(w["Rt"].to(dev), b)
+        L1t, L2t = w["L1t"].to(dev), w["L2t"].to(dev)
+        lays.append({"X": synth.make_activations(sh, seed=seed, M=M).to(dev), "Wq": Wq, "s_w": s_w,
+                     "L1t": L1t, "L2t": L2t, "q": tq.tq_pack_lowrank_q4(L1t, L2t, b),
+                     "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                     "wa": tq.Workspace(dev), "wg": tq.Workspace(dev)})
+        del w
+    torch.cuda.synchronize()
+
+    def int4_branch():
+        for l in lays:
+            qL1, s_L1, qL2, s_L2 = l["q"]
+            Xq8, s_x, XL1q, s_xl1 = tq.tq_quantize_act_qlr_i8(l["X"], b, qL1, s_L1, workspace=l["wa"])
+            tq.tq_w4a4_lr_gemm_a8_qlr(Xq8, s_x, l["Wq"], l["s_w"], XL1q, s_xl1, qL2, s_L2, Y=l["Y"],
+                                      workspace=l["wg"])
+
+    def bf16_branch():
+        for l in lays:
+            Xq8, s_x, XL1b = tq.tq_quantize_act_i8(l["X"], b, l["L1t"])
+            tq.tq_w4a4_lr_gemm_a8(Xq8, s_x, l["Wq"], l["s_w"], XL1b, l["L2t"], Y=l["Y"],
+                                  workspace=l["wg"])
+
+    g1, g2 = capture(torch, int4_branch), capture(torch, bf16_branch)
+    steps, warm = max(5, min(args.steps, 50)), max(3, args.warmup)
+    with ClockSampler(local_rank) as clk:
+        ms = time_graph(torch, g1, steps, warm, dist if world > 1 else None)
+    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
+    ms2 = time_graph(torch, g2, steps, warm)
+    ops = 2 * M * N * K
+    return {
+        "metric": METRIC, "value": round(whole_job(L * ops, world, ms) / 1e12, 2), "unit": "TOPS",
+        "n_gpus": world, "steps": steps, "warmup": warm, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+        "data": "synthetic",
+        "config": {"workload": f"INT4 low-rank branch: M={M}, K={K}, N={N}, rank {r}, Hadamard "
+                               f"block {b}; {L} distinct layers per step",
+                   "M": M, "K": K, "N": N, "r": r, "had_block": b, "layers_per_step": L,
+                   "l2": "inputs larger than L2" if L * per_layer > 126e6 else "L2-resident"},
+        "us_per_layer": round(ms * 1e3 / L, 3),
+        "bf16_branch_us_per_layer": round(ms2 * 1e3 / L, 3),
+        "gpu_launches": 5 * L * steps,
+        "clocks": clk.summary(),
+    }
+
+
 # ------------------------------------------------------------ oracle (CPU)
 
 def cpu_baseline(M, budget_s=12.0):
@@ -784,6 +852,8 @@ def main():
         out = run_sweeps(args, rank, world, local_rank, dist)
     elif args.workload == "gateup_swiglu":
         out = run_gateup(args, rank, world, local_rank, dist)
+    elif args.workload == "qlr":
+        out = run_qlr(args, rank, world, local_rank, dist)
     else:
         out = run_prefill(args, rank, world, local_rank, dist)
     if rank == 0:

@@ -495,6 +495,7 @@ int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block, const
   g.K = K;
   g.r = 0;
   g.acc_out = acc;
+  g.prefer_split = 1;  // r channels: split K rather than one CTA per 128 tokens
   g.ws = gws;
   g.ws_bytes = tq::gemm_workspace_bytes(M, r, K, 0);
   if (cudaError_t e = tq::launch_gemm(g, st)) return from_cuda(e);

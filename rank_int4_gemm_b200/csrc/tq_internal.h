@@ -75,6 +75,7 @@ struct GemmArgs {
   int32_t* acc_out;     // raw accumulators (debug mode; the INT4 low-rank branch's X L1)
   void* ws;
   size_t ws_bytes;
+  int prefer_split = 0;  // few channels, many tokens: the split-K plan for any M
 };
 
 size_t gemm_workspace_bytes(int M, int N, int K, int r);
