@@ -244,23 +244,29 @@ TQ_API int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const fl
  * to a second integer product with INT4 codes of L2 (per output channel:
  * s_L2[n]); the shared epilogue adds s_xl1 s_L2 times that integer sum.
  *
- * tq_pack_lowrank_q4 -- offline: qL1 [r][K/2] u8 packed codes of the rows of
- *   L1^T rotated like weight rows (had_block), s_L1 [r]; qL2 [N][r] the codes
- *   of L2^T rows as bf16 integers, s_L2 [N].  r a multiple of 16, <= 512.
+ * tq_pack_lowrank_q4 -- offline: qL1 [r][K] s8, the codes of the rows of
+ *   L1^T rotated like weight rows (had_block), one per byte (the factor is
+ *   small and this is the tensor cores' operand layout), s_L1 [r]; qL2 [N][r]
+ *   the codes of L2^T rows as bf16 integers, s_L2 [N].  r a multiple of 16,
+ *   <= 512.
  * tq_quantize_act_qlr_i8 -- Xq8 [M][K] s8 codes and s_x [M] as
  *   tq_quantize_act_i8; XL1q [M][r] the requantized X L1 codes as bf16
- *   integers, s_xl1 [M].  Workspace >= tq_quantize_act_qlr_workspace_bytes.
+ *   integers, s_xl1 [M].  The INT32 product runs on the tensor cores with K
+ *   split over a thread-block cluster; the requantization is fused for r <=
+ *   256.  Workspace >= tq_quantize_act_qlr_workspace_bytes (status word,
+ *   INT32 scratch for wider ranks); a timeout is reported through
+ *   tq_query_device_status on that workspace.
  * tq_w4a4_lr_gemm_a8_qlr -- Y = bf16( s_x s_w (Xq8 . Wq) +
  *   s_xl1 s_L2 (XL1q . qL2) ).  The second product runs on the bf16 MMA path
  *   with the integer codes: exact, since |code| <= 7 and |sum| <= 49 r < 2^24
  *   in the fp32 accumulator.
  */
 TQ_API int tq_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
-                              int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2,
+                              int had_block, int8_t* qL1, float* s_L1, uint16_t* qL2,
                               float* s_L2, void* stream);
 TQ_API size_t tq_quantize_act_qlr_workspace_bytes(int M, int K, int r);
 TQ_API int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block,
-                                  const uint8_t* qL1, const float* s_L1, int r, int8_t* Xq8,
+                                  const int8_t* qL1, const float* s_L1, int r, int8_t* Xq8,
                                   float* s_x, uint16_t* XL1q, float* s_xl1, void* workspace,
                                   size_t workspace_bytes, void* stream);
 TQ_API int tq_w4a4_lr_gemm_a8_qlr(const int8_t* Xq8, const float* s_x, const uint8_t* Wq,

@@ -322,7 +322,8 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
                      __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xFFFF0000u));
 }
 
-template <typename T>
+// kBytes: codes one per byte ([N][K] int8) instead of packed ([N][K/2]).
+template <typename T, bool kBytes = false>
 __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __restrict__ Rt,
                                                                    int K, int b, float scale_mul,
                                                                    uint8_t* __restrict__ Wq,
@@ -357,6 +358,12 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __re
   __syncthreads();
   const float amax = red[0];
   const float inv = amax > 0.f ? 7.f / amax : 0.f;
+  if constexpr (kBytes) {
+    int8_t* dst8 = reinterpret_cast<int8_t*>(Wq) + (size_t)n * K;
+    for (int k = threadIdx.x; k < K; k += kPackThreads) dst8[k] = (int8_t)quant_code(row[k], inv);
+    if (threadIdx.x == 0) s_w[n] = amax * scale_mul;
+    return;
+  }
   uint8_t* dst = Wq + (size_t)n * (K / 2);
   for (int byte = threadIdx.x; byte < K / 2; byte += kPackThreads) {
     const int g = byte / 16, i = byte % 16;
@@ -543,15 +550,15 @@ cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uin
 }
 
 cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
-                                   int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2,
+                                   int had_block, int8_t* qL1, float* s_L1, uint16_t* qL2,
                                    float* s_L2, cudaStream_t stream) {
   const size_t smem = (size_t)K * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel<__nv_bfloat16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto pack = pack_weight_kernel<__nv_bfloat16, true>;
+  cudaError_t e = cudaFuncSetAttribute(pack, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  pack_weight_kernel<__nv_bfloat16><<<r, kPackThreads, smem, stream>>>(
-      reinterpret_cast<const __nv_bfloat16*>(L1t), K, had_block, scale_mul, qL1, s_L1);
+  pack<<<r, kPackThreads, smem, stream>>>(reinterpret_cast<const __nv_bfloat16*>(L1t), K, had_block,
+                                          scale_mul, reinterpret_cast<uint8_t*>(qL1), s_L1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lowrank_codes_kernel<<<(N + 7) / 8, 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(L2t), nullptr, nullptr, nullptr, N, r,

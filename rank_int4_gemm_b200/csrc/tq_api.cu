@@ -443,7 +443,7 @@ int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const float* z_
 
 // ----------------------------------------------- INT4 low-rank branch
 int tq_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
-                       int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2, float* s_L2,
+                       int had_block, int8_t* qL1, float* s_L1, uint16_t* qL2, float* s_L2,
                        void* stream) {
   if (!L1t || !L2t || !qL1 || !s_L1 || !qL2 || !s_L2 || N <= 0 || r <= 0)
     return TQ_ERR_INVALID_VALUE;
@@ -455,15 +455,15 @@ int tq_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, i
                                               static_cast<cudaStream_t>(stream)));
 }
 
-// Workspace of tq_quantize_act_qlr_i8: [status 256][packed codes M*K/2]
-// [X L1 INT32 4Mr][the X L1 GEMM's own workspace], 256-aligned parts.
+// Workspace of tq_quantize_act_qlr_i8: [status 256][X L1 INT32 sums 4Mr,
+// used for ranks above 256].
 size_t tq_quantize_act_qlr_workspace_bytes(int M, int K, int r) {
-  if (M <= 0 || K <= 0 || r <= 0) return 256;
-  return 256 + align256((size_t)M * K / 2) + align256((size_t)M * r * 4) +
-         align256(tq::gemm_workspace_bytes(M, r, K, 0));
+  (void)K;
+  if (M <= 0 || r <= 0) return 256;
+  return 256 + align256((size_t)M * r * 4);
 }
 
-int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block, const uint8_t* qL1,
+int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block, const int8_t* qL1,
                            const float* s_L1, int r, int8_t* Xq8, float* s_x, uint16_t* XL1q,
                            float* s_xl1, void* workspace, size_t workspace_bytes, void* stream) {
   if (!X || !qL1 || !s_L1 || !Xq8 || !s_x || !XL1q || !s_xl1 || M <= 0 || r <= 0)
@@ -479,28 +479,15 @@ int tq_quantize_act_qlr_i8(const uint16_t* X, int M, int K, int had_block, const
   if (int s = check_device()) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  uint8_t* Xq = ws + 256;
-  int32_t* acc = reinterpret_cast<int32_t*>(Xq + align256((size_t)M * K / 2));
-  uint8_t* gws = reinterpret_cast<uint8_t*>(acc) + align256((size_t)M * r * 4);
-  // the codes, in both layouts: one per byte (the main GEMM) and packed (X L1)
-  if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, nullptr, 0, Xq, Xq8, s_x, nullptr,
+  int32_t* acc = reinterpret_cast<int32_t*>(ws + 256);
+  // the rotated activation codes, one per byte
+  if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, nullptr, 0, nullptr, Xq8, s_x, nullptr,
                                         nullptr, st))
     return from_cuda(e);
-  // X L1 in INT32 from the same codes and the INT4 L1 (H^T L1 per column)
-  tq::GemmArgs g{};
-  g.Xq = Xq;
-  g.Wq = qL1;
-  g.M = M;
-  g.N = r;
-  g.K = K;
-  g.r = 0;
-  g.acc_out = acc;
-  g.prefer_split = 1;  // r channels: split K rather than one CTA per 128 tokens
-  g.ws = gws;
-  g.ws_bytes = tq::gemm_workspace_bytes(M, r, K, 0);
-  if (cudaError_t e = tq::launch_gemm(g, st)) return from_cuda(e);
+  // X L1 in INT32 from those codes and the INT4 L1 (H^T L1 per column),
   // dequantized with s_x s_L1 and requantized per token to INT4
-  return from_cuda(tq::launch_requant_xl1(acc, s_x, s_L1, M, r, XL1q, s_xl1, st));
+  return from_cuda(tq::launch_xl1_codes(Xq8, qL1, s_x, s_L1, M, K, r, XL1q, s_xl1, acc,
+                                        reinterpret_cast<uint32_t*>(ws), st));
 }
 
 int tq_w4a4_lr_gemm_a8_qlr(const int8_t* Xq8, const float* s_x, const uint8_t* Wq,

@@ -51,8 +51,14 @@ struct GemmA8Args {
 };
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
 cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
-                                   int had_block, uint8_t* qL1, float* s_L1, uint16_t* qL2,
+                                   int had_block, int8_t* qL1, float* s_L1, uint16_t* qL2,
                                    float* s_L2, cudaStream_t stream);
+// X L1 of the INT4 low-rank branch from the activation codes (tq_qlr.cu):
+// INT32 on the tensor cores, requantized per token; acc [M][r] INT32 is
+// scratch for ranks above 256, status the timeout word.
+cudaError_t launch_xl1_codes(const int8_t* Xq8, const int8_t* qL1, const float* s_x,
+                             const float* s_L1, int M, int K, int r, uint16_t* XL1q, float* s_xl1,
+                             int32_t* acc, uint32_t* status, cudaStream_t stream);
 cudaError_t launch_requant_xl1(const int32_t* acc, const float* s_x, const float* s_L1, int M,
                                int r, uint16_t* XL1q, float* s_xl1, cudaStream_t stream);
 cudaError_t launch_weight_code_sums(const uint8_t* Wq, int N, int K, int32_t* wsum,

@@ -286,12 +286,12 @@ def tq_w4a4_lr_gemm_a8_asym(Xq8, s_x, z_x, Wq, s_w, wsum, XL1b=None, L2t=None, Y
 
 
 def tq_pack_lowrank_q4(L1t, L2t, had_block, stream=None):
-    """INT4 low-rank factors: (qL1 [r][K/2] u8, s_L1 [r], qL2 [N][r] bf16
+    """INT4 low-rank factors: (qL1 [r][K] s8 codes, s_L1 [r], qL2 [N][r] bf16
     integer codes, s_L2 [N])."""
     r, K = L1t.shape
     N = L2t.shape[0]
     dev = L1t.device
-    qL1 = torch.empty(r, K // 2, dtype=torch.uint8, device=dev)
+    qL1 = torch.empty(r, K, dtype=torch.int8, device=dev)
     s_L1 = torch.empty(r, dtype=torch.float32, device=dev)
     qL2 = torch.empty(N, r, dtype=torch.bfloat16, device=dev)
     s_L2 = torch.empty(N, dtype=torch.float32, device=dev)

@@ -74,6 +74,9 @@ CASES = [
     ("decode_like", 16, 1024, 384, 32, 128),
     ("one_token", 1, 512, 128, 16, 64),
     ("wide_rank", 150, 512, 256, 128, 32),
+    ("rank256_ragged_k", 200, 640, 256, 256, 128),   # widest fused requantization, 5 k-blocks
+    ("rank272_chunked", 130, 384, 288, 272, 128),     # INT32 sums in two column launches
+    ("rank512_chunked", 64, 1024, 512, 512, 64),
 ]
 
 
@@ -89,7 +92,7 @@ def test_qlr_path_matches_oracle(tq, name, M, K, N, r, b):
     torch.cuda.synchronize()
     o = oracle.layer_qlr(L["X"], L["L1t"], L["L2t"], L["Rt"], b)
     # offline factors: codes under the midpoint rule, scales to fp32 precision
-    gl1 = oracle.unpack_int4(qL1.cpu().numpy())
+    gl1 = qL1.cpu().numpy().astype(np.int64)
     l1o = oracle.pack_weight(L["L1t"], b)
     check_codes(gl1, l1o["qw"], l1o["t_w"], f"{name}: L1 codes", packed=False)
     assert np.allclose(s_L1.cpu().numpy(), o["s_L1"], rtol=2e-6, atol=0)
@@ -111,3 +114,41 @@ def test_qlr_path_matches_oracle(tq, name, M, K, N, r, b):
             + s_xl1.cpu().numpy().astype(np.float64)[:, None]
             * s_L2.cpu().numpy().astype(np.float64)[None, :] * (gq @ gl2.T))
     check_y(Y.double().cpu().numpy(), want, name)
+
+
+@pytest.mark.gpu
+def test_qlr_full_size_sampled(tq):
+    """The Llama-3-8B gate/up prefill shape (2048 x 4096 -> 14336, r = 64) in
+    the benchmark's launch configuration; sampled tokens and channels against
+    the definition (each sampled token row carries its full K)."""
+    sh = synth.CONFIGS["prefill_gateup"]
+    M, K, N, r, b = sh.M, sh.K, sh.N, sh.r, sh.had_block
+    L = synth.make_layer(sh, seed=11, device="cuda")
+    X, L1t, L2t = L["X"].cuda(), L["L1t"].cuda(), L["L2t"].cuda()
+    Wq, s_w = tq.tq_pack_weight(L["Rt"].cuda(), b)
+    qL1, s_L1, qL2, s_L2 = tq.tq_pack_lowrank_q4(L1t, L2t, b)
+    Xq8, s_x, XL1q, s_xl1 = tq.tq_quantize_act_qlr_i8(X, b, qL1, s_L1)
+    Y = tq.tq_w4a4_lr_gemm_a8_qlr(Xq8, s_x, Wq, s_w, XL1q, s_xl1, qL2, s_L2)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([[0, 1, M // 2, M - 1], rng.choice(M, 12, replace=False)]))
+    cols = np.unique(np.concatenate([[0, N - 1], rng.choice(N, 126, replace=False)]))
+    rt, ct = torch.from_numpy(rows).cuda(), torch.from_numpy(cols).cuda()
+    a = oracle.quantize_act(L["X"][torch.from_numpy(rows)], b, None)
+    qx = Xq8[rt].cpu().numpy().astype(np.int64)
+    check_codes(qx, a["qx"], a["t_x"], "activation codes", packed=False)
+    sx = s_x[rt].cpu().numpy().astype(np.float64)
+    l1o = oracle.pack_weight(L["L1t"], b)
+    gl1 = qL1.cpu().numpy().astype(np.int64)
+    check_codes(gl1, l1o["qw"], l1o["t_w"], "L1 codes", packed=False)
+    xl1 = sx[:, None] * s_L1.cpu().numpy().astype(np.float64)[None, :] * (qx @ gl1.T)
+    rq, rs, rtie = oracle.quantize_sym(xl1)
+    gq = XL1q[rt].float().cpu().numpy().astype(np.int64)
+    check_codes(gq, rq, rtie, "requantized X L1 codes", packed=False)
+    assert np.allclose(s_xl1[rt].cpu().numpy(), rs, rtol=2e-6, atol=0)
+    w = oracle.pack_weight(L["Rt"][torch.from_numpy(cols)], b)
+    gl2 = qL2[ct].float().cpu().numpy().astype(np.int64)
+    want = (sx[:, None] * w["s_w"][None, :] * (qx @ w["qw"].astype(np.int64).T)
+            + s_xl1[rt].cpu().numpy().astype(np.float64)[:, None]
+            * s_L2[ct].cpu().numpy().astype(np.float64)[None, :] * (gq @ gl2.T))
+    check_y(Y[rt][:, ct].double().cpu().numpy(), want, "prefill_gateup qlr")
