@@ -36,7 +36,8 @@ namespace {
 
 constexpr int kTok = 128;          // tokens per tile (MMA M)
 constexpr int kBlk = 128;          // columns per block (MMA N of the rotation, MMA K)
-constexpr int kNS = 2;             // X / L1^T stages
+constexpr int kMaxNS = 3;          // X / L1^T stages: three where they fit, else two
+constexpr int kRot = 2;            // rotation accumulators in TMEM (128 columns each)
 constexpr int kMaxC = 16;          // CTAs per cluster along K (above 8: non-portable size)
 constexpr int kMaxRtc = 128;       // X L1 width computed beside the codes
 constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
@@ -63,28 +64,38 @@ struct TcParams {
 // swizzled K-major tiles of 64 bf16 columns.  A stage holds one X block and,
 // when X L1 is computed, the matching L1^T block (2 atoms x r rows); an
 // X-L1-only launch has no Hadamard operand.
-constexpr int kNumBarsTc = 2 * kNS + 5;  // full[kNS], empty[kNS], rot_full[2], rot_empty[2], xl1_full
+constexpr int kNumBarsTc = 2 * kMaxNS + 2 * kRot + 1;  // full, empty; rot_full, rot_empty; xl1_full
 struct TcLayout {
   uint32_t h, stage0, stage, amax, amin, bar, misc, bytes;
+  int ns;  // stages
 };
-__host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
+__host__ __device__ inline TcLayout tc_layout_ns(bool xl1_only, int r, int ns) {
   TcLayout L;
+  L.ns = ns;
   L.h = 0;                                             // Hd^T: 2 atoms x 128 rows
   L.stage0 = xl1_only ? 0u : 2u * kBlk * 128u;
   L.stage = 2u * kTok * 128u + (uint32_t)r * 256u;     // X block + L1^T block
-  L.amax = L.stage0 + kNS * L.stage;                   // [C][128] fp32: absmax, or max
+  L.amax = L.stage0 + (uint32_t)ns * L.stage;          // [C][128] fp32: absmax, or max
   L.amin = L.amax + kMaxC * kTok * 4u;                 // [C][128] fp32: min (asymmetric)
   L.bar = L.amin + kMaxC * kTok * 4u;
   L.misc = L.bar + kNumBarsTc * 8u;
   L.bytes = L.misc + 16u;
   return L;
 }
-static_assert(2u * kBlk * 128u + kNS * (2u * kTok * 128u + kMaxRtc * 256u) + 2u * kMaxC * kTok * 4u +
+// Three stages when they fit (r <= 96 with the rotation; measured 5-8 %
+// faster than two at K >= 4096 and many tokens), else two.
+constexpr uint32_t kSmemCap = 227u * 1024u;  // dynamic shared memory of one CTA
+__host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
+  const TcLayout L3 = tc_layout_ns(xl1_only, r, kMaxNS);
+  return L3.bytes + 1024u <= kSmemCap ? L3 : tc_layout_ns(xl1_only, r, 2);
+}
+static_assert(2u * kBlk * 128u + 2u * (2u * kTok * 128u + kMaxRtc * 256u) + 2u * kMaxC * kTok * 4u +
                       kNumBarsTc * 8u + 16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (codes)");
-static_assert(kNS * (2u * kTok * 128u + kMaxRx * 256u) + 2u * kMaxC * kTok * 4u + kNumBarsTc * 8u +
+static_assert(2u * (2u * kTok * 128u + kMaxRx * 256u) + 2u * kMaxC * kTok * 4u + kNumBarsTc * 8u +
                       16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (X L1 only)");
+static_assert(kRot * kBlk + kMaxRtc <= 512 && kMaxRx <= 512, "tensor memory columns");
 // the X L1 receive area [C][128][ceil(r/C)] reuses the stages after pass 2:
 // 512 (r + C) bytes <= 2 (32 KB + 256 r) for every C <= 128
 
@@ -119,10 +130,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar);
   uint64_t* full = bars;
-  uint64_t* empty = bars + kNS;
-  uint64_t* rot_full = bars + 2 * kNS;
-  uint64_t* rot_empty = rot_full + 2;
-  uint64_t* xl1_full = rot_full + 4;
+  uint64_t* empty = bars + kMaxNS;
+  uint64_t* rot_full = bars + 2 * kMaxNS;
+  uint64_t* rot_empty = rot_full + kRot;
+  uint64_t* xl1_full = rot_full + 2 * kRot;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
@@ -143,7 +154,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   const bool resident = !xo && nb <= 2;
   const int n_loads = (xo || resident) ? nb : 2 * nb;
   auto issue_load = [&](int i, uint64_t pol_x, uint64_t pol_w) {
-    const int s = i % kNS;
+    const int s = i % L.ns;
     const bool second = xo || resident || i >= nb;
     const int j = i < nb ? i : i - nb;
     const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
@@ -158,15 +169,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tma_load_2d(smem + l1 + (uint32_t)r * 128u, &map_l1, &full[s], x + 64, p.r_off, pol_w);
     }
   };
-  const int n_pre = min(kNS, n_loads);  // stages requested in the prologue
+  const int n_pre = min(L.ns, n_loads);  // stages requested in the prologue
 
   // ---------------------------------------------------------------- prologue
   if (warp == 0 && lane == 0) {
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < kMaxNS; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kRot; ++i) {
       mbar_init(&rot_full[i], 1);
       mbar_init(&rot_empty[i], kEpiThreadsTc);
     }
@@ -224,8 +235,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_rot = tmem;        // 2 x 128 columns
-  const uint32_t tmem_xl1 = tmem + 256;  // r columns
+  const uint32_t tmem_rot = tmem;                           // kRot x 128 columns
+  const uint32_t tmem_xl1 = tmem + (xo ? 0u : kRot * kBlk);  // r columns
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -236,7 +247,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const uint64_t pol_x = policy_evict_last();    // read again in pass 2
       const uint64_t pol_w = policy_evict_first();
       for (int i = n_pre; i < n_loads; ++i) {
-        if (!mbar_wait(&empty[i % kNS], ((uint32_t)(i / kNS) & 1u) ^ 1u, nullptr, abort_flag))
+        if (!mbar_wait(&empty[i % L.ns], ((uint32_t)(i / L.ns) & 1u) ^ 1u, nullptr, abort_flag))
           break;
         issue_load(i, pol_x, pol_w);
       }
@@ -254,11 +265,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const uint32_t id_rot = idesc_bf16_f32(kBlk);
     const uint32_t id_xl1 = idesc_bf16_f32(r > 0 ? r : 16);
     for (int i = 0; i < n_loads; ++i) {
-      const int s = i % kNS, u = i & 1;
+      const int s = i % L.ns, u = i % kRot;
       const bool second = xo || resident || i >= nb;
       const int j = i < nb ? i : i - nb;
-      if (!mbar_wait(&full[s], (uint32_t)(i / kNS) & 1u, nullptr, abort_flag)) break;
-      if (!xo && !mbar_wait(&rot_empty[u], ((uint32_t)(i / 2) & 1u) ^ 1u, nullptr, abort_flag))
+      if (!mbar_wait(&full[s], (uint32_t)(i / L.ns) & 1u, nullptr, abort_flag)) break;
+      if (!xo && !mbar_wait(&rot_empty[u], ((uint32_t)(i / kRot) & 1u) ^ 1u, nullptr, abort_flag))
         break;
       tc_fence_after();
       if (lane == 0) {
@@ -302,8 +313,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     const bool asym = p.z_x != nullptr;
     float amax = 0.f, lo = __int_as_float(0x7f800000), hi = -__int_as_float(0x7f800000);
     for (int i = 0; i < (xo ? 0 : nb); ++i) {
-      const int u = i & 1;
-      const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u, nullptr,
+      const int u = i % kRot;
+      const bool ok = __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / kRot) & 1u, nullptr,
                                                   abort_flag));
       tc_fence_after();
       if (ok) {
@@ -352,9 +363,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     //      (inside each 32-code group byte i = code i | code i+16 << 4)
     for (int i = nb; i < (xo ? nb : 2 * nb); ++i) {
       // resident: block i - nb is still in its buffer from pass 1
-      const int u = resident ? i - nb : (i & 1);
+      const int u = resident ? i - nb : (i % kRot);
       const bool ok = resident ? !*abort_flag
-                               : __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / 2) & 1u,
+                               : __all_sync(kFull, mbar_wait(&rot_full[u], (uint32_t)(i / kRot) & 1u,
                                                              nullptr, abort_flag));
       tc_fence_after();
       if (ok) {
@@ -517,10 +528,9 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set >> dev & 1u)) {
-    const uint32_t most = std::max(tc_layout(false, kMaxRtc).bytes, tc_layout(true, kMaxRx).bytes) +
-                          1024u;
+    // every layout is at most kSmemCap (three stages only where they fit)
     cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)most);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(quantize_act_tc_kernel,
                              cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
