@@ -632,12 +632,12 @@ int num_sms_cached() {
 }
 
 
-Plan make_plan(int M, int N, int K, bool prefer_split) {
+Plan make_plan(int M, int N, int K) {
   Plan p{};
   const int kb = K / kKB;
-  if (M <= 128 || prefer_split) {
-    // Decode (and few channels, many tokens): weights on the MMA M side, split
-    // K over a cluster so that about one CTA per SM streams weights.
+  if (M <= 128) {
+    // Decode: weights on the MMA M side, split K over a cluster so that about
+    // one CTA per SM streams weights.
     p.swap = true;
     p.bn = M <= 16 ? 16 : (M <= 32 ? 32 : (M <= 64 ? 64 : 128));
     p.tiles_p = (N + kBM - 1) / kBM;
@@ -724,7 +724,7 @@ size_t gemm_workspace_bytes(int M, int N, int K, int r) {
 
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream) {
   const bool debug = a.acc_out != nullptr;
-  const Plan pl = make_plan(a.M, a.N, a.K, a.prefer_split != 0);
+  const Plan pl = make_plan(a.M, a.N, a.K);
   if (a.ws_bytes < gemm_workspace_bytes(a.M, a.N, a.K, a.r)) return cudaErrorInvalidValue;
   GemmParams prm{};
   prm.s_p = pl.swap ? a.s_w : a.s_x;

@@ -78,10 +78,9 @@ struct GemmArgs {
   const uint16_t* L2t;
   int M, N, K, r;
   uint16_t* Y;          // bf16 output (null in accumulator-debug mode)
-  int32_t* acc_out;     // raw accumulators (debug mode; the INT4 low-rank branch's X L1)
+  int32_t* acc_out;     // raw INT32 accumulators (debug mode), or null
   void* ws;
   size_t ws_bytes;
-  int prefer_split = 0;  // few channels, many tokens: the split-K plan for any M
 };
 
 size_t gemm_workspace_bytes(int M, int N, int K, int r);
