@@ -538,10 +538,13 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
     attr_set |= uint64_t(1) << dev;
   }
   // a cluster of C CTAs along K per 128-token tile: about one CTA per SM,
-  // and no larger than lets every cluster of the grid be resident at once
+  // and no larger than lets every cluster of the grid be resident at once.
+  // Stepping down one size at a time: 16 tiles of 2048 tokens take clusters
+  // of 8 (128 CTAs) where 9 do not all fit; halving fell to 4 (64 CTAs) and
+  // left more than half of the SMs idle.
   int C = std::max(1, std::min(kMaxC, num_sms() / tiles));
   C = std::min(C, p.kb_total);
-  for (;; C /= 2) {
+  for (;; --C) {
     p.nb = (p.kb_total + C - 1) / C;
     const int Ce = (p.kb_total + p.nb - 1) / p.nb;  // every CTA owns at least one block
     if (C <= 1) {
