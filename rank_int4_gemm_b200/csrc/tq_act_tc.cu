@@ -19,8 +19,9 @@
 //   then    X.L1 partial rows pushed to the CTA that owns the row, summed in
 //           cluster-rank order (deterministic) and stored.
 //
-// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-5:
-// TMEM readers (warp w reads lanes 32*(w%4)..: token rows of the tile).
+// Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-9:
+// TMEM readers, two per lane quarter (warp w reads lanes 32*(w%4)..: token
+// rows of the tile; warps 2-5 columns 0-63 of each block, warps 6-9 64-127).
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
@@ -41,9 +42,11 @@ constexpr int kRot = 2;            // rotation accumulators in TMEM (128 columns
 constexpr int kMaxC = 16;          // CTAs per cluster along K (above 8: non-portable size)
 constexpr int kMaxRtc = 128;       // X L1 width computed beside the codes
 constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
-constexpr int kThreadsTc = 192;
+// Readers: two warps per TMEM lane quarter, each taking half of a block's
+// 128 columns (one warp per quarter left the code pass issue-bound).
 constexpr int kEpiFirstWarp = 2;
-constexpr int kEpiThreadsTc = 128;
+constexpr int kEpiThreadsTc = 256;
+constexpr int kThreadsTc = 32 * kEpiFirstWarp + kEpiThreadsTc;
 
 struct TcParams {
   uint8_t* Xq;       // [M][K/2] packed codes, or null
@@ -75,9 +78,9 @@ __host__ __device__ inline TcLayout tc_layout_ns(bool xl1_only, int r, int ns) {
   L.h = 0;                                             // Hd^T: 2 atoms x 128 rows
   L.stage0 = xl1_only ? 0u : 2u * kBlk * 128u;
   L.stage = 2u * kTok * 128u + (uint32_t)r * 256u;     // X block + L1^T block
-  L.amax = L.stage0 + (uint32_t)ns * L.stage;          // [C][128] fp32: absmax, or max
-  L.amin = L.amax + kMaxC * kTok * 4u;                 // [C][128] fp32: min (asymmetric)
-  L.bar = L.amin + kMaxC * kTok * 4u;
+  L.amax = L.stage0 + (uint32_t)ns * L.stage;          // [C][2 halves][128] fp32: absmax, or max
+  L.amin = L.amax + 2u * kMaxC * kTok * 4u;           // [C][2][128] fp32: min (asymmetric)
+  L.bar = L.amin + 2u * kMaxC * kTok * 4u;
   L.misc = L.bar + kNumBarsTc * 8u;
   L.bytes = L.misc + 16u;
   return L;
@@ -89,10 +92,10 @@ __host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
   const TcLayout L3 = tc_layout_ns(xl1_only, r, kMaxNS);
   return L3.bytes + 1024u <= kSmemCap ? L3 : tc_layout_ns(xl1_only, r, 2);
 }
-static_assert(2u * kBlk * 128u + 2u * (2u * kTok * 128u + kMaxRtc * 256u) + 2u * kMaxC * kTok * 4u +
+static_assert(2u * kBlk * 128u + 2u * (2u * kTok * 128u + kMaxRtc * 256u) + 4u * kMaxC * kTok * 4u +
                       kNumBarsTc * 8u + 16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (codes)");
-static_assert(2u * (2u * kTok * 128u + kMaxRx * 256u) + 2u * kMaxC * kTok * 4u + kNumBarsTc * 8u +
+static_assert(2u * (2u * kTok * 128u + kMaxRx * 256u) + 4u * kMaxC * kTok * 4u + kNumBarsTc * 8u +
                       16u + 1024u <= 227u * 1024u,
               "activation tile shared memory (X L1 only)");
 static_assert(kRot * kBlk + kMaxRtc <= 512 && kMaxRx <= 512, "tensor memory columns");
@@ -303,6 +306,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   } else {
     // ===================================================== TMEM readers
     const int q = warp & 3;                       // TMEM lane quarter
+    const int half = (warp - kEpiFirstWarp) >> 2;  // columns [64 half, 64 half + 64) of a block
     const int row = q * 32 + lane;                // token row in the tile
     const int grow = tile * kTok + row;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
@@ -319,7 +323,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       tc_fence_after();
       if (ok) {
 #pragma unroll
-        for (int g = 0; g < kBlk / 32; ++g) {
+        for (int g = 2 * half; g < 2 * half + 2; ++g) {
           uint32_t v[32];
           tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
           tmem_ld_wait();
@@ -337,7 +341,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     }
     if (!xo)
       for (uint32_t z = 0; z < csize; ++z) {
-        const uint32_t off = (crank * kTok + (uint32_t)row) * 4u;
+        const uint32_t off = ((crank * 2u + (uint32_t)half) * kTok + (uint32_t)row) * 4u;
         dsmem_st_f32(dsmem_map(base + L.amax + off, z), asym ? hi : amax);
         if (asym) dsmem_st_f32(dsmem_map(base + L.amin + off, z), lo);
       }
@@ -345,14 +349,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
     cluster_wait_acquire();
     float am = asym ? -__int_as_float(0x7f800000) : 0.f;
     float mn = __int_as_float(0x7f800000);
-    for (uint32_t z = 0; z < csize; ++z) {
+    for (uint32_t z = 0; z < 2u * csize; ++z) {  // every CTA's two halves
       am = fmaxf(am, ld_shared_f32_tc(base + L.amax + (z * kTok + (uint32_t)row) * 4u));
       if (asym) mn = fminf(mn, ld_shared_f32_tc(base + L.amin + (z * kTok + (uint32_t)row) * 4u));
     }
     // asymmetric: codes of (x - min) over the range max - min, in [0, 15]
     // (stored as code - 8), scale range / 15, zero-point min
     const float range = asym ? am - mn : am;
-    if (!xo && crank == 0 && grow < p.M) {
+    if (!xo && crank == 0 && half == 0 && grow < p.M) {
       p.s_x[grow] = range * p.scale_mul;
       if (asym) p.z_x[grow] = mn * p.zmul;
     }
@@ -371,7 +375,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       if (ok) {
         const size_t blk = (size_t)(kb0 + i - nb);
 #pragma unroll
-        for (int g = 0; g < kBlk / 32; ++g) {
+        for (int g = 2 * half; g < 2 * half + 2; ++g) {
           uint32_t v[32];
           tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
           tmem_ld_wait();
@@ -433,7 +437,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int owner = row / rpo;
       const uint32_t dst = dsmem_map(recv + (uint32_t)(((int)crank * rpo + row - owner * rpo) * r) * 4u,
                                      (uint32_t)owner);
-      for (int c0 = 0; c0 < r; c0 += 16) {
+      for (int c0 = 16 * half; c0 < r; c0 += 32) {  // the two halves alternate 16-column chunks
         uint32_t v[16];
         tmem_ld16(tmem_xl1 + (uint32_t)c0 + lane_off, v);
         tmem_ld_wait();
