@@ -85,7 +85,7 @@ __host__ __device__ inline TcLayout tc_layout_ns(bool xl1_only, int r, int ns) {
   L.bytes = L.misc + 16u;
   return L;
 }
-// Three stages when they fit (r <= 96 with the rotation; measured 5-8 %
+// Three stages when they fit (r <= 80 with the rotation; measured 5-8 %
 // faster than two at K >= 4096 and many tokens), else two.
 constexpr uint32_t kSmemCap = 227u * 1024u;  // dynamic shared memory of one CTA
 __host__ __device__ inline TcLayout tc_layout(bool xl1_only, int r) {
