@@ -1,6 +1,6 @@
 """Seeded synthetic layer inputs (activations, low-rank factors, residual).
 
-Recipe (one reading per point, all of them listed in the design doc):
+Recipe (one reading of the pages per point):
 
 * X is bf16 with N(0,1) elements; a seeded choice of input channels is scaled
   (x20 on 2 of 256 channels for the tiny layer, x30 on round(0.01*K) channels
