@@ -87,11 +87,23 @@ TQ_API int tq_pack_weight(const float* Rt, int N, int K, int had_block,
                    uint8_t* Wq, float* s_w, void* stream);
 
 /*
- * tq_quantize_act -- online rotation X H (one 128-wide or had_block-wide
- * fast Walsh-Hadamard transform per block), symmetric per-token INT4
- * quantization (CoQuant Eq. (1); TwinQuant notes section 02) and the
- * low-rank down-projection X L1 (TwinQuant notes section 02.A), all from one
- * read of X.
+ * tq_quantize_act -- online rotation X H (CoQuant Eq. (3), block Hadamard),
+ * symmetric per-token INT4 quantization (CoQuant Eq. (1); TwinQuant notes
+ * section 02) and the low-rank down-projection X L1 (TwinQuant notes
+ * section 02.A).  Two kernels serve it:
+ *  - M >= 64 with had_block <= 128: 128-token tiles on the tensor cores.  The
+ *    rotation of each 128-column block is a bf16 MMA against the
+ *    block-diagonal +-1 Sylvester matrix (exact products, fp32 accumulation)
+ *    and X L1 a second MMA on the same staged tile.  X is read twice: the
+ *    first pass takes the per-token absmax across a thread-block cluster,
+ *    the second (served from L2) recomputes the rotation and writes codes.
+ *    Ranks above 128 run X L1 in extra launches of at most 256 columns.
+ *  - otherwise (few tokens, or had_block = 256): an in-register and
+ *    warp-shuffle fast Walsh-Hadamard transform per block, X L1 on mma.sync,
+ *    all from one read of X; K is split over a thread-block cluster that
+ *    combines the absmax and the X L1 partials in distributed shared memory.
+ * Both give the same codes up to the midpoint allowance of the fp32
+ * summation order.
  *
  *   X    [M][K] bf16    in : activations
  *   L1t  [r][K] bf16    in : L1^T (down-projection weight); NULL iff r == 0
@@ -333,16 +345,23 @@ TQ_API int tq_debug_w4a4_gemm_acc(const uint8_t* Xq, const uint8_t* Wq,
  * library's own device memory, which every GPU that loads the library keeps
  * until the process exits.  Nothing is allocated on any call.
  *
- *  - Shapes needing more scratch than tq_gemm_workspace_bytes() = 256 bytes
- *    are rejected with TQ_ERR_WORKSPACE before anything runs.
- *  - The first call on a device looks up that array's device address (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.
- *  - Every call clears the array on `stream` before its kernel and every call
- *    shares it, so calls that overlap on the GPU (different streams with no
- *    ordering between them) race on it.
- *  - A watchdog timeout in this variant is recorded only in that shared
- *    array and is not reported by tq_query_device_status.
+ *  - Argument errors are returned before any device work, in the same order
+ *    as tq_w4a4_lr_gemm.  Shapes needing more scratch than
+ *    tq_gemm_workspace_bytes() = 256 bytes are rejected with
+ *    TQ_ERR_WORKSPACE.
+ *  - The first call in a CUDA context looks up that array's device address
+ *    (with that context current) and caches it per context; make that first
+ *    call before any stream capture.
+ *  - Every call shares the array, which keeps what the last call left in it.
+ *    Nothing in it needs to start at zero for the result: the kernel writes
+ *    only the status word, and only when a bounded wait gives up.  Calls that
+ *    overlap on the GPU (different streams with no ordering between them)
+ *    race on it.
+ *  - tq_noalloc_query_status(stream) synchronises `stream`, then reads and
+ *    clears that status word: TQ_OK, or TQ_ERR_TIMEOUT if a bounded wait of
+ *    any no-allocation call in this context gave up since the last query.
+ *  - tq_debug_noalloc_set_status(status) is a test hook: it writes `status`
+ *    into that word (synchronously, no kernel).
  * The pages have no counterpart of this entry point; it is an addition of
  * this library.
  */
@@ -351,6 +370,23 @@ TQ_API int tq_w4a4_lr_gemm_noalloc(const uint8_t* Xq, const float* s_x,
                                    const float* XL1, const uint16_t* L2t,
                                    int M, int N, int K, int r, uint16_t* Y,
                                    void* stream);
+TQ_API int tq_noalloc_query_status(void* stream);
+TQ_API int tq_debug_noalloc_set_status(int status);
+
+/*
+ * tq_debug_watchdog -- test hook for the bounded waits every pipelined
+ * kernel here uses.  Launches one CTA (no cluster) in which a producer lane
+ * arrives on an mbarrier, unless `withhold` is non-zero, and a consumer lane
+ * waits for that arrival with the library's bounded wait, giving up after
+ * `budget_cycles` SM cycles (1000 .. 2e9).  A wait that gives up writes
+ * TQ_ERR_TIMEOUT into the status word at the start of `workspace` (>= 256
+ * bytes, a GEMM workspace), read back by tq_query_device_status; the kernel
+ * then returns normally and the context stays usable.  *waited_ok (a device
+ * int) is set to 1 when the arrival was seen, 0 when the wait gave up.
+ * No counterpart on the pages: it tests the library's own failure handling.
+ */
+TQ_API int tq_debug_watchdog(void* workspace, size_t workspace_bytes, int withhold,
+                             long long budget_cycles, int* waited_ok, void* stream);
 
 /*
  * tq_query_device_status -- synchronises `stream`, then reads the status word

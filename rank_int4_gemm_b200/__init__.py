@@ -12,4 +12,5 @@ from .tq import (  # noqa: F401
     tq_quantize_act_i8, tq_w4a4_lr_gemm_a8, tq_layer_path, tq_pack_gate_up,
     tq_gate_up_workspace_bytes, tq_w4a4_lr_gate_up, tq_quantize_act_asym_i8, tq_weight_code_sums,
     tq_w4a4_lr_gemm_a8_asym, tq_pack_lowrank_q4, tq_quantize_act_qlr_i8, tq_w4a4_lr_gemm_a8_qlr,
+    tq_noalloc_query_status, tq_debug_noalloc_set_status, tq_debug_watchdog,
 )

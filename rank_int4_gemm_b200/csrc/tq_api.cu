@@ -45,6 +45,31 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
 
 }  // namespace
 
+namespace tq {
+
+// Argument checks of the packed-code GEMM's operands (everything except the
+// workspace and the device), in the order every GEMM entry applies them.
+int gemm_operand_status(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w,
+                        const float* XL1, const uint16_t* L2t, int M, int N, int K, int r,
+                        const uint16_t* Y, const int32_t* acc) {
+  if (!Xq || !Wq || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (!Y && !acc) return TQ_ERR_INVALID_VALUE;
+  if (Y && (!s_x || !s_w)) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (XL1 != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Xq) || !aligned16(Wq) || (s_x && !aligned16(s_x)) ||
+      (s_w && !aligned16(s_w)) || (XL1 && !aligned16(XL1)) || (L2t && !aligned16(L2t)) ||
+      (Y && !aligned16(Y)) || (acc && !aligned16(acc)))
+    return TQ_ERR_MISALIGNED;
+  return TQ_OK;
+}
+
+int device_status() { return check_device(); }
+
+}  // namespace tq
+
 extern "C" {
 
 const char* tq_status_string(int status) {
@@ -95,17 +120,8 @@ size_t tq_gemm_workspace_bytes(int M, int N, int K, int r) {
 static int gemm_common(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w,
                        const float* XL1, const uint16_t* L2t, int M, int N, int K, int r,
                        uint16_t* Y, int32_t* acc, void* ws, size_t ws_bytes, void* stream) {
-  if (!Xq || !Wq || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
-  if (!Y && !acc) return TQ_ERR_INVALID_VALUE;
-  if (Y && (!s_x || !s_w)) return TQ_ERR_INVALID_VALUE;
-  if (int s = check_k(K, 1)) return s;
-  if (int s = check_r(r)) return s;
-  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
-  if ((r > 0) != (XL1 != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
-  if (!aligned16(Xq) || !aligned16(Wq) || (s_x && !aligned16(s_x)) ||
-      (s_w && !aligned16(s_w)) || (XL1 && !aligned16(XL1)) || (L2t && !aligned16(L2t)) ||
-      (Y && !aligned16(Y)) || (acc && !aligned16(acc)) || (ws && !aligned16(ws)))
-    return TQ_ERR_MISALIGNED;
+  if (int s = tq::gemm_operand_status(Xq, s_x, Wq, s_w, XL1, L2t, M, N, K, r, Y, acc)) return s;
+  if (ws && !aligned16(ws)) return TQ_ERR_MISALIGNED;
   if (!ws || ws_bytes < tq::gemm_workspace_bytes(M, N, K, r)) return TQ_ERR_WORKSPACE;
   if (int s = check_device()) return s;
   tq::GemmArgs a{};

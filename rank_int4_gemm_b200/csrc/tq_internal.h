@@ -84,6 +84,13 @@ struct GemmArgs {
 };
 
 size_t gemm_workspace_bytes(int M, int N, int K, int r);
+// Status of the GEMM's operand arguments (null pointers, shape limits,
+// alignment), without the workspace and device checks; TQ_OK when valid.
+int gemm_operand_status(const uint8_t* Xq, const float* s_x, const uint8_t* Wq, const float* s_w,
+                        const float* XL1, const uint16_t* L2t, int M, int N, int K, int r,
+                        const uint16_t* Y, const int32_t* acc);
+// TQ_OK when the current device is an sm_100 GPU, else TQ_ERR_NO_DEVICE.
+int device_status();
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream);
 
 // The whole layer from bf16 X (decode sizes: one fused kernel).

@@ -85,23 +85,67 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitBudgetCycles: records kDevTimeout in *status (if not null), raises the
-// CTA-wide abort flag and returns false.  Callers stop their role loop then.
+// `budget` cycles (kWaitBudgetCycles unless a test passes a shorter one):
+// records kDevTimeout in *status (if not null), raises the CTA-wide abort
+// flag and returns false.  Callers stop their role loop then.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint32_t* status, volatile int* abort_flag) {
+                                          uint32_t* status, volatile int* abort_flag,
+                                          long long budget = kWaitBudgetCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_sleep(bar, parity, 200u)) return true;
     if ((it & 15u) == 15u) {
       if (abort_flag && *abort_flag) return false;
-      if (clock64() - t0 > kWaitBudgetCycles) {
+      if (clock64() - t0 > budget) {
         if (status) atomicExch(status, kDevTimeout);
         if (abort_flag) *abort_flag = 1;
         return false;
       }
     }
   }
+}
+
+// try_wait with acquire semantics at cluster scope: for barriers whose
+// transactions are stores from other CTAs of the cluster (st.async).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait for such a barrier (same budget, status and abort rules).
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  uint32_t* status, volatile int* abort_flag,
+                                                  long long budget = kWaitBudgetCycles) {
+  if (mbar_try_wait_cluster(bar, parity, 0u)) return true;
+  long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster(bar, parity, 200u)) return true;
+    if ((it & 15u) == 15u) {
+      if (abort_flag && *abort_flag) return false;
+      if (clock64() - t0 > budget) {
+        if (status) atomicExch(status, kDevTimeout);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// 16 bytes into the shared memory of a CTA of this cluster (addresses from
+// mapa), completing as transaction bytes on that CTA's mbarrier `rbar`.
+__device__ __forceinline__ void st_async_v4(uint32_t raddr, uint4 v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(raddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(rbar)
+      : "memory");
 }
 
 // ------------------------------------------------------------------- TMA

@@ -40,6 +40,12 @@ _lib.tq_debug_w4a4_gemm_acc.restype = _I
 _lib.tq_debug_w4a4_gemm_acc.argtypes = [_P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
 _lib.tq_w4a4_lr_gemm_noalloc.restype = _I
 _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.tq_debug_watchdog.restype = _I
+_lib.tq_debug_watchdog.argtypes = [_P, ctypes.c_size_t, _I, ctypes.c_longlong, _P, _P]
+_lib.tq_noalloc_query_status.restype = _I
+_lib.tq_noalloc_query_status.argtypes = [_P]
+_lib.tq_debug_noalloc_set_status.restype = _I
+_lib.tq_debug_noalloc_set_status.argtypes = [_I]
 _lib.tq_layer_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_layer_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_layer_path.restype = _I
@@ -356,6 +362,30 @@ def tq_w4a4_lr_gemm_noalloc(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, stream
                                         M, N, K, r, _ptr(Y), _stream(stream)),
            "tq_w4a4_lr_gemm_noalloc")
     return Y
+
+
+def tq_debug_watchdog(workspace, withhold: bool, budget_cycles: int, waited_ok=None,
+                      stream=None):
+    """Test hook of the bounded waits: one CTA whose consumer waits (at most
+    budget_cycles) for a producer arrival that `withhold` suppresses.
+    Returns the device int set to 1 (arrival seen) or 0 (wait gave up)."""
+    ws = workspace.get(256) if isinstance(workspace, Workspace) else workspace
+    if waited_ok is None:
+        waited_ok = torch.full((1,), -1, dtype=torch.int32, device=ws.device)
+    _check(_lib.tq_debug_watchdog(_ptr(ws), ws.numel(), int(bool(withhold)), int(budget_cycles),
+                                  _ptr(waited_ok), _stream(stream)), "tq_debug_watchdog")
+    return waited_ok
+
+
+def tq_noalloc_query_status(stream=None) -> int:
+    """Status word of the no-allocation entry point's scratch (synchronises
+    the stream, reads and clears it): 0, or 5 (TQ_ERR_TIMEOUT)."""
+    return int(_lib.tq_noalloc_query_status(_stream(stream)))
+
+
+def tq_debug_noalloc_set_status(status: int) -> None:
+    """Test hook: write `status` into that word (synchronous, no kernel)."""
+    _check(_lib.tq_debug_noalloc_set_status(int(status)), "tq_debug_noalloc_set_status")
 
 
 def tq_debug_w4a4_gemm_acc(Xq, Wq, acc=None, workspace=None, stream=None):

@@ -69,6 +69,16 @@ def check_y(gpu_y, y64, what="Y"):
     return fro, mx
 
 
+def y_reference(gpu_codes, o, flips):
+    """The reference for Y: the oracle's fp64 Y64 when the GPU's codes equal
+    the oracle's (flips == 0), else the oracle's epilogue on the GPU's codes.
+    The second case is only reached after check_codes has shown that every
+    difference is an allowed midpoint flip: one flip moves a token's whole
+    row of Y by s_x s_w q_w, which the output tolerance is not meant to
+    absorb (it can reach 2e-3 relative Frobenius alone)."""
+    return o["Y64"] if flips == 0 else y_given_codes(gpu_codes, o)
+
+
 def y_given_codes(gpu_codes, o):
     """The oracle's epilogue evaluated on the GPU's activation codes (already
     checked by check_codes to differ from the oracle's only by midpoint

@@ -85,6 +85,20 @@ def test_gemm_validation(lib):
     assert lib.tq_gemm_workspace_bytes(1, 4096, 4096, 32) >= 256
 
 
+def test_noalloc_validation(lib):
+    # the no-allocation entry checks its arguments before any device work
+    f = lib.tq_w4a4_lr_gemm_noalloc
+    args = lambda **k: [k.get("Xq", P(FAKE)), P(FAKE), P(FAKE), P(FAKE), k.get("XL1"),
+                        k.get("L2t"), k.get("M", 4), k.get("N", 64), k.get("K", 256),
+                        k.get("r", 0), k.get("Y", P(FAKE)), None]
+    assert f(*args(Y=None)) == 1
+    assert f(*args(Xq=None)) == 1
+    assert f(*args(N=60)) == 2
+    assert f(*args(K=200)) == 2
+    assert f(*args(r=16)) == 1
+    assert f(*args(r=16, XL1=P(FAKE), L2t=P(FAKE + 2))) == 3
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU path")
 def test_no_device_is_reported(lib):
     # Valid-looking arguments pass validation, then the device check fails

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 import synth
-from tests.parity_util import check_codes, check_y, y_given_codes
+from tests.parity_util import check_codes, check_y, y_reference
 
 
 def test_swiglu_closed_forms():
@@ -47,6 +47,7 @@ CASES = [
     ("one_token", 1, 512, 128, 16, 64),
     ("rank0", 200, 512, 136, 0, 128),
     ("wide_rank", 150, 512, 256, 128, 32),
+    ("no_rotation", 140, 512, 136, 32, 1),
 ]
 
 
@@ -65,22 +66,24 @@ def test_gate_up_matches_oracle(tq, name, M, K, N, r, b):
     Y = tq.tq_w4a4_lr_gate_up(X, L1t2, Wq2, s_w2, L2t2, b)
     # the same pair as an ordinary layer of 2N interleaved channels
     Ycat = tq.tq_w4a4_lr_layer(X, L1t2, Wq2, s_w2, L2t2, b)
+    # the pair's codes (one activation pass; the codes do not depend on the
+    # rank): midpoint flips allowed
+    Xq8, _, _ = tq.tq_quantize_act_i8(X, b)
     torch.cuda.synchronize()
     og = oracle.layer(g["X"], g["L1t"], g["L2t"], g["Rt"], b)
     ou = oracle.layer(u["X"], u["L1t"], u["L2t"], u["Rt"], b)
+    q8 = Xq8.cpu().numpy().astype(np.int64)
+    fx = check_codes(q8, og["qx"], og["t_x"], f"{name}: activation codes", packed=False)
+    # references: the oracle's fp64 outputs, or, where the codes hold allowed
+    # flips (one flip moves a token's whole row of both g and u), the
+    # oracle's epilogue on these codes
+    yg, yu = y_reference(q8, og, fx), y_reference(q8, ou, fx)
     # the interleaved layer: gate channels on even rows, up on odd rows
     yc = Ycat.double().cpu().numpy()
-    check_y(yc[:, 0::2], og["Y64"], f"{name}: pair layer, gate channels")
-    check_y(yc[:, 1::2], ou["Y64"], f"{name}: pair layer, up channels")
-    # the pair's codes (one activation pass; the codes do not depend on the
-    # rank): midpoint flips allowed, and the reference is silu(g) * u of the
-    # oracle's epilogue on these codes, since one flip moves a token's whole
-    # row of both g and u
-    Xq8, _, _ = tq.tq_quantize_act_i8(X, b)
-    torch.cuda.synchronize()
-    q8 = Xq8.cpu().numpy().astype(np.int64)
-    check_codes(q8, og["qx"], og["t_x"], f"{name}: activation codes", packed=False)
-    want = oracle.swiglu(y_given_codes(q8, og), y_given_codes(q8, ou))
+    check_y(yc[:, 0::2], yg, f"{name}: pair layer, gate channels")
+    check_y(yc[:, 1::2], yu, f"{name}: pair layer, up channels")
+    # the fused pair: silu(g) * u of those references
+    want = oracle.swiglu(yg, yu)
     y = Y.double().cpu().numpy()
     # in Frobenius norm: within the layer bound, or, where a few elements
     # dominate the norm (one token), within 1.1 x what rounding the exact
