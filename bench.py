@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=LAYERS)
     ap.add_argument("--no-sweep", action="store_true", help="skip the M=1/128 side measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the prefill configurations and the rank-overhead point")
     ap.add_argument("--profile", action="store_true",
                     help="replay only the timed step graph (for a profiler); prints one status line")
     ap.add_argument("--workload", default="decode",
@@ -120,7 +122,7 @@ def profiled_traffic(kernel_src: str, profile: str):
 class ClockSampler:
     """Samples SM clocks and throttle reasons through NVML while running."""
 
-    def __init__(self, index: int, period: float = 0.02):
+    def __init__(self, index: int, period: float = 0.005):
         self.index, self.period = index, period
         self.samples, self.reasons = [], set()
         self.max_mhz = None
@@ -182,8 +184,8 @@ def build_layers(tq, torch, M, L, seed0, device):
         w = synth.make_weights(sh, seed=seed0 + 10 * i, device="cuda")
         Rt = w["Rt"].to(device)
         Wq, s_w = tq.tq_pack_weight(Rt, HAD)
-        del Rt
         lay = {
+            "Rt": Rt if i == 0 else None,
             "X": synth.make_activations(sh, seed=seed0 + 10 * i).to(device),
             "L1t": w["L1t"].to(device), "L2t": w["L2t"].to(device), "Wq": Wq, "s_w": s_w,
             "Xq": torch.empty(M, K_DIM // 2, dtype=torch.uint8, device=device),
@@ -400,52 +402,120 @@ def run_tq(args, rank, world, local_rank, dist):
     }
     if sweep:
         out["sweep"] = sweep
+
+    # the flip fraction of the decode layers: codes of the bench's first
+    # layer from the timed path, against the oracle (in the baseline leg)
+    dec_codes = decode_codes_sample(tq, torch, layers[0])
+    dec_cpu = {k: v.cpu() for k, v in decode_cpu_inputs(layers[0]).items()}
+    del layers, g, g_ev, g_e2e
+
+    # the prefill configurations and the rank overhead, measured in the same
+    # process (one GPU only: they are reported beside the decode metric)
+    prefill, pre_cpu = {}, {}
+    if world == 1 and not args.no_prefill:
+        import synth
+        steps_p, warm_p = max(5, min(args.steps, 20)), max(3, min(args.warmup, 5))
+        for name in PREFILL_CONFIGS:
+            sh = synth.CONFIGS[name]
+            lays, per_layer = prefill_layers(tq, torch, sh, sh.M, dev, rank, keep_cpu=True)
+            pt, _ = prefill_point(tq, torch, sh, sh.M, lays, per_layer, steps_p, warm_p, rank,
+                                  local_rank)
+            prefill[name] = pt
+            pre_cpu[name] = (sh, lays[0]["cpu"],
+                             prefill_codes_sample(tq, torch, lays[0], sh, range(CPU_SLICE)))
+            del lays
+            torch.cuda.empty_cache()
+        out["prefill"] = prefill
+        ro = {}
+        for r in (0, 64):
+            sh = synth.CONFIGS["sweep"].with_(r=r)
+            lays, per_layer = prefill_layers(tq, torch, sh, sh.M, dev, rank)
+            ro[r], _ = prefill_point(tq, torch, sh, sh.M, lays, per_layer, steps_p, warm_p, rank,
+                                     local_rank)
+            del lays
+            torch.cuda.empty_cache()
+        out["rank_overhead"] = {
+            "workload": "roofline sweep point M = K = N = 4096, Hadamard block 128: rank 64 "
+                        "against rank 0, layer time (activation kernel + GEMM)",
+            "us_rank0": ro[0]["us_per_layer"], "us_rank64": ro[64]["us_per_layer"],
+            "ratio": round(ro[64]["us_per_layer"] / ro[0]["us_per_layer"], 4),
+            "gemm_us_rank0": ro[0]["gemm_us"], "gemm_us_rank64": ro[64]["gemm_us"],
+            "gemm_ratio": round(ro[64]["gemm_us"] / ro[0]["gemm_us"], 4),
+            "target_ratio_at_most": 1.10,
+            "TOPS_rank0": ro[0]["TOPS"], "TOPS_rank64": ro[64]["TOPS"],
+            "clocks": ro[64]["clocks"],
+        }
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(M, budget_s=12.0)
+        cb, parity = cpu_baseline(M, budget_s=12.0, decode=(dec_cpu, dec_codes),
+                                  prefill=pre_cpu)
+        out["cpu_baseline"] = cb
+        out["parity"] = parity
     return out
+
+
+def decode_cpu_inputs(lay):
+    return {"X": lay["X"], "L1t": lay["L1t"], "L2t": lay["L2t"], "Rt": lay["Rt"]}
+
+
+def decode_codes_sample(tq, torch, lay):
+    """Codes and scales of the decode layer's tokens as the timed path makes
+    them, and its weight codes (host copies), for the flip fraction."""
+    Xq, s_x, _ = tq.tq_quantize_act(lay["X"], HAD, lay["L1t"])
+    torch.cuda.synchronize()
+    return {"Xq": Xq.cpu().numpy(), "s_x": s_x.cpu().numpy(), "Wq": lay["Wq"].cpu().numpy(),
+            "s_w": lay["s_w"].cpu().numpy(), "b": HAD,
+            "source": "tq_quantize_act on the bench's first decode layer (the fused kernel "
+                      "computes the same codes internally and does not store them)"}
 
 
 # --------------------------------------------------------------- prefill arm
 
-def run_prefill(args, rank, world, local_rank, dist):
-    """One prefill layer per step (act + GEMM), over enough distinct layers
-    that the step's operands exceed L2; TOPS = 2 M N K per layer / time."""
-    import torch
+PREFILL_CONFIGS = ("prefill_gateup", "prefill_down", "large_gateup", "large_down")
 
-    import rank_int4_gemm_b200 as tq
-    import synth
 
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    sh = synth.CONFIGS[args.workload]
-    if args.rank is not None:
-        sh = sh.with_(r=args.rank)
-    M = args.m if args.m != 16 else sh.M
+def prefill_layers(tq, torch, sh, M, dev, rank, layers_cap=16, keep_cpu=False):
+    """Distinct layers of one prefill shape, enough that a step's operands
+    exceed L2 (about 200 MB), with every buffer the timed calls use."""
     K, N, r, b = sh.K, sh.N, sh.r, sh.had_block
     per_layer = 2 * M * K + K * N // 2 + 2 * M * N
-    L = max(1, min(args.layers, -(-200_000_000 // per_layer)))
+    L = max(1, min(layers_cap, -(-200_000_000 // per_layer)))
+    import synth
     layers = []
     for i in range(L):
-        w = synth.make_weights(sh, seed=replica_seed(rank) + 10 * i, device="cuda")
-        Rt = w["Rt"].to(dev)
-        Wq, s_w = tq.tq_pack_weight(Rt, b)
-        del Rt
-        layers.append({
-            "X": synth.make_activations(sh, seed=replica_seed(rank) + 10 * i, M=M).to(dev),
-            "L1t": w["L1t"].to(dev) if r else None, "L2t": w["L2t"].to(dev) if r else None,
-            "Wq": Wq, "s_w": s_w,
+        seed = replica_seed(rank) + 10 * i
+        w = synth.make_weights(sh, seed=seed, device="cuda")
+        X = synth.make_activations(sh, seed=seed, M=M)
+        Wq, s_w = tq.tq_pack_weight(w["Rt"].to(dev), b)
+        lay = {
+            "X": X.to(dev), "L1t": w["L1t"].to(dev) if r else None,
+            "L2t": w["L2t"].to(dev) if r else None, "Wq": Wq, "s_w": s_w,
             "Xq": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
             "Xq8": torch.empty(M, K, dtype=torch.int8, device=dev),
             "s_x": torch.empty(M, dtype=torch.float32, device=dev),
             "XL1": torch.empty(M, r, dtype=torch.float32, device=dev) if r else None,
             "XL1b": torch.empty(M, r, dtype=torch.bfloat16, device=dev) if r else None,
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
-            "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8, device=dev),
-        })
-    # the kernels tq_w4a4_lr_layer runs for this shape (codes one per byte
-    # for M > 128 and b <= 128), timed here call by call
-    a8 = tq.tq_layer_path(M, N, K, r, b) == "codes_i8"
+            "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8,
+                              device=dev),
+        }
+        if keep_cpu and i == 0:
+            lay["cpu"] = {"X": X, "Rt": w["Rt"], "L1t": w["L1t"], "L2t": w["L2t"]}
+        del w
+        layers.append(lay)
     torch.cuda.synchronize()
+    return layers, per_layer
+
+
+def prefill_point(tq, torch, sh, M, layers, per_layer, steps, warmup, rank, local_rank,
+                  dist=None, world=1, packed_too=False):
+    """Times one prefill shape: a step is one layer call (activation kernel +
+    GEMM, the kernels tq_w4a4_lr_layer runs for the shape) per distinct
+    layer, replayed as a CUDA graph.  Reports the layer's TOPS (2 M N K per
+    layer over the layer time, the quantity the INT8 target is set on) and
+    the GEMM's alone, both as fractions of the dense INT8 peak."""
+    K, N, r, b = sh.K, sh.N, sh.r, sh.had_block
+    L = len(layers)
+    a8 = tq.tq_layer_path(M, N, K, r, b) == "codes_i8"
 
     def one(lay, ev=None, packed=not a8):
         if ev is not None:
@@ -468,60 +538,121 @@ def run_prefill(args, rank, world, local_rank, dist):
             ev[1].record()
 
     g = capture(torch, lambda: [one(l) for l in layers])
-    if args.profile:
-        time_graph(torch, g, args.steps, args.warmup)
-        return {"profile": f"{args.workload} step graph", "layers": L, "steps": args.steps,
-                "warmup": args.warmup}
     with ClockSampler(local_rank) as clk:
-        ms = time_graph(torch, g, args.steps, args.warmup, dist if world > 1 else None)
-    ms = max_over_ranks(ms, dist if world > 1 else None, dev)
+        ms = time_graph(torch, g, steps, warmup, dist if world > 1 else None)
+    ms = max_over_ranks(ms, dist if world > 1 else None, torch.device("cuda", local_rank))
+    del g
     evs = [tuple(torch.cuda.Event(enable_timing=True, external=True) for _ in range(3))
            for _ in layers]
     g_ev = capture(torch, lambda: [one(l, e) for l, e in zip(layers, evs)])
     gemm_ms, act_ms = [], []
     for _ in range(3):
         g_ev.replay()
-    for _ in range(max(1, min(args.steps, 20))):
+    for _ in range(max(1, min(steps, 20))):
         g_ev.replay()
         torch.cuda.synchronize()
         gemm_ms.extend(e[0].elapsed_time(e[1]) for e in evs)
         act_ms.extend(e[2].elapsed_time(e[0]) for e in evs)
-    gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
-    act_ms_avg = sum(act_ms) / len(act_ms)
-    ops = 2 * M * N * K
-    packed_ms = None
-    if a8:
+    del g_ev
+    gemm_us = sum(gemm_ms) / len(gemm_ms) * 1e3
+    act_us = sum(act_ms) / len(act_ms) * 1e3
+    layer_us = ms * 1e3 / L
+    packed_us = None
+    if a8 and packed_too:
         g_p = capture(torch, lambda: [one(l, packed=True) for l in layers])
-        packed_ms = time_graph(torch, g_p, args.steps, args.warmup)
+        packed_us = time_graph(torch, g_p, steps, warmup) * 1e3 / L
         del g_p
+    ops = 2 * M * N * K
     peak, src = int8_peak(sustained=False)
-    achieved = ops / (gemm_ms_avg * 1e-3) / 1e12
+    peak_s, _ = int8_peak(sustained=True)
+    tops_layer = ops / (layer_us * 1e-6) / 1e12
+    tops_gemm = ops / (gemm_us * 1e-6) / 1e12
+    c = clk.summary()
     out = {
-        "metric": METRIC, "value": round(whole_job(L * ops, world, ms) / 1e12, 2), "unit": "TOPS",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "int4", "data": "synthetic",
-        "config": {"workload": f"{args.workload}: M={M}, K={K}, N={N}, rank {r}, Hadamard "
-                               f"block {b}; {L} distinct layer(s) per step",
-                   "M": M, "K": K, "N": N, "r": r, "had_block": b, "layers_per_step": L,
-                   "l2": "inputs larger than L2" if L * per_layer > 126e6 else "L2-resident"},
-        "GB/s": round(world * L * per_layer / ms / 1e6, 1),
-        "us_per_layer": round(ms * 1e3 / L, 3),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(peak, 1),
-                     "unit": "TOPS", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic("rank_int4_gemm_b200/csrc/tq_gemm_a8.cu",
-                                                 "w4a4_lr_gemm_a8_sweep4096.md")
-                     if a8 and (M, K, N, r) == (4096, 4096, 4096, 64) else None,
-                     "kernel": "w4a4_lr_gemm_a8_kernel" if a8 else "w4a4_lr_gemm_kernel (prefill tiling)",
-                     "gemm_us": round(gemm_ms_avg * 1e3, 2), "peak_source": src,
-                     "act_us": round(act_ms_avg * 1e3, 2),
-                     "lowrank_flops_per_launch": 2 * M * r * (K + N)},
-        "gpu_launches": 2 * L * args.steps,
-        "path": ("tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte), the path "
-                 "tq_w4a4_lr_layer takes" if a8 else "tq_quantize_act + tq_w4a4_lr_gemm"),
-        "packed_code_path_us_per_layer": round(packed_ms * 1e3 / L, 3) if packed_ms else None,
-        "clocks": clk.summary(),
+        "workload": f"{sh.name}: M={M}, K={K}, N={N}, rank {r}, Hadamard block {b}",
+        "M": M, "K": K, "N": N, "r": r, "had_block": b, "layers_per_step": L,
+        "l2": "inputs larger than L2" if L * per_layer > 126e6 else "L2-resident",
+        "steps": steps, "warmup": warmup,
+        "us_per_layer": round(layer_us, 2), "act_us": round(act_us, 2),
+        "gemm_us": round(gemm_us, 2),
+        "TOPS": round(tops_layer, 1), "TOPS_gemm": round(tops_gemm, 1),
+        "roofline": {"bound": "tensor", "unit": "TOPS", "peak": round(peak, 1),
+                     "peak_source": src, "achieved": round(tops_layer, 1),
+                     "frac": round(tops_layer / peak, 4),
+                     "frac_gemm": round(tops_gemm / peak, 4),
+                     "frac_sustained_peak": round(tops_layer / peak_s, 4),
+                     "kernel": "w4a4_lr_gemm_a8_kernel" if a8 else
+                               "w4a4_lr_gemm_kernel (prefill tiling)",
+                     "lowrank_flops_per_layer": 2 * M * r * (K + N)},
+        "path": ("tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte)" if a8
+                 else "tq_quantize_act + tq_w4a4_lr_gemm"),
+        "clocks": c,
     }
+    if c.get("sm_mhz"):
+        out["kcycles_per_layer"] = round(layer_us * c["sm_mhz"] / 1e3, 1)
+    if packed_us is not None:
+        out["packed_code_path_us_per_layer"] = round(packed_us, 3)
+    return out, ops * L / (ms * 1e-3)
+
+
+def prefill_codes_sample(tq, torch, lay, sh, rows):
+    """The timed path's codes and scales of sampled tokens (host copies), for
+    the flip fraction against the oracle."""
+    b = sh.had_block
+    idx = torch.as_tensor(rows, device=lay["Xq8"].device)
+    return {"qx": lay["Xq8"][idx].cpu().numpy(), "s_x": lay["s_x"][idx].cpu().numpy(),
+            "Wq": lay["Wq"].cpu().numpy(), "s_w": lay["s_w"].cpu().numpy(), "b": b}
+
+
+def run_prefill(args, rank, world, local_rank, dist):
+    """One prefill shape per run (--workload): one layer call per distinct
+    layer per step; TOPS = 2 M N K per layer / layer time."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    sh = synth.CONFIGS[args.workload]
+    if args.rank is not None:
+        sh = sh.with_(r=args.rank)
+    M = args.m if args.m != 16 else sh.M
+    layers, per_layer = prefill_layers(tq, torch, sh, M, dev, rank, layers_cap=args.layers)
+    if args.profile:
+        a8 = tq.tq_layer_path(M, sh.N, sh.K, sh.r, sh.had_block) == "codes_i8"
+
+        def step():
+            for l in layers:
+                if a8:
+                    tq.tq_quantize_act_i8(l["X"], sh.had_block, l["L1t"], Xq8=l["Xq8"],
+                                          s_x=l["s_x"], XL1b=l["XL1b"])
+                    tq.tq_w4a4_lr_gemm_a8(l["Xq8"], l["s_x"], l["Wq"], l["s_w"], l["XL1b"],
+                                          l["L2t"], Y=l["Y"], workspace=l["ws"])
+                else:
+                    tq.tq_quantize_act(l["X"], sh.had_block, l["L1t"], Xq=l["Xq"],
+                                       s_x=l["s_x"], XL1=l["XL1"])
+                    tq.tq_w4a4_lr_gemm(l["Xq"], l["s_x"], l["Wq"], l["s_w"], l["XL1"],
+                                       l["L2t"], Y=l["Y"], workspace=l["ws"])
+        g = capture(torch, step)
+        time_graph(torch, g, args.steps, args.warmup)
+        return {"profile": f"{args.workload} step graph", "layers": len(layers),
+                "steps": args.steps, "warmup": args.warmup}
+    pt, ops_per_s = prefill_point(tq, torch, sh, M, layers, per_layer, args.steps, args.warmup,
+                                  rank, local_rank, dist, world, packed_too=True)
+    L = len(layers)
+    out = {
+        "metric": METRIC, "value": round(world * ops_per_s / 1e12, 2), "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(L * pt["us_per_layer"] / 1e3, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int4", "data": "synthetic",
+        "config": {"workload": pt["workload"] + f"; {L} distinct layer(s) per step",
+                   "M": M, "K": sh.K, "N": sh.N, "r": sh.r, "had_block": sh.had_block,
+                   "layers_per_step": L, "l2": pt["l2"]},
+        "GB/s": round(world * L * per_layer / (L * pt["us_per_layer"] * 1e-6) / 1e9, 1),
+        "gpu_launches": 2 * L * args.steps,
+    }
+    out.update({k: v for k, v in pt.items() if k not in ("workload", "l2")})
     return out
 
 
@@ -756,35 +887,145 @@ def run_qlr(args, rank, world, local_rank, dist):
 
 # ------------------------------------------------------------ oracle (CPU)
 
-def cpu_baseline(M, budget_s=12.0):
-    """The fp64 C oracle, as it stands, on a bounded sample of the workload:
-    repeated evaluations of one decode layer (rotation + codes + X L1,
-    integer GEMM, low-rank branch, epilogue; weights packed beforehand)."""
+CPU_SLICE = 64  # tokens of a prefill layer the oracle evaluates (time extrapolated)
+
+
+def _flips(gpu_q, orc_q, orc_t, rel=1e-6):
+    """Fraction of codes that differ from the oracle's, and how many of those
+    differ outside the midpoint allowance (a difference of exactly one where
+    the oracle's v/s lies within rel*|v/s| of the midpoint)."""
+    import numpy as np
+    g = np.asarray(gpu_q).astype(np.int32)
+    o = np.asarray(orc_q).astype(np.int32)
+    d = g - o
+    bad = d != 0
+    n = int(bad.sum())
+    if n == 0:
+        return 0.0, 0, int(g.size)
+    mid = (g[bad] + o[bad]) / 2.0
+    t = np.asarray(orc_t)[bad]
+    ok = (np.abs(d[bad]) == 1) & (np.abs(t - mid) <= rel * np.abs(t))
+    return n / g.size, int((~ok).sum()), int(g.size)
+
+
+def _one_layer(oracle, X, L1t, L2t, w, b):
+    """One evaluation of the layer by the oracle (weights packed beforehand);
+    returns the per-stage times and the activation codes."""
+    t0 = time.perf_counter()
+    a = oracle.quantize_act(X, b)
+    t1 = time.perf_counter()
+    acc = oracle.int_gemm(a["qx"], w["qw"])
+    t2 = time.perf_counter()
+    lr = None
+    if L1t is not None and L1t.shape[0] > 0:
+        _, lr = oracle.lowrank(X, L1t, L2t)
+    t3 = time.perf_counter()
+    oracle.epilogue(a["s_x"], w["s_w"], acc, lr)
+    t4 = time.perf_counter()
+    return {"rotate_quantize": t1 - t0, "int_gemm": t2 - t1, "lowrank": t3 - t2,
+            "epilogue": t4 - t3}, a
+
+
+def cpu_baseline(M, budget_s=12.0, decode=None, prefill=None):
+    """The fp64 C oracle, as it stands, on bounded samples of the workloads.
+
+    * decode: repeated evaluations of one decode layer (the bench's first
+      layer) on all host threads for about budget_s, with the time of each
+      stage (rotation + codes, integer GEMM, low-rank branch, epilogue);
+    * one thread: one evaluation of the tiny layer and of the decode layer;
+    * prefill: the first 64 tokens of each prefill layer (weights packed
+      beforehand, untimed); the layer time is extrapolated linearly in M.
+    Also returns the flip fractions of the timed path's codes against the
+    oracle's on those samples (the benchmark spec's reported fraction)."""
     import numpy as np
 
     import oracle
     import synth
 
-    sh = synth.CONFIGS["decode"].with_(M=M)
-    L = synth.make_layer(sh, seed=0)
-    w = oracle.pack_weight(L["Rt"], HAD)          # offline, untimed
-    X, L1t, L2t = L["X"], L["L1t"], L["L2t"]
-    n, t0 = 0, time.perf_counter()
+    threads = oracle.num_threads()
+    if decode is not None:
+        dec_in, dec_codes = decode
+        X, L1t, L2t, Rt = dec_in["X"], dec_in["L1t"], dec_in["L2t"], dec_in["Rt"]
+    else:
+        dec_codes = None
+        L = synth.make_layer(synth.CONFIGS["decode"].with_(M=M), seed=0)
+        X, L1t, L2t, Rt = L["X"], L["L1t"], L["L2t"], L["Rt"]
+    w = oracle.pack_weight(Rt, HAD)          # offline, untimed
+    n, t0, stages, a = 0, time.perf_counter(), None, None
     while True:
-        a = oracle.quantize_act(X, HAD)
-        acc = oracle.int_gemm(a["qx"], w["qw"])
-        _, lr = oracle.lowrank(X, L1t, L2t)
-        oracle.epilogue(a["s_x"], w["s_w"], acc, lr)
+        st, a = _one_layer(oracle, X, L1t, L2t, w, HAD)
+        stages = st if stages is None else {k: stages[k] + st[k] for k in st}
         n += 1
         if time.perf_counter() - t0 >= budget_s:
             break
     dt = (time.perf_counter() - t0) / n
     val = layer_bytes(M, K_DIM, N_DIM, RANK) / dt / 1e9
-    return {"value": round(val, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": f"{n} evaluations of one decode layer (M={M}, K=N=4096, r=32), "
-                      f"{dt:.2f} s each; weights packed outside the timing",
-            "s_per_layer": round(dt, 3)}
+    cb = {"value": round(val, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+          "sample": f"{n} evaluations of one decode layer (M={M}, K=N=4096, r=32), "
+                    f"{dt:.3f} s each on {threads} threads; weights packed outside the timing",
+          "s_per_layer": round(dt, 4),
+          "stages_s_per_layer": {k: round(v / n, 5) for k, v in stages.items()}}
+    parity = {"rule": "a code may differ by one only where the oracle's v/s lies within "
+                      "1e-6 relative of the rounding midpoint; outside = codes breaking it"}
+    if dec_codes is not None:
+        gq = oracle.unpack_int4(dec_codes["Xq"])
+        f, bad, cnt = _flips(gq, a["qx"], a["t_x"])
+        fw, badw, cntw = _flips(oracle.unpack_int4(dec_codes["Wq"]), w["qw"], w["t_w"])
+        parity["decode"] = {"activation_flip_fraction": f, "activation_codes": cnt,
+                            "outside_allowance": bad, "weight_flip_fraction": fw,
+                            "weight_codes": cntw, "weight_outside_allowance": badw,
+                            "source": dec_codes["source"]}
+
+    # one thread: the tiny layer and the decode layer
+    one = {}
+    oracle.set_num_threads(1)
+    try:
+        tl = synth.make_layer(synth.CONFIGS["tiny"], seed=0)
+        tw = oracle.pack_weight(tl["Rt"], 256)
+        reps, t0 = 0, time.perf_counter()
+        while reps < 3 or time.perf_counter() - t0 < 0.5:
+            _one_layer(oracle, tl["X"], tl["L1t"], tl["L2t"], tw, 256)
+            reps += 1
+        dtt = (time.perf_counter() - t0) / reps
+        one["tiny"] = {"s_per_layer": round(dtt, 6),
+                       "GB/s": round(layer_bytes(16, 256, 256, 16) / dtt / 1e9, 5)}
+        t0 = time.perf_counter()
+        st1, _ = _one_layer(oracle, X, L1t, L2t, w, HAD)
+        dt1 = time.perf_counter() - t0
+        one["decode"] = {"s_per_layer": round(dt1, 4),
+                         "GB/s": round(layer_bytes(M, K_DIM, N_DIM, RANK) / dt1 / 1e9, 5),
+                         "stages_s": {k: round(v, 5) for k, v in st1.items()}}
+    finally:
+        oracle.set_num_threads(threads)
+    cb["one_thread"] = one
+    del w
+
+    # prefill: the first CPU_SLICE tokens of each configuration, extrapolated
+    ext = {}
+    for name, (sh, cpu, codes) in (prefill or {}).items():
+        b = sh.had_block
+        w = oracle.pack_weight(cpu["Rt"], b)
+        Xs = cpu["X"][:CPU_SLICE]
+        t0 = time.perf_counter()
+        st, a = _one_layer(oracle, Xs, cpu["L1t"], cpu["L2t"], w, b)
+        ds = time.perf_counter() - t0
+        full = ds * sh.M / CPU_SLICE
+        ext[name] = {"tokens": CPU_SLICE, "s_slice": round(ds, 3),
+                     "s_layer_extrapolated": round(full, 2),
+                     "TOPS_extrapolated": round(2 * sh.M * sh.N * sh.K / full / 1e12, 6),
+                     "stages_s_slice": {k: round(v, 4) for k, v in st.items()},
+                     "label": "extrapolated"}
+        f, bad, cnt = _flips(codes["qx"], a["qx"], a["t_x"])
+        fw, badw, cntw = _flips(oracle.unpack_int4(codes["Wq"]), w["qw"], w["t_w"])
+        parity[name] = {"activation_flip_fraction": f, "activation_codes": cnt,
+                        "outside_allowance": bad, "weight_flip_fraction": fw,
+                        "weight_codes": cntw, "weight_outside_allowance": badw,
+                        "source": f"tq_quantize_act_i8 codes of the first {CPU_SLICE} tokens "
+                                  f"of the timed layer; all weight codes"}
+        del w, a
+    if ext:
+        cb["prefill_slices"] = ext
+    return cb, parity
 
 
 def run_reference(args):
