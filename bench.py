@@ -362,8 +362,8 @@ def run_tq(args, rank, world, local_rank, dist):
     # overlaps its predecessor's tail): average launch duration = step / L
     kernel_ms = ms / L
     achieved = gb / (kernel_ms * 1e-3) / 1e9
-    traffic = profiled_traffic("rank_int4_gemm_b200/csrc/tq_layer.cu",
-                               "w4a4_lr_layer_decode_m16.md") if M == 16 else None
+    traffic = profiled_traffic("rank_int4_gemm_b200/csrc/tq_decode.cu",
+                               "w4a4_lr_decode_m16.md") if M == 16 else None
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
@@ -385,7 +385,7 @@ def run_tq(args, rank, world, local_rank, dist):
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "w4a4_lr_layer_decode_kernel (whole layer, split-K cluster)",
+            "kernel": "w4a4_lr_decode_kernel (whole layer, split-K cluster of K/256 CTAs)",
             "kernel_us": round(kernel_ms * 1e3, 3),
             "kernel_us_isolated": round(gemm_ms_avg * 1e3, 3),
             "algorithmic_bytes_per_launch": gb, "peak_source": peak_src,

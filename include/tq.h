@@ -150,20 +150,28 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  *   Y = bf16( s_x s_w (Q4(X H) . Wq) + bf16(X L1) L2 )
  *
  * i.e. tq_quantize_act followed by tq_w4a4_lr_gemm, with the same codes,
- * scales and tolerances.  At decode sizes (M <= 16, r <= 32, K % 512 == 0,
- * K <= 4096, had_block <= 128) it runs as ONE kernel: each split-K cluster
- * rotates its own slice of X on the tensor cores, quantizes it, exchanges
- * the absmax and X L1 partials in distributed shared memory and feeds the
- * codes straight to the integer MMAs, while the weights stream in and are
- * expanded into tensor memory (TwinQuant notes section 04.C:
- * the residual GEMM quantizes activations concurrently and both paths share
- * one epilogue).  For M > 128 with had_block <= 128 it runs
+ * scales and tolerances.  At decode sizes (M <= 16, r in {0, 16, 32},
+ * K % 256 == 0, K <= 4096, had_block <= 256) it runs as ONE kernel
+ * (TwinQuant notes section 04.C: the residual GEMM quantizes activations
+ * concurrently and both paths share one epilogue): a thread-block cluster
+ * of K / 256 CTAs per group of output channels, each CTA rotating its
+ * 256-column slice of X with the same butterflies as tq_quantize_act (so
+ * the codes and scales are the same), exchanging the per-token absmax, the
+ * X L1 partials and the split-K sums in distributed shared memory, and
+ * feeding the codes to tcgen05 integer MMAs whose int4 weights were
+ * requested and expanded into tensor memory before the kernel waited on
+ * its predecessor.  Two such CTAs (two consecutive layers) share an SM.  For M > 128 with had_block <= 128 it runs
  * tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte in the
  * workspace).  Other shapes run tq_quantize_act + tq_w4a4_lr_gemm, keeping
  * Xq, s_x and XL1 in the workspace.
  *
  *   X [M][K] bf16, L1t [r][K] bf16 (NULL iff r == 0), Wq [N][K/2] u8,
  *   s_w [N] fp32, L2t [N][r] bf16 (NULL iff r == 0), Y [M][N] bf16 (out)
+ *   The weights (Wq, s_w, L1t, L2t) may be read before the kernel waits for
+ *   the work queued before it on `stream` (programmatic dependent launch):
+ *   they must not be written by the kernel launched immediately before
+ *   this call on the same stream, unless that kernel makes its stores
+ *   visible before it exits (the library's pack kernels do).
  *   workspace: >= tq_layer_workspace_bytes(M, N, K, r) bytes, zero-filled
  *   before first use (its first 4 bytes are the watchdog status word)
  */
@@ -218,6 +226,64 @@ TQ_API int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uin
                               const float* s_w2, const uint16_t* L2t2, int M, int N, int K,
                               int r2, int had_block, uint16_t* Y, void* workspace,
                               size_t workspace_bytes, void* stream);
+
+/*
+ * Shared input, any n <= 8 projections (Q, K and V of attention; CoQuant's
+ * note that layers sharing an input share one transform, Eq. (14)): the
+ * projections as ONE layer, so that one activation pass (rotation, codes,
+ * X L1 of the stacked ranks) and one GEMM serve them all.
+ *
+ * tq_pack_shared_input -- offline, copies only: projection i's operands
+ * (as tq_pack_weight makes them, rank r[i], N[i] channels; host arrays of n
+ * device pointers, L1t[i] / L2t[i] NULL iff r[i] == 0) concatenated:
+ *   Wq_cat  [sum N][K/2] u8   projection 0's rows, then 1's, ...
+ *   s_w_cat [sum N] fp32      likewise
+ *   L1t_cat [sum r][K] bf16   L1^T rows stacked along the rank
+ *   L2t_cat [sum N][sum r]    block-diagonal: rows of projection i hold its
+ *                             L2^T in columns [sum_{j<i} r[j], +r[i]), zeros
+ *                             elsewhere (exact zeros: they add nothing)
+ * L1t_cat and L2t_cat are NULL iff sum r == 0.  Limits: N[i] % 8 == 0,
+ * r[i] % 16 == 0, sum r <= 512.  Asynchronous on `stream`.
+ * Run the result through tq_w4a4_lr_layer (N = sum N, r = sum r): its Y
+ * [M][sum N] holds projection i's Y in columns [sum_{j<i} N[j], +N[i]),
+ * with the codes, integer sums and tolerances of that projection alone.
+ */
+TQ_API int tq_pack_shared_input(int n, const uint8_t* const* Wq, const float* const* s_w,
+                                const uint16_t* const* L1t, const uint16_t* const* L2t,
+                                const int* N, const int* r, int K, uint8_t* Wq_cat,
+                                float* s_w_cat, uint16_t* L1t_cat, uint16_t* L2t_cat,
+                                void* stream);
+
+/*
+ * Randomized Hadamard transform (the TORQUE page, randomized Hadamard
+ * abstract: random signs, then the Hadamard): the rotation U of CoQuant
+ * Eq. (3) becomes D H, with D = diag(d) a +-1 sign vector, on both sides:
+ * activations x -> x D H, weights R -> (D H)^T R (row n of R^T D H).  D H is
+ * orthogonal, so Eq. (3) still gives (x D H)((D H)^T W) = x W.  The signs are
+ * a device bit mask of K / 32 uint32 words: bit (k % 32) of word k / 32 set
+ * means d_k = -1.  X L1 reads the unrotated X and is unchanged.
+ *
+ * tq_pack_weight_rht   -- tq_pack_weight with D H.
+ * tq_quantize_act_rht  -- tq_quantize_act with D H: the butterfly kernel
+ *                         for every M (the sign flips are exact, in
+ *                         registers before the butterflies).
+ * tq_w4a4_lr_layer_rht -- tq_w4a4_lr_layer with D H (weights from
+ *                         tq_pack_weight_rht with the same mask): the
+ *                         one-kernel decode layer where it applies, else
+ *                         tq_quantize_act_rht + tq_w4a4_lr_gemm (packed
+ *                         codes; the tensor-core activation kernel of the
+ *                         int8-code path takes no signs).
+ * Arguments and limits as the plain calls; `signs` 16-byte aligned.
+ */
+TQ_API int tq_pack_weight_rht(const float* Rt, int N, int K, int had_block,
+                              const uint32_t* signs, uint8_t* Wq, float* s_w, void* stream);
+TQ_API int tq_quantize_act_rht(const uint16_t* X, int M, int K, int had_block,
+                               const uint32_t* signs, const uint16_t* L1t, int r, uint8_t* Xq,
+                               float* s_x, float* XL1, void* stream);
+TQ_API int tq_w4a4_lr_layer_rht(const uint16_t* X, const uint32_t* signs, const uint16_t* L1t,
+                                const uint8_t* Wq, const float* s_w, const uint16_t* L2t,
+                                int M, int N, int K, int r, int had_block, uint16_t* Y,
+                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Per-token asymmetric activations (CoQuant Eq. (1) with a zero-point; the
@@ -372,6 +438,22 @@ TQ_API int tq_w4a4_lr_gemm_noalloc(const uint8_t* Xq, const float* s_x,
                                    void* stream);
 TQ_API int tq_noalloc_query_status(void* stream);
 TQ_API int tq_debug_noalloc_set_status(int status);
+
+/*
+ * tq_debug_w4a4_lr_layer_decode -- test hook: the one-kernel decode layer of
+ * tq_w4a4_lr_layer (M <= 16, r in {0, 16, 32}, K % 256 == 0, K <= 4096,
+ * had_block <= 256), also writing what it computes on the way: the
+ * activation codes `codes` [M][K] int8 (RoundClip of X H per token), the
+ * scales `s_x` [M] fp32 and the integer sums `acc` [M][N] int32
+ * (sum_k codes[m][k] qw[n][k], exact).  Each of the three may be NULL.
+ * Shapes the kernel does not serve return TQ_ERR_UNSUPPORTED_SHAPE.
+ */
+TQ_API int tq_debug_w4a4_lr_layer_decode(const uint16_t* X, const uint16_t* L1t,
+                                         const uint8_t* Wq, const float* s_w,
+                                         const uint16_t* L2t, int M, int N, int K, int r,
+                                         int had_block, uint16_t* Y, int8_t* codes, float* s_x,
+                                         int32_t* acc, void* workspace, size_t workspace_bytes,
+                                         void* stream);
 
 /*
  * tq_debug_watchdog -- test hook for the bounded waits every pipelined

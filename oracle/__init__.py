@@ -7,5 +7,5 @@ does.  Every function follows the definition it cites in tq_oracle.c.
 from .oracle import (  # noqa: F401
     hadamard, rotate, quantize_sym, pack_int4, unpack_int4, int_gemm,
     round_bf16, lowrank, epilogue, quantize_act, pack_weight, layer,
-    num_threads, set_num_threads, swiglu, quantize_asym, layer_asym, layer_qlr,
+    num_threads, set_num_threads, swiglu, quantize_asym, layer_asym, layer_qlr, signs_from_bits,
 )

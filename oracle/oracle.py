@@ -62,9 +62,23 @@ def hadamard(b: int) -> np.ndarray:
     return np.array([[lib.orc_hadamard_entry(b, i, j) for j in range(b)] for i in range(b)])
 
 
-def rotate(x, b: int) -> np.ndarray:
-    """Rows of x times diag(H_b, ..., H_b) (fp64)."""
+def signs_from_bits(bits, K: int) -> np.ndarray:
+    """The sign vector d [K] (+1 / -1, fp64) of the randomized Hadamard
+    transform from its bit mask: K / 32 little-endian uint32 words, bit
+    (k % 32) of word k / 32 set where d_k = -1."""
+    w = np.ascontiguousarray(np.asarray(bits, dtype=np.uint32))
+    assert w.size * 32 >= K, (w.size, K)
+    neg = np.unpackbits(w.view(np.uint8), bitorder="little")[:K]
+    return np.where(neg == 1, -1.0, 1.0)
+
+
+def rotate(x, b: int, signs=None) -> np.ndarray:
+    """Rows of x times diag(H_b, ..., H_b) (fp64); with `signs` (the +-1
+    vector d), rows of x times D diag(H_b, ...): the randomized Hadamard
+    transform, signs first, then the Hadamard blocks."""
     x = _f64(x)
+    if signs is not None:
+        x = np.ascontiguousarray(x * np.asarray(signs, dtype=np.float64)[None, :])
     rows, K = x.shape
     assert K % b == 0
     out = np.empty_like(x)
@@ -150,10 +164,11 @@ def epilogue(s_x, s_w, acc, lr=None) -> np.ndarray:
     return Y
 
 
-def quantize_act(X, b: int, L1t=None) -> dict:
-    """Oracle of tq_quantize_act: rotation, per-token codes, scales, X L1."""
+def quantize_act(X, b: int, L1t=None, signs=None) -> dict:
+    """Oracle of tq_quantize_act: rotation (randomized with `signs`),
+    per-token codes, scales, X L1 (of the unrotated X)."""
     Xd = _f64(X)
-    q, s, t = quantize_sym(rotate(Xd, b))
+    q, s, t = quantize_sym(rotate(Xd, b, signs))
     out = {"qx": q, "s_x": s, "t_x": t, "Xq": pack_int4(q)}
     if L1t is not None and _f64(L1t).shape[0] > 0:
         L1d = _f64(L1t)
@@ -162,16 +177,19 @@ def quantize_act(X, b: int, L1t=None) -> dict:
     return out
 
 
-def pack_weight(Rt, b: int) -> dict:
-    """Oracle of tq_pack_weight: rotation of R^T rows, per-channel codes/scales."""
-    q, s, t = quantize_sym(rotate(_f64(Rt), b))
+def pack_weight(Rt, b: int, signs=None) -> dict:
+    """Oracle of tq_pack_weight: rotation of R^T rows (by D H with
+    `signs`: row n of R^T D H is column n of (D H)^T R), per-channel
+    codes / scales."""
+    q, s, t = quantize_sym(rotate(_f64(Rt), b, signs))
     return {"qw": q, "s_w": s, "t_w": t, "Wq": pack_int4(q)}
 
 
-def layer(X, L1t, L2t, Rt, b: int, round_mid: bool = True) -> dict:
-    """The whole layer: dequant(Q4(X H) Q4(H^T R)) + bf16(X L1) L2, in fp64."""
-    a = quantize_act(X, b)
-    w = pack_weight(Rt, b)
+def layer(X, L1t, L2t, Rt, b: int, round_mid: bool = True, signs=None) -> dict:
+    """The whole layer: dequant(Q4(X H) Q4(H^T R)) + bf16(X L1) L2, in fp64;
+    with `signs`, H is the randomized D H on both sides."""
+    a = quantize_act(X, b, signs=signs)
+    w = pack_weight(Rt, b, signs=signs)
     acc = int_gemm(a["qx"], w["qw"])
     XL1, lr = lowrank(X, L1t, L2t, round_mid=round_mid)
     Y64 = epilogue(a["s_x"], w["s_w"], acc, lr if _f64(L1t).shape[0] > 0 else None)

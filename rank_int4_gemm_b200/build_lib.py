@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_api.cu", "tq_act.cu", "tq_act_tc.cu", "tq_gemm.cu", "tq_gemm_a8.cu", "tq_layer.cu", "tq_noalloc.cu", "tq_qlr.cu", "tq_watchdog.cu"]
+SOURCES = ["tq_api.cu", "tq_act.cu", "tq_act_tc.cu", "tq_gemm.cu", "tq_gemm_a8.cu", "tq_decode.cu", "tq_noalloc.cu", "tq_qlr.cu", "tq_watchdog.cu"]
 HEADERS = ["tq_ptx.cuh", "tq_internal.h", "tq_act_common.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -38,6 +38,7 @@ struct ActParams {
   uint8_t* Xq;
   float* s_x;
   float* XL1;
+  const uint32_t* signs;  // randomized Hadamard sign mask [K / 32], or null
   int M, K, b, r;
   int passes_per_cta;  // P: warp passes of W = 32E columns in this CTA's slice
   int total_passes;    // K / W
@@ -161,6 +162,7 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
+      apply_signs<E>(v, p.signs, kbase + ps * W + lane * E);
       fwht_warp<E>(v, p.b);
 #pragma unroll
       for (int i = 0; i < E; ++i) amax[t] = fmaxf(amax[t], fabsf(v[i]));
@@ -281,6 +283,7 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
+      apply_signs<E>(v, p.signs, kbase + ps * W + lane * E);
       fwht_warp<E>(v, p.b);
       if (cs.pre != 1.f) {
 #pragma unroll
@@ -327,13 +330,21 @@ template <typename T, bool kBytes = false>
 __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __restrict__ Rt,
                                                                    int K, int b, float scale_mul,
                                                                    uint8_t* __restrict__ Wq,
-                                                                   float* __restrict__ s_w) {
+                                                                   float* __restrict__ s_w,
+                                                                   const uint32_t* signs) {
   extern __shared__ __align__(16) float row[];
   __shared__ float red[kPackThreads / 32];
   const int n = blockIdx.x;
   const T* src = Rt + (size_t)n * K;
-  for (int k = threadIdx.x * 4; k < K; k += kPackThreads * 4)
-    *reinterpret_cast<float4*>(row + k) = load4(src + k);
+  for (int k = threadIdx.x * 4; k < K; k += kPackThreads * 4) {
+    float4 f = load4(src + k);
+    if (signs) {  // randomized Hadamard: row n of R^T D H
+      float v[4] = {f.x, f.y, f.z, f.w};
+      apply_signs<4>(v, signs, k);
+      f = make_float4(v[0], v[1], v[2], v[3]);
+    }
+    *reinterpret_cast<float4*>(row + k) = f;
+  }
   __syncthreads();
   // in-place Sylvester butterflies, level by level (pairs never cross blocks)
   for (int h = 1; h < b; h <<= 1) {
@@ -362,6 +373,9 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __re
     int8_t* dst8 = reinterpret_cast<int8_t*>(Wq) + (size_t)n * K;
     for (int k = threadIdx.x; k < K; k += kPackThreads) dst8[k] = (int8_t)quant_code(row[k], inv);
     if (threadIdx.x == 0) s_w[n] = amax * scale_mul;
+    // the layer kernels read packed weights before they wait on the
+    // preceding kernel: make these stores visible before the block exits
+    __threadfence();
     return;
   }
   uint8_t* dst = Wq + (size_t)n * (K / 2);
@@ -372,6 +386,9 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __re
     dst[byte] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
   }
   if (threadIdx.x == 0) s_w[n] = amax * scale_mul;
+  // the layer kernels read packed weights before they wait on the preceding
+  // kernel: make these stores visible before the block exits
+  __threadfence();
 }
 
 template <int E>
@@ -514,7 +531,7 @@ __global__ void pack_gate_up_kernel(const uint8_t* __restrict__ Wq_g, const floa
 
 cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, const uint32_t* signs) {
   ActParams prm{};
   prm.X = reinterpret_cast<const __nv_bfloat16*>(X);
   prm.L1t = reinterpret_cast<const __nv_bfloat16*>(L1t);
@@ -526,8 +543,10 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   prm.b = had_block;
   prm.r = r;
   prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores.
-  if (act_tc_supported(M, K, had_block, r))
+  prm.signs = signs;
+  // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores
+  // (plain Hadamard only; sign masks take the butterfly kernel below).
+  if (!signs && act_tc_supported(M, K, had_block, r))
     return launch_act_tc(X, M, K, had_block, L1t, r, Xq, nullptr, s_x, XL1, nullptr, stream);
   // Few token groups (decode): spread K over up to 16 CTAs of 256 columns.
   const int groups = (M + kActRows - 1) / kActRows;
@@ -539,13 +558,14 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
 }
 
 cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
-                               float* s_w, cudaStream_t stream) {
+                               float* s_w, cudaStream_t stream, const uint32_t* signs) {
   const size_t smem = (size_t)K * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel<float>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  pack_weight_kernel<float><<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w);
+  pack_weight_kernel<float><<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w,
+                                                                signs);
   return cudaGetLastError();
 }
 
@@ -558,7 +578,8 @@ cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int
   if (e != cudaSuccess) return e;
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   pack<<<r, kPackThreads, smem, stream>>>(reinterpret_cast<const __nv_bfloat16*>(L1t), K, had_block,
-                                          scale_mul, reinterpret_cast<uint8_t*>(qL1), s_L1);
+                                          scale_mul, reinterpret_cast<uint8_t*>(qL1), s_L1,
+                                          nullptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lowrank_codes_kernel<<<(N + 7) / 8, 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(L2t), nullptr, nullptr, nullptr, N, r,

@@ -50,6 +50,18 @@ __device__ __forceinline__ void fwht_warp(float (&v)[E], int b) {
   }
 }
 
+// Randomized Hadamard transform: x D H with D = diag(d), d_k = -1 where
+// bit (k % 32) of word k / 32 of `signs` is set.  Negates (sign-bit flip,
+// exact) the E values of columns col0 .. col0 + E - 1 held by this thread
+// before the butterflies; col0 is a multiple of E and E divides 32.
+template <int E>
+__device__ __forceinline__ void apply_signs(float (&v)[E], const uint32_t* signs, int col0) {
+  if (!signs) return;
+  const uint32_t w = __ldg(signs + (col0 >> 5)) >> (col0 & 31);
+#pragma unroll
+  for (int i = 0; i < E; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((w >> i) & 1u) << 31));
+}
+
 // RoundClip(v * inv) with ties to even, for any v and inv (weights).
 __device__ __forceinline__ int quant_code(float v, float inv) {
   float t = rintf(v * inv);

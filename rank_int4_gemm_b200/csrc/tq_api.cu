@@ -216,7 +216,7 @@ int tq_layer_path(int M, int N, int K, int r, int had_block) {
   if (int s = check_k(K, had_block)) return -s;
   if (int s = check_r(r)) return -s;
   if (N < 8 || N % 8 != 0) return -TQ_ERR_UNSUPPORTED_SHAPE;
-  if (tq::layer_decode_supported(M, N, K, r, had_block)) return TQ_PATH_FUSED;
+  if (tq::layer_decode2_supported(M, N, K, r, had_block)) return TQ_PATH_FUSED;
   if (layer_uses_a8(M, r, had_block)) return TQ_PATH_CODES_I8;
   return TQ_PATH_CODES_PACKED;
 }
@@ -230,9 +230,10 @@ size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {
   return 256 + (M > 128 ? std::max(packed, bytes8) : packed);
 }
 
-int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
-                     const uint16_t* L2t, int M, int N, int K, int r, int had_block, uint16_t* Y,
-                     void* workspace, size_t workspace_bytes, void* stream) {
+static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* L1t,
+                      const uint8_t* Wq, const float* s_w, const uint16_t* L2t, int M, int N,
+                      int K, int r, int had_block, uint16_t* Y, void* workspace,
+                      size_t workspace_bytes, void* stream) {
   if (!X || !Wq || !s_w || !Y || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
   if (int s = check_k(K, had_block)) return s;
   if (int s = check_r(r)) return s;
@@ -246,8 +247,9 @@ int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, 
     return TQ_ERR_WORKSPACE;
   if (int s = check_device()) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (tq::layer_decode_supported(M, N, K, r, had_block)) {
+  if (tq::layer_decode2_supported(M, N, K, r, had_block)) {
     tq::LayerArgs a{};
+    a.signs = signs;
     a.X = X;
     a.L1t = L1t;
     a.Wq = Wq;
@@ -260,10 +262,10 @@ int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, 
     a.had_block = had_block;
     a.Y = Y;
     a.ws = workspace;
-    return from_cuda(tq::launch_layer_decode(a, st));
+    return from_cuda(tq::launch_layer_decode2(a, st));
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (layer_uses_a8(M, r, had_block)) {
+  if (!signs && layer_uses_a8(M, r, had_block)) {
     int8_t* Xq8 = reinterpret_cast<int8_t*>(ws + 256);
     float* s_x8 = reinterpret_cast<float*>(ws + 256 + align256((size_t)M * K));
     uint16_t* XL1b =
@@ -290,7 +292,7 @@ int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, 
   float* s_x = reinterpret_cast<float*>(Xq + align256((size_t)M * K / 2));
   float* XL1 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + align256((size_t)M * 4));
   if (cudaError_t e = tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x,
-                                              r > 0 ? XL1 : nullptr, st))
+                                              r > 0 ? XL1 : nullptr, st, signs))
     return from_cuda(e);
   tq::GemmArgs g{};
   g.Xq = Xq;
@@ -308,6 +310,85 @@ int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, 
   g.ws = workspace;
   g.ws_bytes = 256;
   return from_cuda(tq::launch_gemm(g, st));
+}
+
+int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
+                     const uint16_t* L2t, int M, int N, int K, int r, int had_block, uint16_t* Y,
+                     void* workspace, size_t workspace_bytes, void* stream) {
+  return layer_impl(X, nullptr, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
+                    workspace_bytes, stream);
+}
+
+// ------------------------------------------------ randomized Hadamard
+int tq_pack_weight_rht(const float* Rt, int N, int K, int had_block, const uint32_t* signs,
+                       uint8_t* Wq, float* s_w, void* stream) {
+  if (!Rt || !Wq || !s_w || !signs || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (!aligned16(Rt) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(signs))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_pack_weight(Rt, N, K, had_block, Wq, s_w,
+                                          static_cast<cudaStream_t>(stream), signs));
+}
+
+int tq_quantize_act_rht(const uint16_t* X, int M, int K, int had_block, const uint32_t* signs,
+                        const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
+                        void* stream) {
+  if (!X || !Xq || !s_x || !signs || M <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1 != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(s_x) || !aligned16(signs) ||
+      (r > 0 && !aligned16(L1t)) || (r > 0 && !aligned16(XL1)))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  return from_cuda(tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x, XL1,
+                                           static_cast<cudaStream_t>(stream), signs));
+}
+
+int tq_w4a4_lr_layer_rht(const uint16_t* X, const uint32_t* signs, const uint16_t* L1t,
+                         const uint8_t* Wq, const float* s_w, const uint16_t* L2t, int M, int N,
+                         int K, int r, int had_block, uint16_t* Y, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (!signs) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(signs)) return TQ_ERR_MISALIGNED;
+  return layer_impl(X, signs, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
+                    workspace_bytes, stream);
+}
+
+int tq_debug_w4a4_lr_layer_decode(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq,
+                                   const float* s_w, const uint16_t* L2t, int M, int N, int K,
+                                   int r, int had_block, uint16_t* Y, int8_t* codes, float* s_x,
+                                   int32_t* acc, void* workspace, size_t workspace_bytes,
+                                   void* stream) {
+  if (!X || !Wq || !s_w || !Y || M <= 0 || N <= 0) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, had_block)) return s;
+  if (int s = check_r(r)) return s;
+  if (N < 8 || N % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r > 0) != (L1t != nullptr) || (r > 0) != (L2t != nullptr)) return TQ_ERR_INVALID_VALUE;
+  if (!tq::layer_decode2_supported(M, N, K, r, had_block)) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(X) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(Y) ||
+      (L1t && !aligned16(L1t)) || (L2t && !aligned16(L2t)) || (codes && !aligned16(codes)) ||
+      (s_x && !aligned16(s_x)) || (acc && !aligned16(acc)) ||
+      (workspace && !aligned16(workspace)))
+    return TQ_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < 256) return TQ_ERR_WORKSPACE;
+  if (int s = check_device()) return s;
+  tq::LayerArgs a{};
+  a.X = X;
+  a.L1t = L1t;
+  a.Wq = Wq;
+  a.s_w = s_w;
+  a.L2t = L2t;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.r = r;
+  a.had_block = had_block;
+  a.Y = Y;
+  a.ws = workspace;
+  return from_cuda(
+      tq::launch_layer_decode2(a, static_cast<cudaStream_t>(stream), codes, s_x, acc));
 }
 
 int tq_query_device_status(void* workspace, void* stream) {
@@ -396,6 +477,62 @@ int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uint8_t* W
   a.ws = workspace;
   a.swiglu = 1;
   return from_cuda(tq::launch_gemm_a8(a, st));
+}
+
+// ------------------------------------------------------- shared input
+// Layers reading the same X (Q, K and V; any n <= 8) as one layer: their
+// rows concatenated, L1^T stacked along the rank, L2^T block-diagonal.  Only
+// copies (no arithmetic): the concatenated layer's Y [M][sum N] holds each
+// projection's Y as a column slice, from one activation pass and one GEMM.
+int tq_pack_shared_input(int n, const uint8_t* const* Wq, const float* const* s_w,
+                         const uint16_t* const* L1t, const uint16_t* const* L2t, const int* N,
+                         const int* r, int K, uint8_t* Wq_cat, float* s_w_cat, uint16_t* L1t_cat,
+                         uint16_t* L2t_cat, void* stream) {
+  if (n < 1 || n > 8 || !Wq || !s_w || !N || !r || !Wq_cat || !s_w_cat) return TQ_ERR_INVALID_VALUE;
+  if (int s = check_k(K, 1)) return s;
+  long long n_cat = 0, r_cat = 0;
+  for (int i = 0; i < n; ++i) {
+    if (!Wq[i] || !s_w[i]) return TQ_ERR_INVALID_VALUE;
+    if (N[i] < 8 || N[i] % 8 != 0) return TQ_ERR_UNSUPPORTED_SHAPE;
+    if (int s = check_r(r[i])) return s;
+    if (r[i] > 0 && (!L1t || !L2t || !L1t[i] || !L2t[i])) return TQ_ERR_INVALID_VALUE;
+    if (!aligned16(Wq[i]) || !aligned16(s_w[i]) ||
+        (r[i] > 0 && (!aligned16(L1t[i]) || !aligned16(L2t[i]))))
+      return TQ_ERR_MISALIGNED;
+    n_cat += N[i];
+    r_cat += r[i];
+  }
+  if (r_cat > 512 || n_cat > (1ll << 30)) return TQ_ERR_UNSUPPORTED_SHAPE;
+  if ((r_cat > 0) != (L1t_cat != nullptr) || (r_cat > 0) != (L2t_cat != nullptr))
+    return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(Wq_cat) || !aligned16(s_w_cat) || (L1t_cat && !aligned16(L1t_cat)) ||
+      (L2t_cat && !aligned16(L2t_cat)))
+    return TQ_ERR_MISALIGNED;
+  if (int s = check_device()) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t row_bytes = (size_t)K / 2;
+  if (r_cat > 0 &&
+      cudaMemsetAsync(L2t_cat, 0, (size_t)n_cat * (size_t)r_cat * 2, st) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  size_t off_n = 0, off_r = 0;
+  for (int i = 0; i < n; ++i) {
+    if (cudaMemcpyAsync(Wq_cat + off_n * row_bytes, Wq[i], (size_t)N[i] * row_bytes,
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(s_w_cat + off_n, s_w[i], (size_t)N[i] * 4, cudaMemcpyDeviceToDevice,
+                        st) != cudaSuccess)
+      return TQ_ERR_CUDA;
+    if (r[i] > 0) {
+      if (cudaMemcpyAsync(L1t_cat + off_r * (size_t)K, L1t[i], (size_t)r[i] * K * 2,
+                          cudaMemcpyDeviceToDevice, st) != cudaSuccess ||
+          cudaMemcpy2DAsync(L2t_cat + off_n * (size_t)r_cat + off_r, (size_t)r_cat * 2, L2t[i],
+                            (size_t)r[i] * 2, (size_t)r[i] * 2, (size_t)N[i],
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return TQ_ERR_CUDA;
+    }
+    off_n += (size_t)N[i];
+    off_r += (size_t)r[i];
+  }
+  return TQ_OK;
 }
 
 // ------------------------------------------------ asymmetric activations

@@ -15,12 +15,14 @@ struct Tuning {
 };
 Tuning& tuning();
 
+// `signs`: the randomized Hadamard's sign mask [K / 32] (rotation by D H),
+// or null for the plain Hadamard.
 cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
-                               float* s_w, cudaStream_t stream);
+                               float* s_w, cudaStream_t stream, const uint32_t* signs = nullptr);
 
 cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
-                                float* XL1, cudaStream_t stream);
+                                float* XL1, cudaStream_t stream, const uint32_t* signs = nullptr);
 
 // Activation stage on tensor cores (many tokens): rotation and X L1 as MMAs.
 // Codes packed (Xq, [M][K/2]) or one int8 per code (Xq8, [M][K]); X L1 as
@@ -95,6 +97,7 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream);
 
 // The whole layer from bf16 X (decode sizes: one fused kernel).
 struct LayerArgs {
+  const uint32_t* signs = nullptr;  // randomized Hadamard sign mask [K / 32], or null
   const uint16_t* X;
   const uint16_t* L1t;
   const uint8_t* Wq;
@@ -104,8 +107,13 @@ struct LayerArgs {
   uint16_t* Y;
   void* ws;  // status word at offset 0
 };
-bool layer_decode_supported(int M, int N, int K, int r, int had_block);
-cudaError_t launch_layer_decode(const LayerArgs& a, cudaStream_t stream);
+// The decode layer sized for two CTAs per SM (clusters of K / 256 CTAs).
+// Optional debug outputs: the activation codes [M][K] int8, the scales [M]
+// and the integer sums [M][N] (sum_k qx qw) of the same launch.
+bool layer_decode2_supported(int M, int N, int K, int r, int had_block);
+cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream,
+                                 int8_t* dbg_codes = nullptr, float* dbg_sx = nullptr,
+                                 int32_t* dbg_acc = nullptr);
 
 // Shared host helpers (defined in tq_gemm.cu).
 int num_sms();

@@ -40,6 +40,18 @@ _lib.tq_debug_w4a4_gemm_acc.restype = _I
 _lib.tq_debug_w4a4_gemm_acc.argtypes = [_P, _P, _I, _I, _I, _P, _P, ctypes.c_size_t, _P]
 _lib.tq_w4a4_lr_gemm_noalloc.restype = _I
 _lib.tq_w4a4_lr_gemm_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.tq_pack_weight_rht.restype = _I
+_lib.tq_pack_weight_rht.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
+_lib.tq_quantize_act_rht.restype = _I
+_lib.tq_quantize_act_rht.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]
+_lib.tq_w4a4_lr_layer_rht.restype = _I
+_lib.tq_w4a4_lr_layer_rht.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                                      ctypes.c_size_t, _P]
+_lib.tq_pack_shared_input.restype = _I
+_lib.tq_pack_shared_input.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
+_lib.tq_debug_w4a4_lr_layer_decode.restype = _I
+_lib.tq_debug_w4a4_lr_layer_decode.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                                               _P, _P, _P, ctypes.c_size_t, _P]
 _lib.tq_debug_watchdog.restype = _I
 _lib.tq_debug_watchdog.argtypes = [_P, ctypes.c_size_t, _I, ctypes.c_longlong, _P, _P]
 _lib.tq_noalloc_query_status.restype = _I
@@ -364,6 +376,57 @@ def tq_w4a4_lr_gemm_noalloc(Xq, s_x, Wq, s_w, XL1=None, L2t=None, Y=None, stream
     return Y
 
 
+def tq_pack_shared_input(projections, stream=None):
+    """Projections reading the same X, each (Wq, s_w, L1t, L2t) as
+    tq_pack_weight makes them (L1t / L2t None for rank 0), packed as one
+    layer: returns (Wq_cat, s_w_cat, L1t_cat, L2t_cat, N_list).  Run it with
+    tq_w4a4_lr_layer; split_shared_output gives each projection's Y."""
+    n = len(projections)
+    Ns = [int(p[0].shape[0]) for p in projections]
+    K = 2 * int(projections[0][0].shape[1])
+    rs = [0 if p[2] is None else int(p[2].shape[0]) for p in projections]
+    dev = projections[0][0].device
+    n_cat, r_cat = sum(Ns), sum(rs)
+    Wq_cat = torch.empty(n_cat, K // 2, dtype=torch.uint8, device=dev)
+    s_w_cat = torch.empty(n_cat, dtype=torch.float32, device=dev)
+    L1t_cat = torch.empty(r_cat, K, dtype=torch.bfloat16, device=dev) if r_cat else None
+    L2t_cat = torch.empty(n_cat, r_cat, dtype=torch.bfloat16, device=dev) if r_cat else None
+    arr = lambda ts: (ctypes.c_void_p * n)(*[None if t is None else t.data_ptr() for t in ts])  # noqa: E731
+    _check(_lib.tq_pack_shared_input(
+        n, arr([p[0] for p in projections]), arr([p[1] for p in projections]),
+        arr([p[2] for p in projections]), arr([p[3] for p in projections]),
+        (ctypes.c_int * n)(*Ns), (ctypes.c_int * n)(*rs), K, _ptr(Wq_cat), _ptr(s_w_cat),
+        _ptr(L1t_cat), _ptr(L2t_cat), _stream(stream)), "tq_pack_shared_input")
+    return Wq_cat, s_w_cat, L1t_cat, L2t_cat, Ns
+
+
+def split_shared_output(Y, Ns):
+    """Views of the concatenated layer's Y [M][sum N], one per projection."""
+    return list(torch.split(Y, list(Ns), dim=1))
+
+
+def tq_debug_w4a4_lr_layer_decode(X, L1t, Wq, s_w, L2t, had_block, workspace=None, stream=None):
+    """The one-kernel decode layer with its debug outputs: returns
+    (Y [M][N] bf16, codes [M][K] int8, s_x [M] fp32, acc [M][N] int32)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    r = 0 if L1t is None else L1t.shape[0]
+    dev = X.device
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    codes = torch.empty(M, K, dtype=torch.int8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    acc = torch.empty(M, N, dtype=torch.int32, device=dev)
+    if workspace is None:
+        workspace = Workspace(dev)
+    ws = workspace.get(256) if isinstance(workspace, Workspace) else workspace
+    _check(_lib.tq_debug_w4a4_lr_layer_decode(_ptr(X), _ptr(L1t), _ptr(Wq), _ptr(s_w), _ptr(L2t),
+                                              M, N, K, r, int(had_block), _ptr(Y), _ptr(codes),
+                                              _ptr(s_x), _ptr(acc), _ptr(ws), ws.numel(),
+                                              _stream(stream)),
+           "tq_debug_w4a4_lr_layer_decode")
+    return Y, codes, s_x, acc
+
+
 def tq_debug_watchdog(workspace, withhold: bool, budget_cycles: int, waited_ok=None,
                       stream=None):
     """Test hook of the bounded waits: one CTA whose consumer waits (at most
@@ -439,6 +502,60 @@ def tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None, st
     _check(_lib.tq_w4a4_lr_layer(_ptr(X), _ptr(L1t) if r else None, _ptr(Wq), _ptr(s_w),
                                  _ptr(L2t) if r else None, M, N, K, r, int(had_block), _ptr(Y),
                                  _ptr(ws), ws.numel(), _stream(stream)), "tq_w4a4_lr_layer")
+    return Y
+
+
+def _signs(signs, K):
+    _need(signs, torch.int32, (K // 32,), "signs")
+    return _ptr(signs)
+
+
+def tq_pack_weight_rht(Rt: torch.Tensor, had_block: int, signs: torch.Tensor, Wq=None, s_w=None,
+                       stream=None):
+    """tq_pack_weight with the randomized Hadamard D H: `signs` is the bit
+    mask [K/32] (int32 words; bit k % 32 of word k / 32 set where d_k = -1)."""
+    N, K = Rt.shape
+    _need(Rt, torch.float32, (N, K), "Rt")
+    Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=Rt.device) if Wq is None else Wq
+    s_w = torch.empty(N, dtype=torch.float32, device=Rt.device) if s_w is None else s_w
+    _check(_lib.tq_pack_weight_rht(_ptr(Rt), N, K, int(had_block), _signs(signs, K), _ptr(Wq),
+                                   _ptr(s_w), _stream(stream)), "tq_pack_weight_rht")
+    return Wq, s_w
+
+
+def tq_quantize_act_rht(X: torch.Tensor, had_block: int, signs: torch.Tensor, L1t=None,
+                        stream=None):
+    """tq_quantize_act with the randomized Hadamard: codes of X D H."""
+    M, K = X.shape
+    _need(X, torch.bfloat16, (M, K), "X")
+    r = 0 if L1t is None else L1t.shape[0]
+    dev = X.device
+    Xq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    XL1 = torch.empty(M, r, dtype=torch.float32, device=dev) if r else None
+    _check(_lib.tq_quantize_act_rht(_ptr(X), M, K, int(had_block), _signs(signs, K),
+                                    _ptr(L1t) if r else None, r, _ptr(Xq), _ptr(s_x),
+                                    _ptr(XL1) if r else None, _stream(stream)),
+           "tq_quantize_act_rht")
+    return Xq, s_x, XL1
+
+
+def tq_w4a4_lr_layer_rht(X, signs, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None,
+                         stream=None):
+    """tq_w4a4_lr_layer with the randomized Hadamard on both sides (weights
+    from tq_pack_weight_rht with the same signs)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    r = 0 if L1t is None else L1t.shape[0]
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=X.device) if Y is None else Y
+    if workspace is None:
+        workspace = Workspace(X.device)
+    ws = workspace.get(tq_layer_workspace_bytes(M, N, K, r)) if isinstance(workspace, Workspace) \
+        else workspace
+    _check(_lib.tq_w4a4_lr_layer_rht(_ptr(X), _signs(signs, K), _ptr(L1t) if r else None,
+                                     _ptr(Wq), _ptr(s_w), _ptr(L2t) if r else None, M, N, K, r,
+                                     int(had_block), _ptr(Y), _ptr(ws), ws.numel(),
+                                     _stream(stream)), "tq_w4a4_lr_layer_rht")
     return Y
 
 

@@ -69,14 +69,20 @@ def check_y(gpu_y, y64, what="Y"):
     return fro, mx
 
 
-def y_reference(gpu_codes, o, flips):
+def y_reference(gpu_codes, o, flips, gpu_wcodes=None, wflips=0):
     """The reference for Y: the oracle's fp64 Y64 when the GPU's codes equal
-    the oracle's (flips == 0), else the oracle's epilogue on the GPU's codes.
-    The second case is only reached after check_codes has shown that every
-    difference is an allowed midpoint flip: one flip moves a token's whole
-    row of Y by s_x s_w q_w, which the output tolerance is not meant to
-    absorb (it can reach 2e-3 relative Frobenius alone)."""
-    return o["Y64"] if flips == 0 else y_given_codes(gpu_codes, o)
+    the oracle's (flips == wflips == 0), else the oracle's epilogue on the
+    GPU's activation codes (if they hold flips) and weight codes (if those
+    do).  The second case is only reached after check_codes has shown that
+    every difference is an allowed midpoint flip: one flip moves a token's
+    whole row (or a channel's whole column) of Y by s_x s_w q, which the
+    output tolerance is not meant to absorb (it can reach 2e-3 relative
+    Frobenius alone)."""
+    if flips == 0 and wflips == 0:
+        return o["Y64"]
+    qa = np.asarray(gpu_codes).astype(np.int8) if flips else o["qx"]
+    qw = np.asarray(gpu_wcodes).astype(np.int8) if wflips else o["qw"]
+    return oracle.epilogue(o["s_x"], o["s_w"], oracle.int_gemm(qa, qw), o["lr"])
 
 
 def y_given_codes(gpu_codes, o):

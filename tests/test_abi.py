@@ -108,8 +108,8 @@ def test_no_device_is_reported(lib):
 
 def test_layer_path_routing():
     """tq_layer_path is a host query (runs without a GPU): the one-kernel
-    decode layer where its limits hold (M <= 16, r <= 32, K % 512 == 0,
-    K <= 4096, Hadamard block <= 128), int8 codes for M > 128 with block
+    decode layer where its limits hold (M <= 16, r <= 32, K % 256 == 0,
+    K <= 4096, Hadamard block <= 256), int8 codes for M > 128 with block
     <= 128, packed codes otherwise; rejected shapes raise."""
     import rank_int4_gemm_b200 as tq
     p = tq.tq_layer_path
@@ -120,8 +120,9 @@ def test_layer_path_routing():
     assert p(16, 4096, 4096, 64, 128) == "codes_packed"
     assert p(16, 8192, 4096, 32, 128) == "fused"        # N does not limit it
     assert p(16, 4096, 4608, 32, 128) == "codes_packed"  # K > 4096
-    assert p(16, 4096, 384, 16, 128) == "codes_packed"   # K % 512 != 0
-    assert p(16, 4096, 4096, 32, 256) == "codes_packed"  # block > 128
+    assert p(16, 4096, 384, 16, 128) == "codes_packed"   # K % 256 != 0
+    assert p(16, 4096, 768, 16, 128) == "fused"          # a cluster of 3 CTAs
+    assert p(16, 4096, 4096, 32, 256) == "fused"
     assert p(128, 4096, 4096, 64, 128) == "codes_packed"
     assert p(129, 4096, 4096, 64, 128) == "codes_i8"
     assert p(4096, 4096, 4096, 128, 128) == "codes_i8"
