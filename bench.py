@@ -198,6 +198,11 @@ def build_layers(tq, torch, M, L, seed0, device):
                                dtype=torch.uint8, device=device),
         }
         layers.append(lay)
+    # a stack of layers as in a decode step: layer i reads layer i-1's output
+    # (K = N), so every layer waits for its predecessor and finds its input in
+    # L2, as a model's next layer does; layer 0 reads the synthetic X
+    for prev, lay in zip(layers, layers[1:]):
+        lay["X"] = prev["Y"]
     torch.cuda.synchronize()
     return layers
 
@@ -316,15 +321,16 @@ def run_tq(args, rank, world, local_rank, dist):
         gemm_ms.extend(a.elapsed_time(b) for a, b in evs)
     gemm_ms_avg = sum(gemm_ms) / len(gemm_ms)
 
-    # end to end: pinned host X in, host Y out, every step
-    hx = [lay["X"].cpu().pin_memory() for lay in layers]
-    hy = [torch.empty_like(lay["Y"], device="cpu").pin_memory() for lay in layers]
+    # end to end: the step's input (layer 0's X) from pinned host memory in,
+    # its result (the last layer's Y) to pinned host memory out, every step
+    hx = [layers[0]["X"].cpu().pin_memory()]
+    hy = [torch.empty_like(layers[-1]["Y"], device="cpu").pin_memory()]
 
     def step_e2e():
-        for lay, x, y in zip(layers, hx, hy):
-            lay["X"].copy_(x, non_blocking=True)
+        layers[0]["X"].copy_(hx[0], non_blocking=True)
+        for lay in layers:
             layer_call(tq, lay)
-            y.copy_(lay["Y"], non_blocking=True)
+        hy[0].copy_(layers[-1]["Y"], non_blocking=True)
 
     g_e2e = capture(torch, step_e2e)
     ms_e2e = time_graph(torch, g_e2e, args.steps, args.warmup, dist if world > 1 else None)
@@ -372,9 +378,12 @@ def run_tq(args, rank, world, local_rank, dist):
                 "W = U diag(i^-1/2) V^T at std 0.02, random-init, no checkpoint)",
         "config": {
             "workload": f"Llama-3-8B attention projection, decode: M={M} tokens, K=N=4096, "
-                        f"rank {RANK}, Hadamard block {HAD}; {L} distinct layers per step",
+                        f"rank {RANK}, Hadamard block {HAD}; a stack of {L} distinct layers per "
+                        f"step, each reading the previous one's output",
             "M": M, "K": K_DIM, "N": N_DIM, "r": RANK, "had_block": HAD,
             "layers_per_step": L,
+            "chain": "layer i reads layer i-1's output (a decode step through a stack of "
+                     "layers); layer 0 reads the synthetic X",
             "l2": f"inputs larger than L2: {L} layers x {gb / 1e6:.1f} MB of GEMM operands",
             "parallelism": f"{world} independent replica(s), no data-path collective",
             "graph": "one CUDA graph per step; one tq_w4a4_lr_layer launch per layer "
@@ -458,14 +467,16 @@ def decode_cpu_inputs(lay):
 
 
 def decode_codes_sample(tq, torch, lay):
-    """Codes and scales of the decode layer's tokens as the timed path makes
-    them, and its weight codes (host copies), for the flip fraction."""
-    Xq, s_x, _ = tq.tq_quantize_act(lay["X"], HAD, lay["L1t"])
+    """Codes and scales of the decode layer's tokens as the timed kernel
+    makes them (its debug hook: the same kernel, also storing its codes), and
+    its weight codes (host copies), for the flip fraction."""
+    _, q, s_x, _ = tq.tq_debug_w4a4_lr_layer_decode(lay["X"], lay["L1t"], lay["Wq"], lay["s_w"],
+                                                     lay["L2t"], HAD)
     torch.cuda.synchronize()
-    return {"Xq": Xq.cpu().numpy(), "s_x": s_x.cpu().numpy(), "Wq": lay["Wq"].cpu().numpy(),
+    return {"q": q.cpu().numpy(), "s_x": s_x.cpu().numpy(), "Wq": lay["Wq"].cpu().numpy(),
             "s_w": lay["s_w"].cpu().numpy(), "b": HAD,
-            "source": "tq_quantize_act on the bench's first decode layer (the fused kernel "
-                      "computes the same codes internally and does not store them)"}
+            "source": "the timed decode kernel's own codes (tq_debug_w4a4_lr_layer_decode) on "
+                      "the bench's first layer; all weight codes"}
 
 
 # --------------------------------------------------------------- prefill arm
@@ -502,6 +513,11 @@ def prefill_layers(tq, torch, sh, M, dev, rank, layers_cap=16, keep_cpu=False):
             lay["cpu"] = {"X": X, "Rt": w["Rt"], "L1t": w["L1t"], "L2t": w["L2t"]}
         del w
         layers.append(lay)
+    # a stack of layers as in a decode step: layer i reads layer i-1's output
+    # (K = N), so every layer waits for its predecessor and finds its input in
+    # L2, as a model's next layer does; layer 0 reads the synthetic X
+    for prev, lay in zip(layers, layers[1:]):
+        lay["X"] = prev["Y"]
     torch.cuda.synchronize()
     return layers, per_layer
 
@@ -968,8 +984,7 @@ def cpu_baseline(M, budget_s=12.0, decode=None, prefill=None):
     parity = {"rule": "a code may differ by one only where the oracle's v/s lies within "
                       "1e-6 relative of the rounding midpoint; outside = codes breaking it"}
     if dec_codes is not None:
-        gq = oracle.unpack_int4(dec_codes["Xq"])
-        f, bad, cnt = _flips(gq, a["qx"], a["t_x"])
+        f, bad, cnt = _flips(dec_codes["q"], a["qx"], a["t_x"])
         fw, badw, cntw = _flips(oracle.unpack_int4(dec_codes["Wq"]), w["qw"], w["t_w"])
         parity["decode"] = {"activation_flip_fraction": f, "activation_codes": cnt,
                             "outside_allowance": bad, "weight_flip_fraction": fw,
