@@ -66,7 +66,7 @@ def parse():
                     help="replay only the timed step graph (for a profiler); prints one status line")
     ap.add_argument("--workload", default="decode",
                     choices=["decode", "prefill_gateup", "prefill_down", "large_gateup",
-                             "large_down", "sweep", "sweeps", "gateup_swiglu", "qlr"],
+                             "large_down", "sweep", "sweeps", "gateup_swiglu", "qlr", "qkv", "rht"],
                     help="decode is the default workload; the others are the prefill "
                          "shapes, scored in TOPS against the dense INT8 peak")
     ap.add_argument("--rank", type=int, default=None, help="low-rank r override (sweep)")
@@ -328,8 +328,7 @@ def run_tq(args, rank, world, local_rank, dist):
 
     def step_e2e():
         layers[0]["X"].copy_(hx[0], non_blocking=True)
-        for lay in layers:
-            layer_call(tq, lay)
+        step()
         hy[0].copy_(layers[-1]["Y"], non_blocking=True)
 
     g_e2e = capture(torch, step_e2e)
@@ -901,6 +900,135 @@ def run_qlr(args, rank, world, local_rank, dist):
     }
 
 
+def _time_pair(torch, f1, f2, steps, warm, local_rank):
+    g1, g2 = capture(torch, f1), capture(torch, f2)
+    with ClockSampler(local_rank) as clk:
+        ms1 = time_graph(torch, g1, steps, warm)
+    ms2 = time_graph(torch, g2, steps, warm)
+    del g1, g2
+    return ms1, ms2, clk.summary()
+
+
+def run_qkv(args, rank, world, local_rank, dist):
+    """Llama-3-8B attention's Q, K and V projections (K = 4096; N = 4096,
+    1024, 1024 under grouped-query attention; rank 32 each) packed as one
+    shared-input layer (tq_pack_shared_input, one activation pass and one
+    GEMM) against the three projections as separate tq_w4a4_lr_layer calls,
+    at decode (M = 16, a stack of layers) and prefill (M = 2048)."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    K, Ns, r, b = 4096, (4096, 1024, 1024), 32, 128
+    steps, warm = max(5, min(args.steps, 50)), max(3, args.warmup)
+    out = {"metric": METRIC, "unit": "TOPS", "n_gpus": world, "steps": steps, "warmup": warm,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+           "data": "synthetic", "config": {"workload": "Llama-3-8B attention QKV: K=4096, N = "
+                                                       "4096 + 1024 + 1024, rank 32 each, block 128"}}
+    for M, L in ((16, 16), (2048, 3)):
+        lays = []
+        for i in range(L):
+            projs = []
+            for j, N in enumerate(Ns):
+                sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=r)
+                w = synth.make_weights(sh, seed=replica_seed(rank) + 10 * i + j, device="cuda")
+                Wq, s_w = tq.tq_pack_weight(w["Rt"].to(dev), b)
+                projs.append((Wq, s_w, w["L1t"].to(dev), w["L2t"].to(dev)))
+            Wc, sc, L1c, L2c, _ = tq.tq_pack_shared_input(projs)
+            X = synth.make_activations(synth.CONFIGS["decode"].with_(M=M), seed=i, M=M).to(dev)
+            lays.append({"X": X, "p": projs, "c": (Wc, sc, L1c, L2c),
+                         "Y": torch.empty(M, sum(Ns), dtype=torch.bfloat16, device=dev),
+                         "Ys": [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for N in Ns],
+                         "ws": tq.Workspace(dev), "wss": [tq.Workspace(dev) for _ in Ns]})
+        torch.cuda.synchronize()
+
+        def packed():
+            for l in lays:
+                Wc, sc, L1c, L2c = l["c"]
+                tq.tq_w4a4_lr_layer(l["X"], L1c, Wc, sc, L2c, b, Y=l["Y"], workspace=l["ws"])
+
+        def separate():
+            for l in lays:
+                for (Wq, s_w, L1t, L2t), Y, w in zip(l["p"], l["Ys"], l["wss"]):
+                    tq.tq_w4a4_lr_layer(l["X"], L1t, Wq, s_w, L2t, b, Y=Y, workspace=w)
+
+        ms1, ms2, clk = _time_pair(torch, packed, separate, steps, warm, local_rank)
+        ops = 2 * M * sum(Ns) * K
+        out[f"M={M}"] = {"us_packed": round(ms1 * 1e3 / L, 3), "us_separate": round(ms2 * 1e3 / L, 3),
+                         "TOPS_packed": round(ops / (ms1 * 1e-3 / L) / 1e12, 2),
+                         "path_packed": tq.tq_layer_path(M, sum(Ns), K, 3 * r, b),
+                         "path_separate": [tq.tq_layer_path(M, N, K, r, b) for N in Ns],
+                         "clocks": clk}
+        del lays
+        torch.cuda.empty_cache()
+    out["value"] = out["M=2048"]["TOPS_packed"]
+    out["gpu_launches"] = None
+    return out
+
+
+def run_rht(args, rank, world, local_rank, dist):
+    """The layer with the randomized Hadamard (a sign mask before the
+    Hadamard blocks) against the plain layer: the decode projection (M = 16,
+    a stack of 16 layers, the one-kernel path) and the Llama-3-8B gate/up
+    prefill shape (M = 2048: butterfly activation kernel + packed-code GEMM
+    with signs, the int8-code path without)."""
+    import torch
+
+    import rank_int4_gemm_b200 as tq
+    import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    steps, warm = max(5, min(args.steps, 50)), max(3, args.warmup)
+    out = {"metric": METRIC, "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": warm,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int4",
+           "data": "synthetic", "config": {"workload": "randomized Hadamard against the plain "
+                                                       "Hadamard, decode and prefill shapes"}}
+    for name, L in (("decode", 16), ("prefill_gateup", 2)):
+        sh = synth.CONFIGS[name]
+        M, K, N, r, b = sh.M, sh.K, sh.N, sh.r, sh.had_block
+        gen = torch.Generator().manual_seed(77)
+        signs = torch.randint(-2 ** 31, 2 ** 31 - 1, (K // 32,), generator=gen,
+                              dtype=torch.int64).to(torch.int32).to(dev)
+        lays = []
+        for i in range(L):
+            w = synth.make_weights(sh, seed=replica_seed(rank) + 10 * i, device="cuda")
+            Rt = w["Rt"].to(dev)
+            lays.append({"X": synth.make_activations(sh, seed=i).to(dev), "L1t": w["L1t"].to(dev),
+                         "L2t": w["L2t"].to(dev), "plain": tq.tq_pack_weight(Rt, b),
+                         "rht": tq.tq_pack_weight_rht(Rt, b, signs),
+                         "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+                         "ws": tq.Workspace(dev)})
+            del Rt
+        torch.cuda.synchronize()
+
+        def plain():
+            for l in lays:
+                tq.tq_w4a4_lr_layer(l["X"], l["L1t"], *l["plain"], l["L2t"], b, Y=l["Y"],
+                                    workspace=l["ws"])
+
+        def signed():
+            for l in lays:
+                tq.tq_w4a4_lr_layer_rht(l["X"], signs, l["L1t"], *l["rht"], l["L2t"], b, Y=l["Y"],
+                                        workspace=l["ws"])
+
+        ms_s, ms_p, clk = _time_pair(torch, signed, plain, steps, warm, local_rank)
+        byt = layer_bytes(M, K, N, r)
+        out[name] = {"M": M, "K": K, "N": N, "r": r, "us_signed": round(ms_s * 1e3 / L, 3),
+                     "us_plain": round(ms_p * 1e3 / L, 3),
+                     "GB/s_signed": round(byt / (ms_s * 1e-3 / L) / 1e9, 1),
+                     "TOPS_signed": round(2 * M * N * K / (ms_s * 1e-3 / L) / 1e12, 2),
+                     "clocks": clk}
+        del lays
+        torch.cuda.empty_cache()
+    out["value"] = out["decode"]["GB/s_signed"]
+    out["gpu_launches"] = None
+    return out
+
+
 # ------------------------------------------------------------ oracle (CPU)
 
 CPU_SLICE = 64  # tokens of a prefill layer the oracle evaluates (time extrapolated)
@@ -1110,6 +1238,10 @@ def main():
         out = run_gateup(args, rank, world, local_rank, dist)
     elif args.workload == "qlr":
         out = run_qlr(args, rank, world, local_rank, dist)
+    elif args.workload == "qkv":
+        out = run_qkv(args, rank, world, local_rank, dist)
+    elif args.workload == "rht":
+        out = run_rht(args, rank, world, local_rank, dist)
     else:
         out = run_prefill(args, rank, world, local_rank, dist)
     if rank == 0:
