@@ -505,18 +505,13 @@ def prefill_layers(tq, torch, sh, M, dev, rank, layers_cap=16, keep_cpu=False):
             "XL1": torch.empty(M, r, dtype=torch.float32, device=dev) if r else None,
             "XL1b": torch.empty(M, r, dtype=torch.bfloat16, device=dev) if r else None,
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
-            "ws": torch.zeros(tq.tq_gemm_workspace_bytes(M, N, K, r), dtype=torch.uint8,
+            "ws": torch.zeros(tq.tq_gemm_a8_workspace_bytes(M, N, K, r), dtype=torch.uint8,
                               device=dev),
         }
         if keep_cpu and i == 0:
             lay["cpu"] = {"X": X, "Rt": w["Rt"], "L1t": w["L1t"], "L2t": w["L2t"]}
         del w
         layers.append(lay)
-    # a stack of layers as in a decode step: layer i reads layer i-1's output
-    # (K = N), so every layer waits for its predecessor and finds its input in
-    # L2, as a model's next layer does; layer 0 reads the synthetic X
-    for prev, lay in zip(layers, layers[1:]):
-        lay["X"] = prev["Y"]
     torch.cuda.synchronize()
     return layers, per_layer
 

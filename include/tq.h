@@ -382,9 +382,21 @@ TQ_API int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block,
  *   Y[m][n] = bf16( s_x[m] s_w[n] sum_k qx[m][k] qw[n][k]
  *                   + sum_j XL1b[m][j] L2t[n][j] )
  *
- * the integer sum exact in INT32.  Same workspace rules as tq_w4a4_lr_gemm
- * (tq_gemm_workspace_bytes bytes, zeroed before first use).
+ * the integer sum exact in INT32.  Workspace: at least
+ * tq_gemm_workspace_bytes bytes, zeroed before first use.  With at least
+ * tq_gemm_a8_workspace_bytes bytes (a ~16 MB scratch after the status word)
+ * and a tile count that is not a whole multiple of the SM count, the
+ * persistent CTAs split the tiles x k-blocks evenly (stream-K): a CTA that
+ * computes part of a tile another CTA finishes leaves its INT32 partial sums
+ * and ready flags in the scratch, and the finishing CTA clears the flags, so
+ * the scratch is zero again after every call that completes.  Y is the same
+ * bit for bit under either schedule (integer sums).  After a call whose
+ * status reports TQ_ERR_TIMEOUT, zero the workspace again.  Calls that share
+ * a workspace must not overlap.  tq_w4a4_lr_gemm_a8_asym, ..._qlr, the layer
+ * (M > 128) and tq_w4a4_lr_gate_up follow the same rule with their own
+ * workspace sizes.
  */
+TQ_API size_t tq_gemm_a8_workspace_bytes(int M, int N, int K, int r);
 TQ_API int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x,
                               const uint8_t* Wq, const float* s_w,
                               const uint16_t* XL1b, const uint16_t* L2t,

@@ -14,5 +14,5 @@ from .tq import (  # noqa: F401
     tq_w4a4_lr_gemm_a8_asym, tq_pack_lowrank_q4, tq_quantize_act_qlr_i8, tq_w4a4_lr_gemm_a8_qlr,
     tq_noalloc_query_status, tq_debug_noalloc_set_status, tq_debug_watchdog,
     tq_debug_w4a4_lr_layer_decode, tq_pack_shared_input, split_shared_output,
-    tq_pack_weight_rht, tq_quantize_act_rht, tq_w4a4_lr_layer_rht,
+    tq_pack_weight_rht, tq_quantize_act_rht, tq_w4a4_lr_layer_rht, tq_gemm_a8_workspace_bytes,
 )

@@ -172,6 +172,17 @@ int tq_quantize_act_i8(const uint16_t* X, int M, int K, int had_block, const uin
                                      static_cast<cudaStream_t>(stream)));
 }
 
+// The a8 GEMM's stream-K scratch at byte `off` of a workspace, if it fits.
+static void* a8_sk(void* ws, size_t ws_bytes, size_t off) {
+  return ws && ws_bytes >= off + tq::gemm_a8_sk_bytes() ? static_cast<uint8_t*>(ws) + off
+                                                          : nullptr;
+}
+
+size_t tq_gemm_a8_workspace_bytes(int M, int N, int K, int r) {
+  (void)M; (void)N; (void)K; (void)r;
+  return 256 + tq::gemm_a8_sk_bytes();
+}
+
 int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x, const uint8_t* Wq, const float* s_w,
                        const uint16_t* XL1b, const uint16_t* L2t, int M, int N, int K, int r,
                        uint16_t* Y, void* ws, size_t ws_bytes, void* stream) {
@@ -198,12 +209,13 @@ int tq_w4a4_lr_gemm_a8(const int8_t* Xq8, const float* s_x, const uint8_t* Wq, c
   a.r = r;
   a.Y = Y;
   a.ws = ws;
+  a.sk = a8_sk(ws, ws_bytes, 256);
   return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
 }
 
 // Layer workspace, 256-aligned parts after the 256-byte status word: either
 // [Xq M*K/2][s_x 4M][XL1 4Mr] (packed codes) or [Xq8 M*K][s_x 4M][XL1b 2Mr]
-// (codes one per byte, M > 128).
+// [stream-K scratch] (codes one per byte, M > 128).
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 static bool layer_uses_a8(int M, int r, int had_block) {
@@ -225,8 +237,8 @@ size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {
   if (M <= 0 || N <= 0 || K <= 0 || r < 0) return 256;
   const size_t packed =
       align256((size_t)M * K / 2) + align256((size_t)M * 4) + align256((size_t)M * r * 4);
-  const size_t bytes8 =
-      align256((size_t)M * K) + align256((size_t)M * 4) + align256((size_t)M * r * 2);
+  const size_t bytes8 = align256((size_t)M * K) + align256((size_t)M * 4) +
+                        align256((size_t)M * r * 2) + tq::gemm_a8_sk_bytes();
   return 256 + (M > 128 ? std::max(packed, bytes8) : packed);
 }
 
@@ -286,6 +298,9 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
     a.r = r;
     a.Y = Y;
     a.ws = workspace;
+    a.sk = a8_sk(workspace, workspace_bytes,
+                 256 + align256((size_t)M * K) + align256((size_t)M * 4) +
+                     align256((size_t)M * r * 2));
     return from_cuda(tq::launch_gemm_a8(a, st));
   }
   uint8_t* Xq = ws + 256;
@@ -409,12 +424,13 @@ int tq_query_device_status(void* workspace, void* stream) {
 }
 
 // ------------------------------------------------------------- gate / up
-// Workspace of tq_w4a4_lr_gate_up: [status 256][Xq8 M*K][s_x 4M][XL1b 2M r2],
-// 256-aligned parts.
+// Workspace of tq_w4a4_lr_gate_up: [status 256][Xq8 M*K][s_x 4M][XL1b 2M r2]
+// [stream-K scratch], 256-aligned parts.
 size_t tq_gate_up_workspace_bytes(int M, int N, int K, int r2) {
   (void)N;
   if (M <= 0 || K <= 0 || r2 < 0) return 256;
-  return 256 + align256((size_t)M * K) + align256((size_t)M * 4) + align256((size_t)M * r2 * 2);
+  return 256 + align256((size_t)M * K) + align256((size_t)M * 4) +
+         align256((size_t)M * r2 * 2) + tq::gemm_a8_sk_bytes();
 }
 
 int tq_pack_gate_up(const uint8_t* Wq_g, const float* s_w_g, const uint16_t* L1t_g,
@@ -475,6 +491,9 @@ int tq_w4a4_lr_gate_up(const uint16_t* X, const uint16_t* L1t2, const uint8_t* W
   a.r = r2;
   a.Y = Y;
   a.ws = workspace;
+  a.sk = a8_sk(workspace, workspace_bytes,
+               256 + align256((size_t)M * K) + align256((size_t)M * 4) +
+                   align256((size_t)M * r2 * 2));
   a.swiglu = 1;
   return from_cuda(tq::launch_gemm_a8(a, st));
 }
@@ -589,6 +608,7 @@ int tq_w4a4_lr_gemm_a8_asym(const int8_t* Xq8, const float* s_x, const float* z_
   a.r = r;
   a.Y = Y;
   a.ws = ws;
+  a.sk = a8_sk(ws, ws_bytes, 256);
   a.z_x = z_x;
   a.wsum = wsum;
   return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));
@@ -672,6 +692,7 @@ int tq_w4a4_lr_gemm_a8_qlr(const int8_t* Xq8, const float* s_x, const uint8_t* W
   a.r = r;
   a.Y = Y;
   a.ws = ws;
+  a.sk = a8_sk(ws, ws_bytes, 256);
   a.s_xl1 = s_xl1;
   a.s_l2 = s_L2;
   return from_cuda(tq::launch_gemm_a8(a, static_cast<cudaStream_t>(stream)));

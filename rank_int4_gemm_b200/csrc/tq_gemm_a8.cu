@@ -20,6 +20,16 @@
 // tokens and weights per stage, then the low-rank chunks (64 columns of
 // bf16(XL1) and L2^T per stage, kind::f16 into the low-rank accumulator).
 //
+// Schedule.  Where the tiles fill whole waves of the CTAs well (or without
+// scratch in the workspace) CTA c takes tiles c, c + G, ...  Otherwise (stream-K) the
+// tiles x stages of k-blocks are dealt out in tile order as equal ranges of
+// stages, so no CTA idles through a last partial wave: a tile split between
+// CTAs is finished by the CTA holding its first stage (which also runs the
+// low-rank stages and the epilogue); each other CTA holding part of it (its
+// range starts inside that tile, so the part is the first thing it computes)
+// stores its INT32 partial sums in the workspace and raises one flag per
+// epilogue warp.  INT32 addition is exact, so Y does not depend on the split.
+//
 // Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-9:
 // weight expansion into TMEM, then the epilogue of the tile (warp w owns
 // lanes 32*(w%4)..: channel rows; warps w and w+4 split the k-blocks and the
@@ -72,7 +82,43 @@ struct A8Params {
   const int32_t* wsum;       //   [N] sums of each channel's weight codes
   const float* s_xl1;        // INT4 low-rank branch: [M] scales of the requantized X L1
   const float* s_l2;         //   and [N] of L2; the low-rank accumulator holds integers
+  int sk;                    // stream-K schedule
+  long long w_st;            //   tiles * n_st stages, dealt out as equal ranges
+  int32_t* part;             //   [gridDim.x][128][TK] INT32 partial sums
+  uint32_t* flags;           //   [gridDim.x][8] partial ready (one per epilogue warp)
 };
+
+// The segments of a CTA: (tile, stages [st0, st1) of its n_st).
+struct SegIter {
+  long long u, u_end;  // stream-K: this CTA's range of stages
+  int tile;            // otherwise: next tile
+  __device__ explicit SegIter(const A8Params& p) {
+    u = (long long)blockIdx.x * p.w_st / gridDim.x;
+    u_end = (long long)(blockIdx.x + 1) * p.w_st / gridDim.x;
+    tile = blockIdx.x;
+  }
+  __device__ bool next(const A8Params& p, int& t, int& st0, int& st1) {
+    if (p.sk) {
+      if (u >= u_end) return false;
+      t = (int)(u / p.n_st);
+      st0 = (int)(u - (long long)t * p.n_st);
+      st1 = (int)min((long long)p.n_st, (long long)st0 + (u_end - u));
+      u += st1 - st0;
+      return true;
+    }
+    if (tile >= p.tiles) return false;
+    t = tile;
+    st0 = 0;
+    st1 = p.n_st;
+    tile += gridDim.x;
+    return true;
+  }
+};
+
+// First stage of CTA c's stream-K range.
+__device__ __forceinline__ long long sk_begin(const A8Params& p, int c) {
+  return (long long)c * p.w_st / gridDim.x;
+}
 
 // Shared memory (offsets from the 1024-aligned base).  Stage s: tokens
 // [2 k-blocks][TK rows][128 B] then packed weights [128 rows][128 B]
@@ -174,13 +220,17 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       const uint64_t pol_t = policy_evict_last();   // tokens: reused by every channel tile
       bool waited = false;                          // the weights need no predecessor
       int it = 0;
-      for (int tile = blockIdx.x; tile < p.tiles && !*abort_flag; tile += gridDim.x) {
+      SegIter seg(p);
+      int tile, st0, st1;
+      while (!*abort_flag && seg.next(p, tile, st0, st1)) {
         const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
-        for (int st = 0; st < p.n_st + p.n_lr; ++st, ++it) {
+        const int n_lr = st0 == 0 ? p.n_lr : 0;  // the finishing CTA runs the low-rank stages
+        for (int j = 0; j < st1 - st0 + n_lr; ++j, ++it) {
           const int s = it % kNS;
           if (!mbar_wait(&empty[s], ((uint32_t)(it / kNS) & 1u) ^ 1u, p.status, abort_flag)) break;
           uint8_t* sp = smem + (uint32_t)s * L::kStage;
-          if (st < p.n_st) {
+          if (j < st1 - st0) {
+            const int st = st0 + j;
             const int kb = 2 * st;
             const bool two = kb + 1 < p.kb_total;
             mbar_arrive_expect_tx(&full[s], L::kWBytes + (two ? 2u : 1u) * L::kTokSub);
@@ -192,7 +242,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
             tma_load_2d(sp, &map_t, &full[s], kb * kKb, tm * TK, pol_t);
             if (two) tma_load_2d(sp + L::kTokSub, &map_t, &full[s], (kb + 1) * kKb, tm * TK, pol_t);
           } else {
-            const int c = st - p.n_st;  // 64-column low-rank chunk
+            const int c = j - (st1 - st0);  // 64-column low-rank chunk
             mbar_arrive_expect_tx(&full[s], L::kWBytes + L::kTokSub);
             if (!waited) {
               pdl_wait();
@@ -211,19 +261,22 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     const uint32_t id_bf = idesc_bf16_f32(TK);
     int it = 0, ab = 0, tcount = 0;
     bool alive = true;
-    for (int tile = blockIdx.x; tile < p.tiles && alive && !*abort_flag;
-         tile += gridDim.x, ++tcount) {
-      // the epilogue has drained the accumulators of the previous tile
+    SegIter seg(p);
+    int tile, st0, st1;
+    for (; alive && !*abort_flag && seg.next(p, tile, st0, st1); ++tcount) {
+      const int n_lr = st0 == 0 ? p.n_lr : 0;
+      // the epilogue has drained the accumulators of the previous segment
       if (!mbar_wait(acc_empty, ((uint32_t)tcount & 1u) ^ 1u, p.status, abort_flag)) break;
       tc_fence_after();
-      for (int st = 0; st < p.n_st + p.n_lr && alive; ++st, ++it) {
+      for (int j = 0; j < st1 - st0 + n_lr && alive; ++j, ++it) {
         const int s = it % kNS;
         if (!mbar_wait(&full[s], (uint32_t)(it / kNS) & 1u, p.status, abort_flag)) {
           alive = false;
           break;
         }
         const uint32_t sp = base + (uint32_t)s * L::kStage;
-        if (st < p.n_st) {
+        if (j < st1 - st0) {
+          const int st = st0 + j;
           for (int sub = 0; sub < 2 && 2 * st + sub < p.kb_total; ++sub, ++ab) {
             const int u = ab % kNA;
             if (!mbar_wait(&a_full[u], (uint32_t)(ab / kNA) & 1u, p.status, abort_flag)) {
@@ -236,7 +289,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk)  // K = 32 int8 = 8 TMEM columns per step
                 mma_i8_tmem_a(tmem + kColAcc, tmem + kColA + 32u * (uint32_t)u + 8u * (uint32_t)kk,
-                              db + 2 * kk, id_i8, (st > 0 || sub > 0 || kk > 0) ? 1u : 0u);
+                              db + 2 * kk, id_i8, (st > st0 || sub > 0 || kk > 0) ? 1u : 0u);
               mma_commit(&a_empty[u]);
             }
             __syncwarp();
@@ -244,7 +297,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         } else {
           tc_fence_after();
           if (lane == 0) {
-            const int c = st - p.n_st;
+            const int c = j - (st1 - st0);
             const uint64_t da = sdesc_sw128(sp + 2 * L::kTokSub);  // L2^T chunk [128][64]
             const uint64_t db = sdesc_sw128(sp);                    // bf16(XL1) chunk [192][64]
 #pragma unroll
@@ -269,17 +322,32 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     pdl_wait();  // s_x comes from the preceding kernel
     int it = 0, ab = 0, tcount = 0;
     bool alive = true;
-    for (int tile = blockIdx.x; tile < p.tiles && alive && !*abort_flag;
-         tile += gridDim.x, ++tcount) {
+    SegIter seg(p);
+    int tile, st0, st1;
+    for (; alive && !*abort_flag && seg.next(p, tile, st0, st1); ++tcount) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int gc = tn * kCh + row;
       const float sw = gc < p.N ? __ldg(p.s_w + gc) : 0.f;
       const int ws = (EPI == kEpiAsym && gc < p.N) ? __ldg(p.wsum + gc) : 0;
       const float sl2 = (EPI == kEpiQlr && p.r > 0 && gc < p.N) ? __ldg(p.s_l2 + gc) : 0.f;
+      // the per-token scales of this warp's epilogue chunks (token lane of
+      // chunk half + 2i), requested now so that their latency is hidden
+      // behind the main loop
+      constexpr int kChunks = TK / 64;
+      float sx_pre[kChunks], zx_pre[kChunks];
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int t = tm * TK + 32 * (half + 2 * i) + lane;
+        const bool in = st0 == 0 && t < p.M;
+        sx_pre[i] = in ? __ldg(p.s_x + t) : 0.f;
+        zx_pre[i] = (EPI == kEpiAsym && in) ? __ldg(p.z_x + t)
+                    : (EPI == kEpiQlr && p.r > 0 && in) ? __ldg(p.s_xl1 + t)
+                                                        : 0.f;
+      }
       // int4 -> int8 (16 * code) for this thread's channel row, one k-block
       // (32 TMEM columns) at a time; inside each 16-byte packed chunk the low
       // nibbles are codes 0-15 and the high nibbles codes 16-31 of the group
-      for (int st = 0; st < p.n_st && alive; ++st, ++it) {
+      for (int st = st0; st < st1 && alive; ++st, ++it) {
         const int s = it % kNS;
         if (!mbar_wait(&full[s], (uint32_t)(it / kNS) & 1u, p.status, abort_flag)) {
           alive = false;
@@ -322,7 +390,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         if (mine) mbar_arrive(&a_full[(ab + half) % kNA]);
         ab += nsub;
       }
-      it += p.n_lr;  // low-rank stages go to the MMA only
+      it += st0 == 0 ? p.n_lr : 0;  // low-rank stages go to the MMA only
       if (!alive) break;
       // ---- epilogue: Y[t][c] = s_x[t] s_w[c] (acc >> 4) + lr, bf16.  Each
       //      warp owns 32 channels; per 32 tokens it transposes its block
@@ -330,17 +398,55 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       if (!__all_sync(0xffffffffu, mbar_wait(acc_full, (uint32_t)tcount & 1u, p.status, abort_flag)))
         break;
       tc_fence_after();
+      const int ew = warp - 2;  // epilogue warp: its rows and token chunks are the same in every CTA
+      if (st0 > 0) {
+        // part of a tile another CTA finishes: this warp's INT32 sums to the
+        // workspace, then its flag
+        // (slot layout [chunk][8 x 16 bytes][row]: a warp's store of one
+        // 16-byte piece covers 512 contiguous bytes)
+        uint32_t a[kChunks][32];
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i)
+          tmem_ld32(tmem + kColAcc + (uint32_t)(32 * (half + 2 * i)) + lane_off, a[i]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(acc_empty);  // the next segment's MMAs may start
+        uint4* dst = reinterpret_cast<uint4*>(p.part + (size_t)blockIdx.x * kCh * TK);
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[((half + 2 * i) * 8 + v) * kCh + row] =
+                make_uint4(a[i][4 * v], a[i][4 * v + 1], a[i][4 * v + 2], a[i][4 * v + 3]);
+        __syncwarp();
+        if (lane == 0) {
+          __threadfence();
+          st_release_gpu(p.flags + (size_t)blockIdx.x * kConvWarpsA8 + ew, 1u);
+        }
+        __syncwarp();
+        continue;
+      }
+      // the CTAs whose ranges start inside this tile: their partials
+      int c_lo = blockIdx.x + 1, c_hi = c_lo;
+      if (st1 < p.n_st) {
+        const long long tile_end = (long long)(tile + 1) * p.n_st;
+        while (c_hi < (int)gridDim.x && sk_begin(p, c_hi) < tile_end) ++c_hi;
+        bool ok = true;
+        for (int c = c_lo; c < c_hi && ok; ++c)
+          ok = flag_wait(p.flags + (size_t)c * kConvWarpsA8 + ew, 1u, p.status, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
       const uint32_t ybuf = base + L::kYBuf + (uint32_t)(warp - 2) * 32u * L::kYRow;
       const int gc0 = tn * kCh + q * 32;  // first channel of this warp
-      for (int j = half; j < TK / 32; j += 2) {
+#pragma unroll
+      for (int i = 0; i < kChunks; ++i) {
+        const int j = half + 2 * i;
         uint32_t a[32], l[32];
         tmem_ld32(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
         if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
         const int t0 = tm * TK + 32 * j;
-        const float sx_l = (t0 + lane < p.M) ? __ldg(p.s_x + t0 + lane) : 0.f;
-        const float zx_l = (EPI == kEpiAsym && t0 + lane < p.M) ? __ldg(p.z_x + t0 + lane)
-                           : (EPI == kEpiQlr && p.r > 0 && t0 + lane < p.M) ? __ldg(p.s_xl1 + t0 + lane)
-                                                                 : 0.f;
+        const float sx_l = sx_pre[i];
+        const float zx_l = zx_pre[i];
         // adds the low-rank term: fp32 (bf16 branch), or s_xl1 s_L2 times the
         // exact integer sum of the INT4 branch.  The token's s_xl1 shuffle
         // stays outside the r > 0 branch: inside it the 32 shuffles of a
@@ -363,6 +469,17 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
           return sw * (sx * (float)(acc + 8 * ws) + zx * (float)ws);
         };
         tmem_ld_wait();
+        for (int c = c_lo; c < c_hi; ++c) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.part + (size_t)c * kCh * TK);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = ld_cg_v4(src + (j * 8 + v) * kCh + row);
+            a[4 * v] += x.x;
+            a[4 * v + 1] += x.y;
+            a[4 * v + 2] += x.z;
+            a[4 * v + 3] += x.w;
+          }
+        }
         if constexpr (EPI != kEpiSwiglu) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -422,6 +539,9 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
         }
         __syncwarp();
       }
+      // the partials are consumed: clear their flags for the next launch
+      if (lane == 0)
+        for (int c = c_lo; c < c_hi; ++c) p.flags[(size_t)c * kConvWarpsA8 + ew] = 0u;
       tc_fence_before();
       mbar_arrive(acc_empty);
     }
@@ -438,6 +558,12 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
 }  // namespace
 
 namespace {
+
+// stream-K scratch: [kSkMaxCtas][8] flags, then [kSkMaxCtas][128][192] INT32
+constexpr int kSkMaxCtas = 160;
+constexpr size_t kSkFlagBytes = (size_t)kSkMaxCtas * kConvWarpsA8 * 4;
+constexpr size_t kSkPartBytes = (size_t)kSkMaxCtas * kCh * kTkMax * 4;
+static_assert(kSkFlagBytes % 256 == 0, "partials 256-byte aligned");
 
 template <int TK, int EPI>
 cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stream) {
@@ -459,6 +585,19 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
     map_xb = map_t;  // never read
     map_l2 = map_t;
   }
+  // stream-K (see the schedule note at the top) where tile-by-tile CTAs
+  // would leave much of their last wave idle: the waves' useful fraction
+  // tiles / (G ceil(tiles / G)) below 0.85.  Above it the tile schedule was
+  // measured faster (2048 x 4096 x 14336: 0.92, equal; 4096^3: 0.95, 3 %
+  // faster; 2048 x 14336 x 4096: 0.79, stream-K 11 % faster).  One CTA per
+  // SM, all resident at once.
+  const int sms = num_sms();
+  p.w_st = (long long)p.tiles * p.n_st;
+  const int waves = (p.tiles + sms - 1) / sms;
+  const bool uneven = (double)p.tiles < 0.85 * (double)waves * (double)sms;
+  p.sk = (a.sk != nullptr && sms <= kSkMaxCtas && uneven && p.w_st >= sms) ? 1 : 0;
+  p.flags = p.sk ? static_cast<uint32_t*>(a.sk) : nullptr;
+  p.part = p.sk ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(a.sk) + kSkFlagBytes) : nullptr;
   static uint64_t attr_set = 0;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -470,7 +609,7 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
     attr_set |= uint64_t(1) << dev;
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(std::min(p.tiles, num_sms()), 1, 1);
+  cfg.gridDim = dim3(p.sk ? sms : std::min(p.tiles, sms), 1, 1);
   cfg.blockDim = dim3(kThreadsA8, 1, 1);
   cfg.dynamicSmemBytes = A8Smem<TK>::kAlloc;
   cfg.stream = stream;
@@ -483,6 +622,8 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
 }
 
 }  // namespace
+
+size_t gemm_a8_sk_bytes() { return kSkFlagBytes + kSkPartBytes; }
 
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream) {
   A8Params p{};

@@ -50,8 +50,13 @@ struct GemmA8Args {
   const int32_t* wsum = nullptr;  //   and [N] weight code sums
   const float* s_xl1 = nullptr;   // INT4 low-rank branch: [M] and [N] scales (XL1b and
   const float* s_l2 = nullptr;    //   L2t then hold integer codes in bf16)
+  void* sk = nullptr;             // stream-K scratch (gemm_a8_sk_bytes(), zero-filled before
+                                  //   first use), or null for tile-by-tile CTAs only
 };
 cudaError_t launch_gemm_a8(const GemmA8Args& a, cudaStream_t stream);
+// Bytes of the a8 GEMM's stream-K scratch: ready flags and INT32 partial
+// tiles for up to one split tile per CTA.
+size_t gemm_a8_sk_bytes();
 cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int N, int K, int r,
                                    int had_block, int8_t* qL1, float* s_L1, uint16_t* qL2,
                                    float* s_L2, cudaStream_t stream);

@@ -139,6 +139,44 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
   }
 }
 
+// Global-memory flags between CTAs of one grid (all resident at once):
+// release store / acquire load at GPU scope, and a bounded wait on a flag
+// (same budget, status and abort rules as mbar_wait).
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool flag_wait(const uint32_t* f, uint32_t want, uint32_t* status,
+                                          volatile int* abort_flag,
+                                          long long budget = kWaitBudgetCycles) {
+  if (ld_acquire_gpu(f) == want) return true;
+  const long long t0 = clock64();
+  for (uint32_t it = 0;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(f) == want) return true;
+    if ((it & 15u) == 15u) {
+      if (abort_flag && *abort_flag) return false;
+      if (clock64() - t0 > budget) {
+        if (status) atomicExch(status, kDevTimeout);
+        if (abort_flag) *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+// 16-byte global load cached in L2 only (data another SM wrote this launch).
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 // 16 bytes into the shared memory of a CTA of this cluster (addresses from
 // mapa), completing as transaction bytes on that CTA's mbarrier `rbar`.
 __device__ __forceinline__ void st_async_v4(uint32_t raddr, uint4 v, uint32_t rbar) {

@@ -33,6 +33,8 @@ _lib.tq_quantize_act.restype = _I
 _lib.tq_quantize_act.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P]
 _lib.tq_gemm_workspace_bytes.restype = ctypes.c_size_t
 _lib.tq_gemm_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.tq_gemm_a8_workspace_bytes.restype = ctypes.c_size_t
+_lib.tq_gemm_a8_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.tq_w4a4_lr_gemm.restype = _I
 _lib.tq_w4a4_lr_gemm.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P,
                                   ctypes.c_size_t, _P]
@@ -202,6 +204,11 @@ def tq_gemm_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
     return int(_lib.tq_gemm_workspace_bytes(M, N, K, r))
 
 
+def tq_gemm_a8_workspace_bytes(M: int, N: int, K: int, r: int) -> int:
+    """Workspace of the codes-one-per-byte GEMMs with their stream-K scratch."""
+    return int(_lib.tq_gemm_a8_workspace_bytes(M, N, K, r))
+
+
 class Workspace:
     """A zero-filled device workspace that grows on demand (plumbing)."""
 
@@ -245,7 +252,7 @@ def tq_w4a4_lr_gemm_a8(Xq8, s_x, Wq, s_w, XL1b=None, L2t=None, Y=None, workspace
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
     if workspace is None:
         workspace = Workspace(Xq8.device)
-    need = tq_gemm_workspace_bytes(M, N, K, r)
+    need = tq_gemm_a8_workspace_bytes(M, N, K, r)
     ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
     _check(_lib.tq_w4a4_lr_gemm_a8(_ptr(Xq8), _ptr(s_x), _ptr(Wq), _ptr(s_w),
                                    _ptr(XL1b) if r else None, _ptr(L2t) if r else None,
@@ -293,7 +300,7 @@ def tq_w4a4_lr_gemm_a8_asym(Xq8, s_x, z_x, Wq, s_w, wsum, XL1b=None, L2t=None, Y
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
     if workspace is None:
         workspace = Workspace(Xq8.device)
-    need = tq_gemm_workspace_bytes(M, N, K, r)
+    need = tq_gemm_a8_workspace_bytes(M, N, K, r)
     ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
     _check(_lib.tq_w4a4_lr_gemm_a8_asym(_ptr(Xq8), _ptr(s_x), _ptr(z_x), _ptr(Wq), _ptr(s_w),
                                         _ptr(wsum), _ptr(XL1b) if r else None,
@@ -349,7 +356,7 @@ def tq_w4a4_lr_gemm_a8_qlr(Xq8, s_x, Wq, s_w, XL1q, s_xl1, qL2, s_L2, Y=None, wo
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=Xq8.device)
     if workspace is None:
         workspace = Workspace(Xq8.device)
-    need = tq_gemm_workspace_bytes(M, N, K, r)
+    need = tq_gemm_a8_workspace_bytes(M, N, K, r)
     ws = workspace.get(need) if isinstance(workspace, Workspace) else workspace
     _check(_lib.tq_w4a4_lr_gemm_a8_qlr(_ptr(Xq8), _ptr(s_x), _ptr(Wq), _ptr(s_w), _ptr(XL1q),
                                        _ptr(s_xl1), _ptr(qL2), _ptr(s_L2), M, N, K, r, _ptr(Y),

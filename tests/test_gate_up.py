@@ -48,6 +48,7 @@ CASES = [
     ("rank0", 200, 512, 136, 0, 128),
     ("wide_rank", 150, 512, 256, 128, 32),
     ("no_rotation", 140, 512, 136, 32, 1),
+    ("stream_k", 600, 2048, 1024, 32, 128),   # 64 tiles x 8 stages over the SMs
 ]
 
 
