@@ -129,10 +129,14 @@ struct A8Smem {
   static constexpr uint32_t kTokSub = TK * 128;             // 24 KB at TK = 192
   static constexpr uint32_t kWBytes = kCh * 128;            // 16 KB
   static constexpr uint32_t kStage = 2 * kTokSub + kWBytes;  // 64 KB
-  // epilogue transpose buffers, one per converter warp: [32 tokens][40 bf16]
+  // epilogue buffers per converter warp: a [32 tokens][40 bf16] transpose
+  // buffer (SwiGLU), or two [32 tokens][32 bf16] tiles in the 64-byte
+  // swizzle of the Y tensor map (the TMA store's source, alternating)
   static constexpr uint32_t kYRow = 80;
+  static constexpr uint32_t kYTile = 2048;
+  static constexpr uint32_t kYWarp = 2 * kYTile;
   static constexpr uint32_t kYBuf = kNS * kStage;
-  static constexpr uint32_t kBar = kYBuf + kConvWarpsA8 * 32 * kYRow;
+  static constexpr uint32_t kBar = kYBuf + kConvWarpsA8 * kYWarp;
   // full[kNS], empty[kNS], a_full[kNA], a_empty[kNA], acc_full, acc_empty
   static constexpr uint32_t kNumBars = 2 * kNS + 2 * A8Tmem<TK>::kNA + 2;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
@@ -140,6 +144,15 @@ struct A8Smem {
   static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 static_assert(A8Smem<kTkMax>::kAlloc <= 227 * 1024, "a8 GEMM shared memory");
+static_assert(A8Smem<kTkMax>::kYBuf % 1024 == 0 && A8Smem<kTkMax>::kYWarp >= 32 * A8Smem<kTkMax>::kYRow,
+              "Y tiles 1024-B aligned; the SwiGLU transpose buffer fits a warp's share");
+
+// (float) n for |n| < 2^22, exactly, on the FMA pipe: n added to the bit
+// pattern of 1.5 * 2^23 is the float 1.5 * 2^23 + n (the spacing there is
+// 1), and the subtraction is exact.
+__device__ __forceinline__ float int22_to_float(int n) {
+  return __int_as_float(n + 0x4B400000) - 12582912.f;
+}
 
 __device__ __forceinline__ uint4 ld_shared_v4_a8(uint32_t addr) {
   uint4 v;
@@ -159,6 +172,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
                            const __grid_constant__ CUtensorMap map_w,   // weights [N][K/2]
                            const __grid_constant__ CUtensorMap map_xb,  // bf16(XL1) [M][r]
                            const __grid_constant__ CUtensorMap map_l2,  // L2^T [N][r]
+                           const __grid_constant__ CUtensorMap map_y,   // Y [M][N] (not SwiGLU)
                            const A8Params p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -199,6 +213,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     fence_barrier_init();
     tma_prefetch_desc(&map_t);
     tma_prefetch_desc(&map_w);
+    if (EPI != kEpiSwiglu) tma_prefetch_desc(&map_y);
     if (p.r > 0) {
       tma_prefetch_desc(&map_xb);
       tma_prefetch_desc(&map_l2);
@@ -319,30 +334,48 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     const int row = q * 32 + lane;                   // channel row of the tile
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
     const uint32_t x7 = (uint32_t)row & 7u;
+    // every variant but SwiGLU reads the accumulators in the 16x256b
+    // fragment layout and stores Y through stmatrix (no shuffles)
+    constexpr bool kFrag = EPI != kEpiSwiglu;
     pdl_wait();  // s_x comes from the preceding kernel
-    int it = 0, ab = 0, tcount = 0;
+    int it = 0, ab = 0, tcount = 0, n_ystores = 0;
     bool alive = true;
     SegIter seg(p);
     int tile, st0, st1;
     for (; alive && !*abort_flag && seg.next(p, tile, st0, st1); ++tcount) {
       const int tm = tile % p.tiles_m, tn = tile / p.tiles_m;
       const int gc = tn * kCh + row;
-      const float sw = gc < p.N ? __ldg(p.s_w + gc) : 0.f;
-      const int ws = (EPI == kEpiAsym && gc < p.N) ? __ldg(p.wsum + gc) : 0;
-      const float sl2 = (EPI == kEpiQlr && p.r > 0 && gc < p.N) ? __ldg(p.s_l2 + gc) : 0.f;
-      // the per-token scales of this warp's epilogue chunks (token lane of
-      // chunk half + 2i), requested now so that their latency is hidden
-      // behind the main loop
+      const float sw = (!kFrag && gc < p.N) ? __ldg(p.s_w + gc) : 0.f;  // SwiGLU's row scale
+      // the epilogue's scales, requested now so that their latency hides
+      // behind the main loop.  Fragment epilogue (every variant but SwiGLU):
+      // this thread's tokens 8g + 2 (lane % 4) + {0, 1} of each of its 32-token
+      // chunks (s_x, and z_x or s_xl1) and channels 16h + lane / 4 + 8s of the
+      // warp's 32 (s_w, and wsum or s_L2), f = 2h + s.  SwiGLU: the token lane
+      // of each chunk (entry 0).
       constexpr int kChunks = TK / 64;
-      float sx_pre[kChunks], zx_pre[kChunks];
+      float sx_pre[kChunks][8], zx_pre[kChunks][8];
 #pragma unroll
       for (int i = 0; i < kChunks; ++i) {
-        const int t = tm * TK + 32 * (half + 2 * i) + lane;
-        const bool in = st0 == 0 && t < p.M;
-        sx_pre[i] = in ? __ldg(p.s_x + t) : 0.f;
-        zx_pre[i] = (EPI == kEpiAsym && in) ? __ldg(p.z_x + t)
-                    : (EPI == kEpiQlr && p.r > 0 && in) ? __ldg(p.s_xl1 + t)
-                                                        : 0.f;
+        const int tb = tm * TK + 32 * (half + 2 * i);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int t = kFrag ? tb + 8 * (e >> 1) + 2 * (lane & 3) + (e & 1) : tb + lane;
+          const bool in = st0 == 0 && t < p.M && (kFrag || e == 0);
+          sx_pre[i][e] = in ? __ldg(p.s_x + t) : 0.f;
+          zx_pre[i][e] = (EPI == kEpiAsym && in) ? __ldg(p.z_x + t)
+                         : (EPI == kEpiQlr && p.r > 0 && in) ? __ldg(p.s_xl1 + t)
+                                                             : 0.f;
+        }
+      }
+      float sw_f[4], sl2_f[4];
+      int ws_f[4];
+#pragma unroll
+      for (int f = 0; f < 4; ++f) {
+        const int c = tn * kCh + q * 32 + 16 * (f >> 1) + (lane >> 2) + 8 * (f & 1);
+        const bool in = kFrag && st0 == 0 && c < p.N;
+        sw_f[f] = in ? __ldg(p.s_w + c) : 0.f;
+        ws_f[f] = (EPI == kEpiAsym && in) ? __ldg(p.wsum + c) : 0;
+        sl2_f[f] = (EPI == kEpiQlr && p.r > 0 && in) ? __ldg(p.s_l2 + c) : 0.f;
       }
       // int4 -> int8 (16 * code) for this thread's channel row, one k-block
       // (32 TMEM columns) at a time; inside each 16-byte packed chunk the low
@@ -402,22 +435,45 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
       if (st0 > 0) {
         // part of a tile another CTA finishes: this warp's INT32 sums to the
         // workspace, then its flag
-        // (slot layout [chunk][8 x 16 bytes][row]: a warp's store of one
-        // 16-byte piece covers 512 contiguous bytes)
-        uint32_t a[kChunks][32];
-#pragma unroll
-        for (int i = 0; i < kChunks; ++i)
-          tmem_ld32(tmem + kColAcc + (uint32_t)(32 * (half + 2 * i)) + lane_off, a[i]);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(acc_empty);  // the next segment's MMAs may start
+        // (slot layout [chunk][8 x 16 bytes][row] in the layout of the
+        // finishing CTA's loads: a warp's store of one 16-byte piece covers
+        // 512 contiguous bytes)
         uint4* dst = reinterpret_cast<uint4*>(p.part + (size_t)blockIdx.x * kCh * TK);
+        if constexpr (kFrag) {
+          uint32_t a[kChunks][2][16];
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i)
+          for (int i = 0; i < kChunks; ++i)
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            dst[((half + 2 * i) * 8 + v) * kCh + row] =
-                make_uint4(a[i][4 * v], a[i][4 * v + 1], a[i][4 * v + 2], a[i][4 * v + 3]);
+            for (int h = 0; h < 2; ++h)
+              tmem_ld16x256_x4(tmem + kColAcc + (uint32_t)(32 * (half + 2 * i)) + lane_off +
+                                   ((uint32_t)(16 * h) << 16), a[i][h]);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(acc_empty);  // the next segment's MMAs may start
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[(((half + 2 * i) * 2 + h) * 4 + k) * kCh + q * 32 + lane] =
+                    make_uint4(a[i][h][4 * k], a[i][h][4 * k + 1], a[i][h][4 * k + 2],
+                               a[i][h][4 * k + 3]);
+        } else {
+          uint32_t a[kChunks][32];
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i)
+            tmem_ld32(tmem + kColAcc + (uint32_t)(32 * (half + 2 * i)) + lane_off, a[i]);
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(acc_empty);  // the next segment's MMAs may start
+#pragma unroll
+          for (int i = 0; i < kChunks; ++i)
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[((half + 2 * i) * 8 + v) * kCh + row] =
+                  make_uint4(a[i][4 * v], a[i][4 * v + 1], a[i][4 * v + 2], a[i][4 * v + 3]);
+        }
         __syncwarp();
         if (lane == 0) {
           __threadfence();
@@ -436,91 +492,136 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
           ok = flag_wait(p.flags + (size_t)c * kConvWarpsA8 + ew, 1u, p.status, abort_flag);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
-      const uint32_t ybuf = base + L::kYBuf + (uint32_t)(warp - 2) * 32u * L::kYRow;
+      const uint32_t ybuf = base + L::kYBuf + (uint32_t)(warp - 2) * L::kYWarp;
       const int gc0 = tn * kCh + q * 32;  // first channel of this warp
+      if constexpr (kFrag) {
+        const bool small_k = p.K <= 85504;  // 49 K < 2^22
 #pragma unroll
-      for (int i = 0; i < kChunks; ++i) {
-        const int j = half + 2 * i;
-        uint32_t a[32], l[32];
-        tmem_ld32(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
-        if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
-        const int t0 = tm * TK + 32 * j;
-        const float sx_l = sx_pre[i];
-        const float zx_l = zx_pre[i];
-        // adds the low-rank term: fp32 (bf16 branch), or s_xl1 s_L2 times the
-        // exact integer sum of the INT4 branch.  The token's s_xl1 shuffle
-        // stays outside the r > 0 branch: inside it the 32 shuffles of a
-        // block do not pipeline (measured 17 % on the whole GEMM)
-        auto add_lowrank = [&](float& y, int e) {
-          if constexpr (EPI == kEpiQlr) {
-            const float sxl = __shfl_sync(0xffffffffu, zx_l, e);
-            if (p.r > 0) y += sxl * sl2 * __uint_as_float(l[e]);
-          } else {
-            if (p.r > 0) y += __uint_as_float(l[e]);
-          }
-        };
-        // y = s_x s_w acc; asymmetric codes c = q - 8 with zero-point z:
-        // sum q qw = acc + 8 wsum (exact), y = s_w (s_x (acc + 8 wsum) + z wsum)
-        auto dequant = [&](int e) -> float {
-          const int acc = ((int)a[e]) >> 4;
-          const float sx = __shfl_sync(0xffffffffu, sx_l, e);
-          if constexpr (EPI != kEpiAsym) return sx * sw * (float)acc;
-          const float zx = __shfl_sync(0xffffffffu, zx_l, e);
-          return sw * (sx * (float)(acc + 8 * ws) + zx * (float)ws);
-        };
-        tmem_ld_wait();
-        for (int c = c_lo; c < c_hi; ++c) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.part + (size_t)c * kCh * TK);
-#pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            const uint4 x = ld_cg_v4(src + (j * 8 + v) * kCh + row);
-            a[4 * v] += x.x;
-            a[4 * v + 1] += x.y;
-            a[4 * v + 2] += x.z;
-            a[4 * v + 3] += x.w;
-          }
-        }
-        if constexpr (EPI != kEpiSwiglu) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float y = dequant(e);
-            add_lowrank(y, e);
-            const __nv_bfloat16 h = __float2bfloat16_rn(y);
-            asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + 2u * (uint32_t)lane),
-                         "h"(*reinterpret_cast<const unsigned short*>(&h))
-                         : "memory");
-          }
+        for (int i = 0; i < kChunks; ++i) {
+          const int j = half + 2 * i;
+          // this warp's tile buffers alternate over all its stores: the
+          // store before the last one (same buffer) has read it
+          const uint32_t ytile = base + L::kYBuf + (uint32_t)(warp - 2) * L::kYWarp +
+                                 (uint32_t)(n_ystores & 1) * L::kYTile;
+          if (lane == 0) bulk_wait_read_but1();
           __syncwarp();
+          // a[h] / l[h]: lanes 16h .. 16h + 15 of the warp's quarter, 32 tokens
+          uint32_t a[2][16], l[2][16];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int idx = lane + 32 * k;      // 32 token rows x 4 16-byte parts
-            const int e = idx >> 2, part = idx & 3;
-            const uint4 v = ld_shared_v4_a8(ybuf + (uint32_t)e * L::kYRow + (uint32_t)part * 16u);
-            const int t = t0 + e, c = gc0 + part * 8;
-            if (t < p.M && c < p.N)
-              *reinterpret_cast<uint4*>(p.Y + (size_t)t * p.N + c) = v;
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t lo = lane_off + ((uint32_t)(16 * h) << 16) + (uint32_t)(32 * j);
+            tmem_ld16x256_x4(tmem + kColAcc + lo, a[h]);
+            if (p.r > 0) tmem_ld16x256_x4(tmem + kColLr + lo, l[h]);
           }
-        } else {
-          // channel rows alternate gate (even lane) and up (odd lane).  For
-          // each pair of tokens (2i, 2i+1) one shuffle gives the even lane
-          // (g, u) of token 2i and the odd lane those of token 2i+1, so every
-          // lane computes 16 of the warp's 16 x 32 outputs; silu(g) =
-          // g / (1 + e^-g) with the fast exponential and division (relative
-          // error ~1e-6, far below the bf16 output's 2^-9)
+          tmem_ld_wait();
+          for (int c = c_lo; c < c_hi; ++c) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.part + (size_t)c * kCh * TK);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const uint4 x = ld_cg_v4(src + ((j * 2 + h) * 4 + k) * kCh + q * 32 + lane);
+                a[h][4 * k] += x.x;
+                a[h][4 * k + 1] += x.y;
+                a[h][4 * k + 2] += x.z;
+                a[h][4 * k + 3] += x.w;
+              }
+          }
+          const int t0 = tm * TK + 32 * j;
+          // per group of 8 tokens, four 8x8 blocks (channels 8f .. 8f + 7 of
+          // the warp's 32): this thread's two tokens of one channel each, the
+          // stmatrix fragment of the channel x token block, stored transposed
+          // as token rows of 8 channels
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint32_t P[4];
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              const int h = f >> 1, sb = f & 1;
+              float y[2];
+#pragma unroll
+              for (int u = 0; u < 2; ++u) {
+                const int rg = 4 * g + 2 * sb + u;  // register of (channel, token 8g + 2(lane%4) + u)
+                const int acc = ((int)a[h][rg]) >> 4;
+                // |acc| <= 49 K for symmetric codes
+                const float facc = (EPI != kEpiAsym && small_k) ? int22_to_float(acc) : (float)acc;
+                const float sx = sx_pre[i][2 * g + u];
+                float v;
+                // y = s_x s_w acc; asymmetric codes c = q - 8 with zero-point
+                // z: sum q qw = acc + 8 wsum (exact), y = s_w (s_x (acc + 8
+                // wsum) + z wsum); then the low-rank term: fp32 (bf16 branch),
+                // or s_xl1 s_L2 times the exact integer sum of the INT4 branch
+                if constexpr (EPI == kEpiAsym)
+                  v = sw_f[f] * (sx * (float)(acc + 8 * ws_f[f]) + zx_pre[i][2 * g + u] * (float)ws_f[f]);
+                else
+                  v = sx * sw_f[f] * facc;
+                if constexpr (EPI == kEpiQlr) {
+                  if (p.r > 0) v += zx_pre[i][2 * g + u] * sl2_f[f] * __uint_as_float(l[h][rg]);
+                } else {
+                  if (p.r > 0) v += __uint_as_float(l[h][rg]);
+                }
+                y[u] = v;
+              }
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(y[0], y[1]);
+              P[f] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            // row 8g + lane % 8 (a token), 16-byte chunk lane / 8 (8
+            // channels), in the 64-byte swizzle: chunk ^ ((row / 2) % 4)
+            const uint32_t yr = (uint32_t)(8 * g + (lane & 7));
+            stmatrix_x4_trans(ytile + yr * 64u + ((((uint32_t)(lane >> 3)) ^ ((yr >> 1) & 3u)) << 4),
+                              P[0], P[1], P[2], P[3]);
+          }
+          fence_proxy_async_smem();  // the tile is read by the TMA store
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_y, ytile, gc0, t0);
+            bulk_commit_group();
+          }
+          ++n_ystores;
+        }
+      } else {
+        // SwiGLU: rows alternate gate (even lane) and up (odd lane)
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) {
+          const int j = half + 2 * i;
+          uint32_t a[32], l[32];
+          tmem_ld32(tmem + kColAcc + (uint32_t)(32 * j) + lane_off, a);
+          if (p.r > 0) tmem_ld32(tmem + kColLr + (uint32_t)(32 * j) + lane_off, l);
+          const int t0 = tm * TK + 32 * j;
+          const float sx_l = sx_pre[i][0];
+          tmem_ld_wait();
+          for (int c = c_lo; c < c_hi; ++c) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.part + (size_t)c * kCh * TK);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const uint4 x = ld_cg_v4(src + (j * 8 + v) * kCh + row);
+              a[4 * v] += x.x;
+              a[4 * v + 1] += x.y;
+              a[4 * v + 2] += x.z;
+              a[4 * v + 3] += x.w;
+            }
+          }
+          // y = s_x s_w acc + bf16(X L1) L2^T per element, then for each pair
+          // of tokens (2i, 2i+1) one shuffle gives the even lane (g, u) of
+          // token 2i and the odd lane those of token 2i+1, so every lane
+          // computes 16 of the warp's 16 x 32 outputs; silu(g) = g / (1 +
+          // e^-g) with the fast exponential and division (relative error
+          // ~1e-6, far below the bf16 output's 2^-9)
           float y[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            y[e] = dequant(e);
-            add_lowrank(y[e], e);
+            const float sx = __shfl_sync(0xffffffffu, sx_l, e);
+            y[e] = sx * sw * (float)(((int)a[e]) >> 4);
+            if (p.r > 0) y[e] += __uint_as_float(l[e]);
           }
           const bool odd = lane & 1;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float other = __shfl_xor_sync(0xffffffffu, odd ? y[2 * i] : y[2 * i + 1], 1);
-            const float g = odd ? other : y[2 * i];
-            const float u = odd ? y[2 * i + 1] : other;
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const float other = __shfl_xor_sync(0xffffffffu, odd ? y[2 * i2] : y[2 * i2 + 1], 1);
+            const float g = odd ? other : y[2 * i2];
+            const float u = odd ? y[2 * i2 + 1] : other;
             const __nv_bfloat16 h = __float2bfloat16_rn(__fdividef(g, 1.f + __expf(-g)) * u);
-            const int e = 2 * i + (odd ? 1 : 0);  // this lane's token
+            const int e = 2 * i2 + (odd ? 1 : 0);  // this lane's token
             asm volatile("st.shared.b16 [%0], %1;" ::"r"(ybuf + (uint32_t)e * L::kYRow + (uint32_t)(lane & ~1)),
                          "h"(*reinterpret_cast<const unsigned short*>(&h))
                          : "memory");
@@ -536,8 +637,8 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
             if (t < p.M && c < n_out)
               *reinterpret_cast<uint4*>(p.Y + (size_t)t * n_out + c) = v;
           }
+          __syncwarp();
         }
-        __syncwarp();
       }
       // the partials are consumed: clear their flags for the next launch
       if (lane == 0)
@@ -547,6 +648,7 @@ __global__ void __launch_bounds__(kThreadsA8, 1)
     }
   }
 
+  if (EPI != kEpiSwiglu && warp >= 2 && lane == 0) bulk_wait_all();  // Y tiles written
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -585,6 +687,11 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
     map_xb = map_t;  // never read
     map_l2 = map_t;
   }
+  CUtensorMap map_y = map_t;  // SwiGLU stores Y itself
+  if (EPI != kEpiSwiglu &&
+      !encode_tiled_2d(&map_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.Y, (uint64_t)a.N, (uint64_t)a.M,
+                       (uint64_t)a.N * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    return cudaErrorInvalidValue;
   // stream-K (see the schedule note at the top) where tile-by-tile CTAs
   // would leave much of their last wave idle: the waves' useful fraction
   // tiles / (G ceil(tiles / G)) below 0.85.  Above it the tile schedule was
@@ -618,7 +725,8 @@ cudaError_t launch_gemm_a8_tk(const GemmA8Args& a, A8Params p, cudaStream_t stre
   attr[0].val.programmaticStreamSerializationAllowed = tuning().pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel<TK, EPI>, map_t, map_w, map_xb, map_l2, p);
+  return cudaLaunchKernelEx(&cfg, w4a4_lr_gemm_a8_kernel<TK, EPI>, map_t, map_w, map_xb, map_l2, map_y,
+                            p);
 }
 
 }  // namespace
