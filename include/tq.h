@@ -150,8 +150,9 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  *   Y = bf16( s_x s_w (Q4(X H) . Wq) + bf16(X L1) L2 )
  *
  * i.e. tq_quantize_act followed by tq_w4a4_lr_gemm, with the same codes,
- * scales and tolerances.  At decode sizes (M <= 16, r in {0, 16, 32},
- * K % 256 == 0, K <= 4096, had_block <= 256) it runs as ONE kernel
+ * scales and tolerances.  At decode sizes (M <= 16, r in {0, 16, 32, 64},
+ * K % 256 == 0, K <= 4096, K / 256 dividing 16 at rank 64, had_block <=
+ * 256) it runs as ONE kernel
  * (TwinQuant notes section 04.C: the residual GEMM quantizes activations
  * concurrently and both paths share one epilogue): a thread-block cluster
  * of K / 256 CTAs per group of output channels, each CTA rotating its
@@ -160,7 +161,8 @@ TQ_API int tq_w4a4_lr_gemm(const uint8_t* Xq, const float* s_x,
  * X L1 partials and the split-K sums in distributed shared memory, and
  * feeding the codes to tcgen05 integer MMAs whose int4 weights were
  * requested and expanded into tensor memory before the kernel waited on
- * its predecessor.  Two such CTAs (two consecutive layers) share an SM.  For M > 128 with had_block <= 128 it runs
+ * its predecessor.  Two such CTAs (two consecutive layers) share an SM.
+ * For M > 128 with had_block <= 128 it runs
  * tq_quantize_act_i8 + tq_w4a4_lr_gemm_a8 (codes one per byte in the
  * workspace).  Other shapes run tq_quantize_act + tq_w4a4_lr_gemm, keeping
  * Xq, s_x and XL1 in the workspace.
@@ -453,7 +455,7 @@ TQ_API int tq_debug_noalloc_set_status(int status);
 
 /*
  * tq_debug_w4a4_lr_layer_decode -- test hook: the one-kernel decode layer of
- * tq_w4a4_lr_layer (M <= 16, r in {0, 16, 32}, K % 256 == 0, K <= 4096,
+ * tq_w4a4_lr_layer (M <= 16, r in {0, 16, 32, 64}, K % 256 == 0, K <= 4096,
  * had_block <= 256), also writing what it computes on the way: the
  * activation codes `codes` [M][K] int8 (RoundClip of X H per token), the
  * scales `s_x` [M] fp32 and the integer sums `acc` [M][N] int32

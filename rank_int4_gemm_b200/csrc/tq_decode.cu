@@ -64,7 +64,7 @@ constexpr int kSlice = 256;      // columns of K per CTA (two 128-column k-block
 constexpr int kMaxC = 16;        // cluster size limit: K <= 4096
 constexpr int kMaxT = 4;         // 128-channel tiles per CTA
 constexpr int kTmemTiles = 3;    // tiles whose expanded weights live in TMEM
-constexpr int kMaxR = 32;        // low-rank width handled here
+constexpr int kMaxR = 64;        // low-rank width handled here (0, 16, 32 or 64)
 constexpr int kWorkers = 256;    // warps 0-7
 constexpr int kCtrlWarp = 8;
 constexpr int kThreads = kWorkers + 32;
@@ -86,8 +86,10 @@ struct DecodeParams {
   float scale_mul;           // 1 / (7 sqrt(b))
 };
 
-// Shared-memory map (offsets from the 1024-aligned base).
+// Shared-memory map (offsets from the 1024-aligned base), for rank R.
+template <int R>
 struct Sm {
+  static constexpr int kRr = R > 16 ? R : 16;                 // L1^T rows staged
   static constexpr uint32_t kWTile = 128 * 128;               // packed tile [128][128 B], SW128
   static constexpr uint32_t kW = 0;                           // [T] packed tiles
   static constexpr uint32_t kA3 = 0;                          // tile 3 int8 [2 k-blocks][128][128 B]
@@ -96,28 +98,47 @@ struct Sm {
   static constexpr uint32_t kKRecvMax = 17 * 1024;
   static constexpr uint32_t kX = 64 * 1024;                   // X [4 chunks of 64 cols][16][128 B]
   static constexpr uint32_t kXChunk = kMT * 128;
-  static constexpr uint32_t kL1 = kX + 4 * kXChunk;           // L1^T [4 chunks][32][128 B]
-  static constexpr uint32_t kL1Chunk = kMaxR * 128;
-  static constexpr uint32_t kB = kL1 + 4 * kL1Chunk;          // codes [2 k-blocks][16][128 B]
+  static constexpr uint32_t kL1 = kX + 4 * kXChunk;           // L1^T [4 chunks][R][128 B]
+  static constexpr uint32_t kL1Chunk = kRr * 128;
+  // rank 64: chunk 3 of L1^T goes to the weight staging's tail, free once
+  // the weights are expanded (above the split-K area), so that two CTAs
+  // still share an SM
+  static constexpr int kL1Here = R == 64 ? 3 : 4;
+  static constexpr uint32_t kL1Hi = 50 * 1024;
+  static constexpr uint32_t kB = kL1 + kL1Here * kL1Chunk;    // codes [2 k-blocks][16][128 B]
   static constexpr uint32_t kBBlock = kMT * 128;
   static constexpr uint32_t kAmax = kB + 2 * kBBlock;         // [C][16] fp32
-  static constexpr uint32_t kXl1Recv = kAmax + kMaxC * kMT * 4;  // [C][tpo][r] fp32
-  static constexpr uint32_t kXl1Part = kXl1Recv + 4096;       // [KP][16][r] fp32
+  // [C][tpo][r] fp32: C ceil(16 / C) <= 30 token slots (C = 15); rank 64
+  // takes only clusters that divide 16 (16 slots)
+  static constexpr uint32_t kXl1Recv = kAmax + kMaxC * kMT * 4;
+  static constexpr uint32_t kXl1RecvBytes = 4096;
+  static constexpr uint32_t kXl1Part = kXl1Recv + kXl1RecvBytes;  // [KP][16][r] fp32
   static constexpr uint32_t kXl1B = kXl1Part + 4096;          // bf16 X L1 [16][r]
-  static constexpr uint32_t kSx = kXl1B + kMT * kMaxR * 2;    // s_x [16], partial absmax [16]
+  static constexpr uint32_t kSx = kXl1B + kMT * kRr * 2;      // s_x [16], partial absmax [16]
   static constexpr uint32_t kBar = kSx + 2 * kMT * 4;
   static constexpr uint32_t kNumBars = 12;
   static constexpr uint32_t kMisc = kBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;
+  static_assert((R == 64 ? 16 : 30) * kRr * 4 <= kXl1RecvBytes &&
+                    (8 / (kRr / 8 > 8 ? 8 : kRr / 8)) * kMT * kRr * 4 <= 4096,
+                "X L1 exchange buffers");
+  static_assert(R != 64 || (kL1Hi >= kKRecv + kKRecvMax && kL1Hi + kL1Chunk <= kX &&
+                            kL1Hi % 1024 == 0),
+                "L1^T chunk 3 between the split-K area and X");
+  static_assert(kKRecv + kKRecvMax <= kX, "split-K area inside the weight staging");
+  static_assert(kA3 + 2 * kA3Block <= kKRecv, "tile 3 below the split-K area");
+  static_assert(kX % 1024 == 0 && kL1 % 1024 == 0 && kB % 1024 == 0 && kXChunk % 1024 == 0 &&
+                    kL1Chunk % 1024 == 0 && kBBlock % 1024 == 0,
+                "1024-byte aligned swizzled tiles");
 };
-static_assert(Sm::kKRecv + Sm::kKRecvMax <= Sm::kX, "split-K area inside the weight staging");
-static_assert(Sm::kA3 + 2 * Sm::kA3Block <= Sm::kKRecv, "tile 3 below the split-K area");
-static_assert(Sm::kX % 1024 == 0 && Sm::kL1 % 1024 == 0 && Sm::kB % 1024 == 0 &&
-                  Sm::kXChunk % 1024 == 0 && Sm::kL1Chunk % 1024 == 0 && Sm::kBBlock % 1024 == 0,
-              "1024-byte aligned swizzled tiles");
-// two CTAs per SM: 228 KB of shared memory per SM, 1 KB reserved per CTA
-static_assert(2 * (Sm::kAlloc + 1024) <= 228 * 1024, "two CTAs per SM");
+// two CTAs per SM (228 KB of shared memory per SM, 1 KB reserved per CTA):
+// the second slot of an SM takes the next layer's CTA (one CTA per SM
+// measured 17.5 against 10.6 us per layer at rank 32)
+static_assert(2 * (Sm<32>::kAlloc + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(2 * (Sm<64>::kAlloc + 1024) <= 228 * 1024, "two CTAs per SM at rank 64");
+template <int R>
+constexpr int kCtasPerSm = 2;
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -191,16 +212,17 @@ __device__ __forceinline__ void expand16(uint4 w, uint4& lo, uint4& hi) {
 }
 
 template <int R>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     w4a4_lr_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                           const __grid_constant__ CUtensorMap map_x,
                           const __grid_constant__ CUtensorMap map_l1, const DecodeParams p) {
+  using S = Sm<R>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* smem = smem_raw + (base - raw_addr);
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Sm::kBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kBar);
   uint64_t* w_full = bars + 0;       // weight tiles (TMA)
   uint64_t* x_full = bars + 1;       // X slice (TMA)
   uint64_t* l1_full = bars + 2;      // L1^T slice (TMA)
@@ -210,9 +232,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint64_t* codes_ready = bars + 6;  // workers: weights in TMEM / smem, codes in smem
   uint64_t* part_bar = bars + 7;     // split-K sums of owned channels (st.async)
   uint64_t* acc_full = bars + 8;     // [kMaxT]: tile j's MMAs done (commit)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Sm::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Sm::kMisc + 4);
-  int* verdict = reinterpret_cast<int*>(smem + Sm::kMisc + 8);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kMisc + 4);
+  int* verdict = reinterpret_cast<int*>(smem + S::kMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -252,15 +274,15 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_prefetch_desc(&map_x);
     const uint64_t pol_w = policy_evict_first();
     // weights and L1^T never depend on the preceding kernel: requested now
-    mbar_arrive_expect_tx(w_full, (uint32_t)(t_valid * Sm::kWTile));
+    mbar_arrive_expect_tx(w_full, (uint32_t)(t_valid * S::kWTile));
     for (int j = 0; j < t_valid; ++j)
-      tma_load_2d(smem + Sm::kW + j * Sm::kWTile, &map_w, w_full, kbase / 2, n0 + 128 * j, pol_w);
+      tma_load_2d(smem + S::kW + j * S::kWTile, &map_w, w_full, kbase / 2, n0 + 128 * j, pol_w);
     if (r > 0) {
       tma_prefetch_desc(&map_l1);
       const uint64_t pol_l = policy_evict_last();  // every group reads the same L1^T
       mbar_arrive_expect_tx(l1_full, (uint32_t)(4 * r * 128));
-      for (int cc = 0; cc < 4; ++cc)
-        tma_load_2d(smem + Sm::kL1 + cc * Sm::kL1Chunk, &map_l1, l1_full, kbase + 64 * cc, 0,
+      for (int cc = 0; cc < S::kL1Here; ++cc)
+        tma_load_2d(smem + S::kL1 + cc * S::kL1Chunk, &map_l1, l1_full, kbase + 64 * cc, 0,
                     pol_l);
     }
   }
@@ -279,10 +301,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ============================================================ control
     if (lane == 0) {
       pdl_wait();  // X comes from the preceding kernel
-      mbar_arrive_expect_tx(x_full, 4 * Sm::kXChunk);
+      mbar_arrive_expect_tx(x_full, 4 * S::kXChunk);
       const uint64_t pol_x = policy_evict_first();
       for (int cc = 0; cc < 4; ++cc)
-        tma_load_2d(smem + Sm::kX + cc * Sm::kXChunk, &map_x, x_full, kbase + 64 * cc, 0, pol_x);
+        tma_load_2d(smem + S::kX + cc * S::kXChunk, &map_x, x_full, kbase + 64 * cc, 0, pol_x);
       const bool ok = mbar_wait(codes_ready, 0u, p.status, abort_flag) && !*abort_flag;
       tc_fence_after();
       // tile by tile (measured faster than interleaving the tiles'
@@ -292,8 +314,8 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (ok && j < t_valid) {
 #pragma unroll
           for (int kb = 0; kb < 2; ++kb) {
-            const uint64_t db = sdesc_sw128(base + Sm::kB + (uint32_t)kb * Sm::kBBlock);
-            const uint64_t da = sdesc_sw128(base + Sm::kA3 + (uint32_t)kb * Sm::kA3Block);
+            const uint64_t db = sdesc_sw128(base + S::kB + (uint32_t)kb * S::kBBlock);
+            const uint64_t da = sdesc_sw128(base + S::kA3 + (uint32_t)kb * S::kA3Block);
             const uint32_t d = tmem + kColAcc + 16u * (uint32_t)j;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
@@ -329,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int jj = 0; jj < 2; ++jj) {
         const int j = h + 2 * jj;
         if (j >= t_valid) continue;
-        const uint32_t src = base + Sm::kW + (uint32_t)j * Sm::kWTile;
+        const uint32_t src = base + S::kW + (uint32_t)j * S::kWTile;
         if (j < kTmemTiles) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
@@ -351,13 +373,21 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
     bar_sync_workers();  // tiles 0 and 1 are read: their staging may be overwritten
+    if constexpr (S::kL1Here < 4) {
+      // the packed tiles 2 and 3 are read too: L1^T chunk 3 into their tail
+      // (its bytes were counted on l1_full with the others)
+      if (tid == 0) {
+        fence_proxy_async_smem();
+        tma_load_2d(smem + S::kL1Hi, &map_l1, l1_full, kbase + 192, 0, policy_evict_last());
+      }
+    }
     if (ok && h == 1 && t_valid > kTmemTiles) {
       // tile 3: packed chunk c -> int8 chunks 2 (c % 4), +1 of k-block c / 4
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint4 lo, hi;
         expand16(t3[c], lo, hi);
-        const uint32_t dst = base + Sm::kA3 + (uint32_t)(c >> 2) * Sm::kA3Block;
+        const uint32_t dst = base + S::kA3 + (uint32_t)(c >> 2) * S::kA3Block;
         sts128(dst + sw128_offset((uint32_t)row, (uint32_t)(2 * (c & 3))), lo);
         sts128(dst + sw128_offset((uint32_t)row, (uint32_t)(2 * (c & 3) + 1)), hi);
       }
@@ -371,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       const int t = warp + 8 * tt;
-      const uint4 u = lds128(base + Sm::kX + (uint32_t)(lane >> 3) * Sm::kXChunk +
+      const uint4 u = lds128(base + S::kX + (uint32_t)(lane >> 3) * S::kXChunk +
                              sw128_offset((uint32_t)t, (uint32_t)(lane & 7)));
       const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -397,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       am_part[0] = fmaxf(am_part[0], __shfl_xor_sync(0xffffffffu, am_part[0], o));
       am_part[1] = fmaxf(am_part[1], __shfl_xor_sync(0xffffffffu, am_part[1], o));
     }
-    const uint32_t amax_stage = base + Sm::kSx + kMT * 4;  // this CTA's partials [16]
+    const uint32_t amax_stage = base + S::kSx + kMT * 4;  // this CTA's partials [16]
     if (lane == 0) {
       stsf(amax_stage + (uint32_t)(warp * 4), am_part[0]);
       stsf(amax_stage + (uint32_t)((warp + 8) * 4), am_part[1]);
@@ -406,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     bar_sync_workers();
     if (ok && tid < C * 4) {  // peer tid / 4 gets floats 4 (tid % 4) .. +3
       const uint32_t z = (uint32_t)(tid >> 2), qq = (uint32_t)(tid & 3);
-      st_async_v4(dsmem_map(base + Sm::kAmax + (crank * kMT + 4u * qq) * 4u, z),
+      st_async_v4(dsmem_map(base + S::kAmax + (crank * kMT + 4u * qq) * 4u, z),
                   lds128(amax_stage + 16u * qq), dsmem_map(smem_u32(amax_bar), z));
     }
 
@@ -418,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       float am = 0.f;
 #pragma unroll
       for (int z = 0; z < kMaxC; ++z)
-        if (z < C) am = fmaxf(am, ldsf(base + Sm::kAmax + (uint32_t)((z * kMT + t) * 4)));
+        if (z < C) am = fmaxf(am, ldsf(base + S::kAmax + (uint32_t)((z * kMT + t) * 4)));
       const CodeScale cs = code_scale(am);
       if (cs.pre != 1.f) {
 #pragma unroll
@@ -430,13 +460,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       const uint32_t lo = low_bytes4(cb[0], cb[1], cb[2], cb[3]);
       const uint32_t hi = low_bytes4(cb[4], cb[5], cb[6], cb[7]);
       // columns 8 lane .. +7: k-block lane / 16, byte (lane % 16) * 8 of the row
-      sts64(base + Sm::kB + (uint32_t)(lane >> 4) * Sm::kBBlock +
+      sts64(base + S::kB + (uint32_t)(lane >> 4) * S::kBBlock +
                 sw128_offset((uint32_t)t, (uint32_t)((lane & 15) >> 1)) + 8u * (uint32_t)(lane & 1),
             lo, hi);
       if (p.dbg_codes && t < p.M)
         *reinterpret_cast<uint2*>(p.dbg_codes + (size_t)t * p.K + kbase + 8 * lane) = make_uint2(lo, hi);
       if (lane == 0) {
-        stsf(base + Sm::kSx + (uint32_t)(t * 4), am * p.scale_mul);
+        stsf(base + S::kSx + (uint32_t)(t * 4), am * p.scale_mul);
         if (p.dbg_sx && crank == 0 && t < p.M) p.dbg_sx[t] = am * p.scale_mul;
       }
     }
@@ -447,30 +477,35 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ---- 4. X L1 partial over the slice (while the integer MMAs run) ->
     //         the owner of each token
     if constexpr (R > 0) {
-      constexpr int kNt = R / 8;             // 8-column tiles of the rank: 2 or 4
-      constexpr int kKP = 8 / kNt;           // k-parts: 4 or 2
+      constexpr int kNt = R / 8;             // 8-column tiles of the rank: 2, 4 or 8
+      constexpr int kKP = 8 / kNt;           // k-parts: 4, 2 or 1
       constexpr int kSteps = (kSlice / 16) / kKP;
+      constexpr int kGrp = kSteps < 8 ? kSteps : 8;  // operands held at once
       const bool l1_ok = workers_wait<false>(l1_full, p.status, abort_flag, verdict);
       ok = ok && l1_ok;
       const int nt = warp % kNt, kp = warp / kNt;
-      uint32_t a[kSteps][4], bb[kSteps][2];
-#pragma unroll
-      for (int s2 = 0; s2 < kSteps; ++s2) {
-        const int kk = (kp * kSteps + s2) * 16;
-        const int mat = lane >> 3, trow = (lane & 7) + (mat & 1) * 8;
-        const int ka = kk + (mat >> 1) * 8;
-        ldmatrix_x4(a[s2], base + Sm::kX + (uint32_t)(ka >> 6) * Sm::kXChunk +
-                               sw128_offset((uint32_t)trow, (uint32_t)((ka & 63) >> 3)));
-        const int l = lane & 15;
-        const int jr = nt * 8 + (l & 7), kb2 = kk + (l >> 3) * 8;
-        ldmatrix_x2(bb[s2], base + Sm::kL1 + (uint32_t)(kb2 >> 6) * Sm::kL1Chunk +
-                                sw128_offset((uint32_t)jr, (uint32_t)((kb2 & 63) >> 3)));
-      }
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int s2 = 0; s2 < kSteps; ++s2) mma_16816(acc[s2 & 1], a[s2], bb[s2]);
+      for (int g0 = 0; g0 < kSteps; g0 += kGrp) {
+        uint32_t a[kGrp][4], bb[kGrp][2];
+#pragma unroll
+        for (int s3 = 0; s3 < kGrp; ++s3) {
+          const int kk = (kp * kSteps + g0 + s3) * 16;
+          const int mat = lane >> 3, trow = (lane & 7) + (mat & 1) * 8;
+          const int ka = kk + (mat >> 1) * 8;
+          ldmatrix_x4(a[s3], base + S::kX + (uint32_t)(ka >> 6) * S::kXChunk +
+                                 sw128_offset((uint32_t)trow, (uint32_t)((ka & 63) >> 3)));
+          const int l = lane & 15;
+          const int jr = nt * 8 + (l & 7), kb2 = kk + (l >> 3) * 8;
+          const int l1c = kb2 >> 6;  // 64-column chunk of the slice
+          ldmatrix_x2(bb[s3], base + ((l1c < S::kL1Here) ? S::kL1 + (uint32_t)l1c * S::kL1Chunk : S::kL1Hi) +
+                                  sw128_offset((uint32_t)jr, (uint32_t)((kb2 & 63) >> 3)));
+        }
+#pragma unroll
+        for (int s3 = 0; s3 < kGrp; ++s3) mma_16816(acc[(g0 + s3) & 1], a[s3], bb[s3]);
+      }
       // C fragment: tokens lane / 4 and lane / 4 + 8, columns nt 8 + 2 (lane % 4), +1
-      const uint32_t part = base + Sm::kXl1Part;
+      const uint32_t part = base + S::kXl1Part;
       const int trw = lane >> 2, cc = nt * 8 + 2 * (lane & 3);
       stsf(part + (uint32_t)(((kp * kMT + trw) * R + cc) * 4), acc[0][0] + acc[1][0]);
       stsf(part + (uint32_t)(((kp * kMT + trw) * R + cc + 1) * 4), acc[0][1] + acc[1][1]);
@@ -496,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t owner = (uint32_t)(t % C);
           const uint32_t slot = (crank * (uint32_t)tpo + (uint32_t)(t / C)) * (uint32_t)R + 4u * c4;
           if (ok)
-            st_async_v4(dsmem_map(base + Sm::kXl1Recv + slot * 4u, owner),
+            st_async_v4(dsmem_map(base + S::kXl1Recv + slot * 4u, owner),
                         make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]),
                                    __float_as_uint(f[2]), __float_as_uint(f[3])),
                         dsmem_map(smem_u32(xl1p_bar), owner));
@@ -517,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int z = 0; z < kMaxC; ++z) {
             if (z < C) {
-              const uint32_t src = base + Sm::kXl1Recv + (uint32_t)(((z * tpo + li) * R + 8 * c8) * 4);
+              const uint32_t src = base + S::kXl1Recv + (uint32_t)(((z * tpo + li) * R + 8 * c8) * 4);
               const uint4 a0 = lds128(src), b0 = lds128(src + 16);
               f[0] += __uint_as_float(a0.x); f[1] += __uint_as_float(a0.y);
               f[2] += __uint_as_float(a0.z); f[3] += __uint_as_float(a0.w);
@@ -529,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                                        bf16x2(f[6], f[7]));
           if (ok && got)
             for (int z = 0; z < C; ++z)
-              st_async_v4(dsmem_map(base + Sm::kXl1B + (uint32_t)((t * R + 8 * c8) * 2), (uint32_t)z),
+              st_async_v4(dsmem_map(base + S::kXl1B + (uint32_t)((t * R + 8 * c8) * 2), (uint32_t)z),
                           val, dsmem_map(smem_u32(xl1b_bar), (uint32_t)z));
         }
       }
@@ -540,14 +575,19 @@ __global__ void __launch_bounds__(kThreads, 2)
     const bool fast_epi = per <= 64 && (kWorkers % per) == 0;
     const int c_own = fast_epi ? tid % per : 0;
     const int n_own = n0 + own_lo + c_own;
+    // (rank 64 loads its L2^T row in the epilogue: held through the MMAs
+    // its 32 registers would spill)
+    constexpr int kPre = (R > 0 && R <= 32) ? R / 8 : 1;
     float sw_own = 0.f;
-    uint4 l2_own[R > 0 ? R / 8 : 1];
+    uint4 l2_own[kPre];
 #pragma unroll
-    for (int i = 0; i < (R > 0 ? R / 8 : 1); ++i) l2_own[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < kPre; ++i) l2_own[i] = make_uint4(0u, 0u, 0u, 0u);
     if (fast_epi && tid < 4 * per && n_own < p.N) {
       sw_own = ldg_nc_f32(p.s_w + n_own);
+      if constexpr (R > 0 && R <= 32) {
 #pragma unroll
-      for (int i = 0; i < R / 8; ++i) l2_own[i] = ldg_nc_v4(p.L2t + (size_t)n_own * R + 8 * i);
+        for (int i = 0; i < R / 8; ++i) l2_own[i] = ldg_nc_v4(p.L2t + (size_t)n_own * R + 8 * i);
+      }
     }
 
     // ---- 5. accumulators -> the channel's owner (int16 sums of this slice),
@@ -577,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int rg = 128 * j + row;             // channel within the group
       const int o = (rg * C) / G;               // its owner
       const int lo_o = (o * G + C - 1) / C;
-      const uint32_t dst = dsmem_map(base + Sm::kKRecv +
+      const uint32_t dst = dsmem_map(base + S::kKRecv +
                                          (uint32_t)(((int)crank * per_max + (rg - lo_o)) * kMT * 2),
                                      (uint32_t)o);
       const uint32_t rb = dsmem_map(smem_u32(part_bar), (uint32_t)o);
@@ -605,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int z = 0; z < kMaxC; ++z) {
           u[z] = make_uint2(0u, 0u);
           if (z < C) {
-            const uint32_t ad = base + Sm::kKRecv + (uint32_t)(((z * per_max + c) * kMT + 4 * tq4) * 2);
+            const uint32_t ad = base + S::kKRecv + (uint32_t)(((z * per_max + c) * kMT + 4 * tq4) * 2);
             asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(u[z].x), "=r"(u[z].y) : "r"(ad));
           }
         }
@@ -618,10 +658,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         float sw = sw_own;
         uint4 l2[R > 0 ? R / 8 : 1];
+        if constexpr (R > 0 && R <= 32) {
 #pragma unroll
-        for (int i = 0; i < (R > 0 ? R / 8 : 1); ++i) l2[i] = l2_own[i];
-        if (!fast_epi) {
-          sw = ldg_nc_f32(p.s_w + n);
+          for (int i = 0; i < R / 8; ++i) l2[i] = l2_own[i];
+        }
+        if (!fast_epi) sw = ldg_nc_f32(p.s_w + n);
+        if (!fast_epi || R > 32) {
 #pragma unroll
           for (int i = 0; i < R / 8; ++i) l2[i] = ldg_nc_v4(p.L2t + (size_t)n * R + 8 * i);
         }
@@ -631,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           if (t >= p.M) break;
           float lr = 0.f;
           if constexpr (R > 0) {
-            const uint32_t xr = base + Sm::kXl1B + (uint32_t)(t * R * 2);
+            const uint32_t xr = base + S::kXl1B + (uint32_t)(t * R * 2);
 #pragma unroll
             for (int i = 0; i < R / 8; ++i) {
               const uint4 xa = lds128(xr + 16u * (uint32_t)i);
@@ -644,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 2)
               }
             }
           }
-          const float s_x = ldsf(base + Sm::kSx + (uint32_t)(t * 4));
+          const float s_x = ldsf(base + S::kSx + (uint32_t)(t * 4));
           p.Y[(size_t)t * p.N + n] = __float2bfloat16_rn(sw * s_x * (float)acc4[e4] + lr);
           if (p.dbg_acc) p.dbg_acc[(size_t)t * p.N + n] = acc4[e4];
         }
@@ -670,8 +712,9 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 bool layer_decode2_supported(int M, int N, int K, int r, int had_block) {
   (void)N;
-  return M >= 1 && M <= kMT && (r == 0 || r == 16 || r == 32) && K % kSlice == 0 &&
-         K / kSlice <= kMaxC && had_block >= 1 && had_block <= kSlice;
+  // rank 64: clusters that divide 16 (its X L1 exchange holds 16 token slots)
+  return M >= 1 && M <= kMT && (r == 0 || r == 16 || r == 32 || (r == 64 && K > 0 && K % kSlice == 0 && 16 % (K / kSlice) == 0)) &&
+         K % kSlice == 0 && K / kSlice <= kMaxC && had_block >= 1 && had_block <= kSlice;
 }
 
 cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream, int8_t* dbg_codes,
@@ -717,16 +760,17 @@ cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream, int8_t
     map_l1 = map_x;  // never read
   }
   using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, DecodeParams);
-  const int ri = a.r / 16;  // 0, 1, 2
-  const KernelFn fns[3] = {w4a4_lr_decode_kernel<0>, w4a4_lr_decode_kernel<16>,
-                           w4a4_lr_decode_kernel<32>};
+  const int ri = a.r == 64 ? 3 : a.r / 16;  // 0, 1, 2, 3
+  const KernelFn fns[4] = {w4a4_lr_decode_kernel<0>, w4a4_lr_decode_kernel<16>,
+                           w4a4_lr_decode_kernel<32>, w4a4_lr_decode_kernel<64>};
+  const uint32_t allocs[4] = {Sm<0>::kAlloc, Sm<16>::kAlloc, Sm<32>::kAlloc, Sm<64>::kAlloc};
   const KernelFn fn = fns[ri];
-  static uint64_t attr_set[3] = {0, 0, 0};
+  static uint64_t attr_set[4] = {0, 0, 0, 0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set[ri] >> dev & 1u)) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Sm::kAlloc);
+                                         (int)allocs[ri]);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
@@ -735,7 +779,7 @@ cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream, int8_t
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.C, groups, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = Sm::kAlloc;
+  cfg.dynamicSmemBytes = allocs[ri];
   cfg.stream = stream;
   cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

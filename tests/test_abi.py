@@ -108,7 +108,7 @@ def test_no_device_is_reported(lib):
 
 def test_layer_path_routing():
     """tq_layer_path is a host query (runs without a GPU): the one-kernel
-    decode layer where its limits hold (M <= 16, r <= 32, K % 256 == 0,
+    decode layer where its limits hold (M <= 16, r in {0, 16, 32, 64}, K % 256 == 0,
     K <= 4096, Hadamard block <= 256), int8 codes for M > 128 with block
     <= 128, packed codes otherwise; rejected shapes raise."""
     import rank_int4_gemm_b200 as tq
@@ -117,7 +117,10 @@ def test_layer_path_routing():
     assert p(1, 4096, 4096, 0, 128) == "fused"
     assert p(16, 4096, 4096, 32, 1) == "fused"
     assert p(17, 4096, 4096, 32, 128) == "codes_packed"
-    assert p(16, 4096, 4096, 64, 128) == "codes_packed"
+    assert p(16, 4096, 4096, 64, 128) == "fused"
+    assert p(16, 4096, 4096, 48, 128) == "codes_packed"   # ranks 0, 16, 32, 64 only
+    assert p(16, 4096, 3840, 64, 128) == "codes_packed"   # rank 64: clusters dividing 16
+    assert p(16, 4096, 3840, 32, 128) == "fused"
     assert p(16, 8192, 4096, 32, 128) == "fused"        # N does not limit it
     assert p(16, 4096, 4608, 32, 128) == "codes_packed"  # K > 4096
     assert p(16, 4096, 384, 16, 128) == "codes_packed"   # K % 256 != 0

@@ -43,6 +43,11 @@ CASES = [
     ("block2", 4, 1024, 256, 16, 2),
     ("no_rotation", 2, 1024, 128, 32, 1),
     ("wide_n", 16, 1024, 8192, 32, 128),
+    # rank 64 (one CTA per SM)
+    ("rank64_m16", 16, 4096, 4096, 64, 128),
+    ("rank64_cluster8", 5, 2048, 1024, 64, 128),
+    ("rank64_cluster4_ragged", 11, 1024, 136, 64, 64),
+    ("rank64_m1_block256", 1, 2048, 640, 64, 256),
 ]
 
 

@@ -18,7 +18,7 @@ def tq(cuda_ok):
 
 
 CASES = [
-    # name, M, K, N, r, b      (fused: M<=16, r<=32, K%512==0, K<=4096, b<=128)
+    # name, M, K, N, r, b      (fused: M<=16, r in {0,16,32,64}, K%256==0, K<=4096, b<=256)
     ("decode_m1", 1, 4096, 4096, 32, 128),
     ("decode_m3", 3, 4096, 4096, 32, 128),
     ("decode_m16", 16, 4096, 4096, 32, 128),
