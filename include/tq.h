@@ -271,10 +271,13 @@ TQ_API int tq_pack_shared_input(int n, const uint8_t* const* Wq, const float* co
  *                         registers before the butterflies).
  * tq_w4a4_lr_layer_rht -- tq_w4a4_lr_layer with D H (weights from
  *                         tq_pack_weight_rht with the same mask): the
- *                         one-kernel decode layer where it applies, else
+ *                         one-kernel decode layer where it applies; for
+ *                         M > 128 with had_block <= 128 the butterfly
+ *                         kernel writing one code per byte and bf16(X L1),
+ *                         then tq_w4a4_lr_gemm_a8 (the tensor-core
+ *                         activation kernel takes no signs); else
  *                         tq_quantize_act_rht + tq_w4a4_lr_gemm (packed
- *                         codes; the tensor-core activation kernel of the
- *                         int8-code path takes no signs).
+ *                         codes).  tq_layer_path reports the same choice.
  * Arguments and limits as the plain calls; `signs` 16-byte aligned.
  */
 TQ_API int tq_pack_weight_rht(const float* Rt, int N, int K, int had_block,

@@ -35,9 +35,11 @@ constexpr int kActThreads = 32 * kActWarps;
 struct ActParams {
   const __nv_bfloat16* X;
   const __nv_bfloat16* L1t;
-  uint8_t* Xq;
+  uint8_t* Xq;              // packed codes [M][K/2], or
+  int8_t* Xq8;              //   one code per byte [M][K] (when non-null)
   float* s_x;
-  float* XL1;
+  float* XL1;               // fp32 X L1 [M][r], or
+  __nv_bfloat16* XL1b;      //   bf16(X L1) (when non-null)
   const uint32_t* signs;  // randomized Hadamard sign mask [K / 32], or null
   int M, K, b, r;
   int passes_per_cta;  // P: warp passes of W = 32E columns in this CTA's slice
@@ -279,7 +281,8 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     if (my_row >= p.M) continue;  // warp-uniform
     const float am = amax_row[rr];
     const CodeScale cs = code_scale(am);
-    uint8_t* xrow = p.Xq + (size_t)my_row * (p.K / 2);
+    uint8_t* xrow = p.Xq8 ? nullptr : p.Xq + (size_t)my_row * (p.K / 2);
+    int8_t* xrow8 = p.Xq8 ? p.Xq8 + (size_t)my_row * p.K : nullptr;
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
@@ -292,7 +295,21 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
       uint32_t cb[E];
 #pragma unroll
       for (int i = 0; i < E; ++i) cb[i] = code_bits(v[i], cs.inv);
-      store_packed<E>(cb, xrow + (kbase + ps * W) / 2);
+      if (xrow8) {
+        // E consecutive codes, byte i the low byte of cb[i]
+        int8_t* dst = xrow8 + kbase + ps * W + lane * E;
+        if constexpr (E == 4) {
+          *reinterpret_cast<uint32_t*>(dst) = low_bytes4(cb[0], cb[1], cb[2], cb[3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < E; i += 8)
+            *reinterpret_cast<uint2*>(dst + i) =
+                make_uint2(low_bytes4(cb[i], cb[i + 1], cb[i + 2], cb[i + 3]),
+                           low_bytes4(cb[i + 4], cb[i + 5], cb[i + 6], cb[i + 7]));
+        }
+      } else {
+        store_packed<E>(cb, xrow + (kbase + ps * W) / 2);
+      }
     }
     if (crank == 0 && lane == 0) p.s_x[my_row] = am * p.scale_mul;
   }
@@ -307,7 +324,10 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
       if (row0 + rr >= p.M) continue;
       float v = 0.f;
       for (uint32_t c = 0; c < csize; ++c) v += recv[((int)c * kActRows + rr) * L.cols_max + cc];
-      p.XL1[(size_t)(row0 + rr) * p.r + lo + cc] = v;
+      if (p.XL1b)
+        p.XL1b[(size_t)(row0 + rr) * p.r + lo + cc] = __float2bfloat16_rn(v);
+      else
+        p.XL1[(size_t)(row0 + rr) * p.r + lo + cc] = v;
     }
   }
 }
@@ -549,6 +569,29 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   if (!signs && act_tc_supported(M, K, had_block, r))
     return launch_act_tc(X, M, K, had_block, L1t, r, Xq, nullptr, s_x, XL1, nullptr, stream);
   // Few token groups (decode): spread K over up to 16 CTAs of 256 columns.
+  const int groups = (M + kActRows - 1) / kActRows;
+  if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);
+  if (K % 512 == 0) return launch_act_e<16>(prm, 8, stream);
+  if (K % 256 == 0) return launch_act_e<8>(prm, 8, stream);
+  if (had_block <= 128) return launch_act_e<4>(prm, 8, stream);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_block,
+                                      const uint16_t* L1t, int r, int8_t* Xq8, float* s_x,
+                                      uint16_t* XL1b, cudaStream_t stream, const uint32_t* signs) {
+  ActParams prm{};
+  prm.X = reinterpret_cast<const __nv_bfloat16*>(X);
+  prm.L1t = reinterpret_cast<const __nv_bfloat16*>(L1t);
+  prm.Xq8 = Xq8;
+  prm.s_x = s_x;
+  prm.XL1b = reinterpret_cast<__nv_bfloat16*>(XL1b);
+  prm.M = M;
+  prm.K = K;
+  prm.b = had_block;
+  prm.r = r;
+  prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
+  prm.signs = signs;
   const int groups = (M + kActRows - 1) / kActRows;
   if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);
   if (K % 512 == 0) return launch_act_e<16>(prm, 8, stream);

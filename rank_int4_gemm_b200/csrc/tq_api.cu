@@ -277,13 +277,18 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
     return from_cuda(tq::launch_layer_decode2(a, st));
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (!signs && layer_uses_a8(M, r, had_block)) {
+  if (layer_uses_a8(M, r, had_block)) {
     int8_t* Xq8 = reinterpret_cast<int8_t*>(ws + 256);
     float* s_x8 = reinterpret_cast<float*>(ws + 256 + align256((size_t)M * K));
     uint16_t* XL1b =
         reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(s_x8) + align256((size_t)M * 4));
-    if (cudaError_t e = tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8, nullptr,
-                                          r > 0 ? XL1b : nullptr, st))
+    // the tensor-core activation kernel has one Hadamard operand for every
+    // column, so a sign mask takes the butterfly kernel (same int8 outputs)
+    if (cudaError_t e = signs ? tq::launch_quantize_act_bf_i8(X, M, K, had_block, L1t, r, Xq8,
+                                                              s_x8, r > 0 ? XL1b : nullptr, st,
+                                                              signs)
+                              : tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8,
+                                                  nullptr, r > 0 ? XL1b : nullptr, st))
       return from_cuda(e);
     tq::GemmA8Args a{};
     a.Xq8 = Xq8;

@@ -24,6 +24,13 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
                                 float* XL1, cudaStream_t stream, const uint32_t* signs = nullptr);
 
+// The butterfly activation kernel writing one code per byte and bf16(X L1)
+// (the int8-code GEMM's operands), with an optional sign mask.
+cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_block,
+                                      const uint16_t* L1t, int r, int8_t* Xq8, float* s_x,
+                                      uint16_t* XL1b, cudaStream_t stream,
+                                      const uint32_t* signs = nullptr);
+
 // Activation stage on tensor cores (many tokens): rotation and X L1 as MMAs.
 // Codes packed (Xq, [M][K/2]) or one int8 per code (Xq8, [M][K]); X L1 as
 // fp32 (XL1) and / or rounded to bf16 (XL1b), either may be null.

@@ -155,7 +155,8 @@ def test_signed_activation_codes_match_oracle(tq, M, b, r):
 
 @pytest.mark.gpu
 @pytest.mark.parametrize("M,K,N,r,b", [(16, 4096, 4096, 32, 128), (1, 4096, 1024, 16, 256),
-                                       (5, 1024, 520, 32, 64), (200, 2048, 512, 64, 128)])
+                                       (5, 1024, 520, 32, 64), (200, 2048, 512, 64, 128),
+                                       (600, 4096, 1024, 32, 128), (130, 1024, 264, 16, 256)])
 def test_signed_layer_matches_oracle(tq, M, K, N, r, b):
     sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=r, had_block=b)
     L = synth.make_layer(sh, seed=23, device="cuda" if K * N >= 1 << 22 else "cpu")
@@ -173,6 +174,26 @@ def test_signed_layer_matches_oracle(tq, M, K, N, r, b):
     fro, mx = check_y(Y.double().cpu().numpy(), y_reference(q, o, fx, qw, fw),
                       f"signed layer M={M} K={K} N={N}")
     print(f"FLIPS rht layer M={M} path={tq.tq_layer_path(M, N, K, r, b)}: fro={fro:.3e}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,K,N,b", [(300, 1024, 384, 128), (1000, 4096, 1024, 64)])
+def test_signed_layer_int8_path_equals_packed_path_at_rank0(tq, M, K, N, b):
+    # above 128 tokens the signed layer writes one code per byte from the
+    # butterfly kernel and runs the int8-code GEMM; at rank 0 its Y equals
+    # the packed codes of the same kernel through the packed-code GEMM bit for
+    # bit (same codes, exact integer sums, the same fp32 epilogue)
+    sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=0, had_block=b)
+    L = synth.make_layer(sh, seed=25, device="cuda")
+    sg = _dev_signs(K, M + 7)
+    X = L["X"].cuda()
+    Wq, s_w = tq.tq_pack_weight_rht(L["Rt"].cuda(), b, sg)
+    assert tq.tq_layer_path(M, N, K, 0, b) == "codes_i8"
+    Y = tq.tq_w4a4_lr_layer_rht(X, sg, None, Wq, s_w, None, b)
+    Xq, s_x, _ = tq.tq_quantize_act_rht(X, b, sg)
+    Y2 = tq.tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
 
 
 @pytest.mark.gpu
