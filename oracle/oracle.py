@@ -67,6 +67,8 @@ def signs_from_bits(bits, K: int) -> np.ndarray:
     transform from its bit mask: K / 32 little-endian uint32 words, bit
     (k % 32) of word k / 32 set where d_k = -1."""
     w = np.ascontiguousarray(np.asarray(bits, dtype=np.uint32))
+    if w.ndim == 2:  # n masks (composed transforms): rows of signs
+        return np.stack([signs_from_bits(row, K) for row in w])
     assert w.size * 32 >= K, (w.size, K)
     neg = np.unpackbits(w.view(np.uint8), bitorder="little")[:K]
     return np.where(neg == 1, -1.0, 1.0)
@@ -75,15 +77,25 @@ def signs_from_bits(bits, K: int) -> np.ndarray:
 def rotate(x, b: int, signs=None) -> np.ndarray:
     """Rows of x times diag(H_b, ..., H_b) (fp64); with `signs` (the +-1
     vector d), rows of x times D diag(H_b, ...): the randomized Hadamard
-    transform, signs first, then the Hadamard blocks."""
+    transform, signs first, then the Hadamard blocks.  `signs` of shape
+    (n, K) composes n randomized Hadamard transforms, the first row's
+    first: x D_1 H D_2 H ... D_n H."""
     x = _f64(x)
-    if signs is not None:
-        x = np.ascontiguousarray(x * np.asarray(signs, dtype=np.float64)[None, :])
     rows, K = x.shape
     assert K % b == 0
-    out = np.empty_like(x)
-    _load().orc_rotate(_ptr(x), rows, K, int(b), _ptr(out))
-    return out
+    if signs is None:
+        masks = [None]
+    else:
+        d = np.asarray(signs, dtype=np.float64)
+        masks = list(d) if d.ndim == 2 else [d]
+    for m in masks:
+        if m is not None:
+            assert m.shape == (K,)
+            x = np.ascontiguousarray(x * m[None, :])
+        out = np.empty_like(x)
+        _load().orc_rotate(_ptr(x), rows, K, int(b), _ptr(out))
+        x = out
+    return x
 
 
 def quantize_sym(v, qmax: int = 7):

@@ -225,3 +225,61 @@ def test_signed_entry_argument_checks():
     assert lib.tq_quantize_act_rht(P(F), 4, 256, 128, None, None, 0, P(F), P(F), None, None) == 1
     assert lib.tq_w4a4_lr_layer_rht(P(F), None, None, P(F), P(F), None, 4, 64, 256, 0, 128, P(F),
                                     P(F), ctypes.c_size_t(1 << 20), None) == 1
+
+
+# ------------------------------------------ composed randomized Hadamards
+
+def _mask(sgn):
+    return np.array([1.0 if c == "+" else -1.0 for c in sgn])
+
+
+def test_composed_hand_worked_examples():
+    path = os.path.join(os.path.dirname(__file__), "golden", "rht_composed_worked.txt")
+    for line in open(path).read().splitlines():
+        if line.startswith("#") or not line.strip():
+            continue
+        name, b, masks, x, want = [f.strip() for f in line.split("|")]
+        d = np.stack([_mask(m) for m in masks.split(";")])
+        x = np.array([float(v) for v in x.split(",")])[None, :]
+        got = oracle.rotate(x, int(b), signs=d)[0]
+        assert np.allclose(got, [float(v) for v in want.split(",")], rtol=0, atol=1e-14), name
+
+
+@pytest.mark.parametrize("b,n", [(2, 2), (16, 3), (128, 2)])
+def test_composed_rotation_is_the_product_of_single_transforms(b, n):
+    # against matrices built here from scipy's Hadamard: D_1 Hd D_2 Hd ...
+    from scipy.linalg import hadamard
+    K = 4 * b
+    rng = np.random.default_rng(b + n)
+    d = rng.choice([-1.0, 1.0], size=(n, K))
+    Hd = np.kron(np.eye(K // b), hadamard(b) / np.sqrt(b))
+    Q = np.eye(K)
+    for i in range(n):
+        Q = Q @ np.diag(d[i]) @ Hd
+    x = rng.normal(size=(5, K))
+    assert np.allclose(oracle.rotate(x, b, signs=d), x @ Q, rtol=0, atol=1e-12)
+    assert np.allclose(Q @ Q.T, np.eye(K), atol=1e-12)  # orthogonal
+    # the single-transform case of the same call
+    assert np.allclose(oracle.rotate(x, b, signs=d[:1]), oracle.rotate(x, b, signs=d[0]),
+                       rtol=0, atol=0)
+
+
+@pytest.mark.parametrize("b", [4, 128])
+def test_two_all_plus_masks_give_the_identity(b):
+    x = np.random.default_rng(b).normal(size=(3, 2 * b))
+    assert np.allclose(oracle.rotate(x, b, signs=np.ones((2, 2 * b))), x, rtol=0, atol=1e-12)
+
+
+def test_composed_eq3_invariance_and_bit_masks():
+    # (X Q)(Q^T W) = X W for the composed transform on both sides; masks as
+    # bit words decode row by row
+    rng = np.random.default_rng(7)
+    K, b = 256, 64
+    bits = rng.integers(0, 2**32, size=(3, K // 32), dtype=np.uint64).astype(np.uint32)
+    d = oracle.signs_from_bits(bits, K)
+    assert d.shape == (3, K)
+    for i in range(3):
+        assert np.array_equal(d[i], oracle.signs_from_bits(bits[i], K))
+    X, W = rng.normal(size=(4, K)), rng.normal(size=(6, K))
+    lhs = oracle.rotate(X, b, signs=d) @ oracle.rotate(W, b, signs=d).T
+    assert np.allclose(lhs, X @ W.T, rtol=0, atol=1e-10)
