@@ -291,6 +291,27 @@ TQ_API int tq_w4a4_lr_layer_rht(const uint16_t* X, const uint32_t* signs, const 
                                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Composed randomized Hadamard transforms (two make every coordinate's
+ * marginal near-Gaussian, three also decorrelate blocks of coordinates for
+ * vector quantization): x D_1 H D_2 H ... D_n H
+ * with n = n_rht in 1..3 masks, stored one after another in `signs`
+ * ([n_rht][K / 32] words, the first applied first); weights packed by
+ * tq_pack_weight_rhtn with the same masks.  The _rht calls above are
+ * n_rht = 1.  Same arguments, paths and limits otherwise.
+ */
+TQ_API int tq_pack_weight_rhtn(const float* Rt, int N, int K, int had_block,
+                               const uint32_t* signs, int n_rht, uint8_t* Wq, float* s_w,
+                               void* stream);
+TQ_API int tq_quantize_act_rhtn(const uint16_t* X, int M, int K, int had_block,
+                                const uint32_t* signs, int n_rht, const uint16_t* L1t, int r,
+                                uint8_t* Xq, float* s_x, float* XL1, void* stream);
+TQ_API int tq_w4a4_lr_layer_rhtn(const uint16_t* X, const uint32_t* signs, int n_rht,
+                                 const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
+                                 const uint16_t* L2t, int M, int N, int K, int r, int had_block,
+                                 uint16_t* Y, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/*
  * Per-token asymmetric activations (CoQuant Eq. (1) with a zero-point; the
  * protocol CoQuant follows quantizes activations per token asymmetrically):
  * for each token's rotated row v, z = min(v), s = (max(v) - min(v)) / 15,

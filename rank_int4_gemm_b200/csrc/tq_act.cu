@@ -40,7 +40,8 @@ struct ActParams {
   float* s_x;
   float* XL1;               // fp32 X L1 [M][r], or
   __nv_bfloat16* XL1b;      //   bf16(X L1) (when non-null)
-  const uint32_t* signs;  // randomized Hadamard sign mask [K / 32], or null
+  const uint32_t* signs;  // randomized Hadamard sign masks [n_rht][K / 32], or null
+  int n_rht;              // composed transforms (masks)
   int M, K, b, r;
   int passes_per_cta;  // P: warp passes of W = 32E columns in this CTA's slice
   int total_passes;    // K / W
@@ -164,8 +165,7 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
-      apply_signs<E>(v, p.signs, kbase + ps * W + lane * E);
-      fwht_warp<E>(v, p.b);
+      rotate_signed<E>(v, p.signs, p.n_rht, p.K / 32, kbase + ps * W + lane * E, p.b);
 #pragma unroll
       for (int i = 0; i < E; ++i) amax[t] = fmaxf(amax[t], fabsf(v[i]));
     }
@@ -286,8 +286,7 @@ __global__ void __launch_bounds__(kActThreads) quantize_act_kernel(const ActPara
     for (int ps = 0; ps < np; ++ps) {
       float v[E];
       load_row_values<E>(xs + (size_t)rr * L.xs_stride + ps * W + lane * E, v);
-      apply_signs<E>(v, p.signs, kbase + ps * W + lane * E);
-      fwht_warp<E>(v, p.b);
+      rotate_signed<E>(v, p.signs, p.n_rht, p.K / 32, kbase + ps * W + lane * E, p.b);
       if (cs.pre != 1.f) {
 #pragma unroll
         for (int i = 0; i < E; ++i) v[i] *= cs.pre;
@@ -351,7 +350,8 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __re
                                                                    int K, int b, float scale_mul,
                                                                    uint8_t* __restrict__ Wq,
                                                                    float* __restrict__ s_w,
-                                                                   const uint32_t* signs) {
+                                                                   const uint32_t* signs,
+                                                                   int n_rht) {
   extern __shared__ __align__(16) float row[];
   __shared__ float red[kPackThreads / 32];
   const int n = blockIdx.x;
@@ -366,15 +366,29 @@ __global__ void __launch_bounds__(kPackThreads) pack_weight_kernel(const T* __re
     *reinterpret_cast<float4*>(row + k) = f;
   }
   __syncthreads();
-  // in-place Sylvester butterflies, level by level (pairs never cross blocks)
-  for (int h = 1; h < b; h <<= 1) {
-    for (int t = threadIdx.x; t < K / 2; t += kPackThreads) {
-      const int i = (t / h) * 2 * h + (t % h);
-      const float a = row[i], c = row[i + h];
-      row[i] = a + c;
-      row[i + h] = a - c;
+  // in-place Sylvester butterflies, level by level (pairs never cross
+  // blocks); composed randomized transforms: the next mask, then again
+  for (int pass = 0; pass < (signs ? n_rht : 1); ++pass) {
+    if (pass > 0) {
+      for (int k = threadIdx.x * 4; k < K; k += kPackThreads * 4) {
+        float v[4] = {row[k], row[k + 1], row[k + 2], row[k + 3]};
+        apply_signs<4>(v, signs + (size_t)pass * (K / 32), k);
+        row[k] = v[0];
+        row[k + 1] = v[1];
+        row[k + 2] = v[2];
+        row[k + 3] = v[3];
+      }
+      __syncthreads();
     }
-    __syncthreads();
+    for (int h = 1; h < b; h <<= 1) {
+      for (int t = threadIdx.x; t < K / 2; t += kPackThreads) {
+        const int i = (t / h) * 2 * h + (t % h);
+        const float a = row[i], c = row[i + h];
+        row[i] = a + c;
+        row[i + h] = a - c;
+      }
+      __syncthreads();
+    }
   }
   float m = 0.f;
   for (int k = threadIdx.x; k < K; k += kPackThreads) m = fmaxf(m, fabsf(row[k]));
@@ -549,9 +563,14 @@ __global__ void pack_gate_up_kernel(const uint8_t* __restrict__ Wq_g, const floa
 
 }  // namespace
 
+// 1 / (7 sqrt(b)^n): the codes' scale after n unnormalised transforms
+static float scale_after(int had_block, int n) {
+  return (float)(1.0 / (7.0 * pow(sqrt((double)had_block), (double)n)));
+}
+
 cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
-                                cudaStream_t stream, const uint32_t* signs) {
+                                cudaStream_t stream, const uint32_t* signs, int n_rht) {
   ActParams prm{};
   prm.X = reinterpret_cast<const __nv_bfloat16*>(X);
   prm.L1t = reinterpret_cast<const __nv_bfloat16*>(L1t);
@@ -562,8 +581,9 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   prm.K = K;
   prm.b = had_block;
   prm.r = r;
-  prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   prm.signs = signs;
+  prm.n_rht = signs ? n_rht : 1;
+  prm.scale_mul = scale_after(had_block, prm.n_rht);
   // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores
   // (plain Hadamard only; sign masks take the butterfly kernel below).
   if (!signs && act_tc_supported(M, K, had_block, r))
@@ -579,7 +599,8 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
 
 cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_block,
                                       const uint16_t* L1t, int r, int8_t* Xq8, float* s_x,
-                                      uint16_t* XL1b, cudaStream_t stream, const uint32_t* signs) {
+                                      uint16_t* XL1b, cudaStream_t stream, const uint32_t* signs,
+                                      int n_rht) {
   ActParams prm{};
   prm.X = reinterpret_cast<const __nv_bfloat16*>(X);
   prm.L1t = reinterpret_cast<const __nv_bfloat16*>(L1t);
@@ -590,8 +611,9 @@ cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_b
   prm.K = K;
   prm.b = had_block;
   prm.r = r;
-  prm.scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   prm.signs = signs;
+  prm.n_rht = signs ? n_rht : 1;
+  prm.scale_mul = scale_after(had_block, prm.n_rht);
   const int groups = (M + kActRows - 1) / kActRows;
   if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);
   if (K % 512 == 0) return launch_act_e<16>(prm, 8, stream);
@@ -601,14 +623,15 @@ cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_b
 }
 
 cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
-                               float* s_w, cudaStream_t stream, const uint32_t* signs) {
+                               float* s_w, cudaStream_t stream, const uint32_t* signs, int n_rht) {
   const size_t smem = (size_t)K * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(pack_weight_kernel<float>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
-  pack_weight_kernel<float><<<N, kPackThreads, smem, stream>>>(Rt, K, had_block, scale_mul, Wq, s_w,
-                                                                signs);
+  const int n = signs ? n_rht : 1;
+  pack_weight_kernel<float><<<N, kPackThreads, smem, stream>>>(Rt, K, had_block,
+                                                                scale_after(had_block, n), Wq, s_w,
+                                                                signs, n);
   return cudaGetLastError();
 }
 
@@ -622,7 +645,7 @@ cudaError_t launch_pack_lowrank_q4(const uint16_t* L1t, const uint16_t* L2t, int
   const float scale_mul = (float)(1.0 / (7.0 * sqrt((double)had_block)));
   pack<<<r, kPackThreads, smem, stream>>>(reinterpret_cast<const __nv_bfloat16*>(L1t), K, had_block,
                                           scale_mul, reinterpret_cast<uint8_t*>(qL1), s_L1,
-                                          nullptr);
+                                          nullptr, 1);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   lowrank_codes_kernel<<<(N + 7) / 8, 256, 0, stream>>>(
       reinterpret_cast<const __nv_bfloat16*>(L2t), nullptr, nullptr, nullptr, N, r,

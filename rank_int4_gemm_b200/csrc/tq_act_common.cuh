@@ -62,6 +62,22 @@ __device__ __forceinline__ void apply_signs(float (&v)[E], const uint32_t* signs
   for (int i = 0; i < E; ++i) v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (((w >> i) & 1u) << 31));
 }
 
+// x D_1 H D_2 H ... D_n H on this lane's E values (n_rht composed randomized
+// Hadamard transforms, masks of `words` words each, the first first), or x H
+// without masks.  n_rht is warp-uniform (the butterflies shuffle).
+template <int E>
+__device__ __forceinline__ void rotate_signed(float (&v)[E], const uint32_t* signs, int n_rht,
+                                              int words, int col0, int b) {
+  if (!signs) {
+    fwht_warp<E>(v, b);
+    return;
+  }
+  for (int i = 0; i < n_rht; ++i) {
+    apply_signs<E>(v, signs + (size_t)i * words, col0);
+    fwht_warp<E>(v, b);
+  }
+}
+
 // RoundClip(v * inv) with ties to even, for any v and inv (weights).
 __device__ __forceinline__ int quant_code(float v, float inv) {
   float t = rintf(v * inv);

@@ -242,7 +242,7 @@ size_t tq_layer_workspace_bytes(int M, int N, int K, int r) {
   return 256 + (M > 128 ? std::max(packed, bytes8) : packed);
 }
 
-static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* L1t,
+static int layer_impl(const uint16_t* X, const uint32_t* signs, int n_rht, const uint16_t* L1t,
                       const uint8_t* Wq, const float* s_w, const uint16_t* L2t, int M, int N,
                       int K, int r, int had_block, uint16_t* Y, void* workspace,
                       size_t workspace_bytes, void* stream) {
@@ -262,6 +262,7 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
   if (tq::layer_decode2_supported(M, N, K, r, had_block)) {
     tq::LayerArgs a{};
     a.signs = signs;
+    a.n_rht = n_rht;
     a.X = X;
     a.L1t = L1t;
     a.Wq = Wq;
@@ -286,7 +287,7 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
     // column, so a sign mask takes the butterfly kernel (same int8 outputs)
     if (cudaError_t e = signs ? tq::launch_quantize_act_bf_i8(X, M, K, had_block, L1t, r, Xq8,
                                                               s_x8, r > 0 ? XL1b : nullptr, st,
-                                                              signs)
+                                                              signs, n_rht)
                               : tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8,
                                                   nullptr, r > 0 ? XL1b : nullptr, st))
       return from_cuda(e);
@@ -312,7 +313,7 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
   float* s_x = reinterpret_cast<float*>(Xq + align256((size_t)M * K / 2));
   float* XL1 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(s_x) + align256((size_t)M * 4));
   if (cudaError_t e = tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x,
-                                              r > 0 ? XL1 : nullptr, st, signs))
+                                              r > 0 ? XL1 : nullptr, st, signs, n_rht))
     return from_cuda(e);
   tq::GemmArgs g{};
   g.Xq = Xq;
@@ -335,26 +336,34 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, const uint16_t* 
 int tq_w4a4_lr_layer(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
                      const uint16_t* L2t, int M, int N, int K, int r, int had_block, uint16_t* Y,
                      void* workspace, size_t workspace_bytes, void* stream) {
-  return layer_impl(X, nullptr, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
+  return layer_impl(X, nullptr, 1, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
                     workspace_bytes, stream);
 }
 
 // ------------------------------------------------ randomized Hadamard
-int tq_pack_weight_rht(const float* Rt, int N, int K, int had_block, const uint32_t* signs,
-                       uint8_t* Wq, float* s_w, void* stream) {
-  if (!Rt || !Wq || !s_w || !signs || N <= 0) return TQ_ERR_INVALID_VALUE;
+// n_rht composed randomized Hadamard transforms: masks [n_rht][K / 32]
+static bool rht_count_ok(int n_rht) { return n_rht >= 1 && n_rht <= 3; }
+
+int tq_pack_weight_rhtn(const float* Rt, int N, int K, int had_block, const uint32_t* signs,
+                        int n_rht, uint8_t* Wq, float* s_w, void* stream) {
+  if (!Rt || !Wq || !s_w || !signs || N <= 0 || !rht_count_ok(n_rht)) return TQ_ERR_INVALID_VALUE;
   if (int s = check_k(K, had_block)) return s;
   if (!aligned16(Rt) || !aligned16(Wq) || !aligned16(s_w) || !aligned16(signs))
     return TQ_ERR_MISALIGNED;
   if (int s = check_device()) return s;
   return from_cuda(tq::launch_pack_weight(Rt, N, K, had_block, Wq, s_w,
-                                          static_cast<cudaStream_t>(stream), signs));
+                                          static_cast<cudaStream_t>(stream), signs, n_rht));
 }
 
-int tq_quantize_act_rht(const uint16_t* X, int M, int K, int had_block, const uint32_t* signs,
-                        const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
-                        void* stream) {
-  if (!X || !Xq || !s_x || !signs || M <= 0) return TQ_ERR_INVALID_VALUE;
+int tq_pack_weight_rht(const float* Rt, int N, int K, int had_block, const uint32_t* signs,
+                       uint8_t* Wq, float* s_w, void* stream) {
+  return tq_pack_weight_rhtn(Rt, N, K, had_block, signs, 1, Wq, s_w, stream);
+}
+
+int tq_quantize_act_rhtn(const uint16_t* X, int M, int K, int had_block, const uint32_t* signs,
+                         int n_rht, const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
+                         float* XL1, void* stream) {
+  if (!X || !Xq || !s_x || !signs || M <= 0 || !rht_count_ok(n_rht)) return TQ_ERR_INVALID_VALUE;
   if (int s = check_k(K, had_block)) return s;
   if (int s = check_r(r)) return s;
   if ((r > 0) != (L1t != nullptr) || (r > 0) != (XL1 != nullptr)) return TQ_ERR_INVALID_VALUE;
@@ -363,17 +372,31 @@ int tq_quantize_act_rht(const uint16_t* X, int M, int K, int had_block, const ui
     return TQ_ERR_MISALIGNED;
   if (int s = check_device()) return s;
   return from_cuda(tq::launch_quantize_act(X, M, K, had_block, L1t, r, Xq, s_x, XL1,
-                                           static_cast<cudaStream_t>(stream), signs));
+                                           static_cast<cudaStream_t>(stream), signs, n_rht));
+}
+
+int tq_quantize_act_rht(const uint16_t* X, int M, int K, int had_block, const uint32_t* signs,
+                        const uint16_t* L1t, int r, uint8_t* Xq, float* s_x, float* XL1,
+                        void* stream) {
+  return tq_quantize_act_rhtn(X, M, K, had_block, signs, 1, L1t, r, Xq, s_x, XL1, stream);
+}
+
+int tq_w4a4_lr_layer_rhtn(const uint16_t* X, const uint32_t* signs, int n_rht,
+                          const uint16_t* L1t, const uint8_t* Wq, const float* s_w,
+                          const uint16_t* L2t, int M, int N, int K, int r, int had_block,
+                          uint16_t* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!signs || !rht_count_ok(n_rht)) return TQ_ERR_INVALID_VALUE;
+  if (!aligned16(signs)) return TQ_ERR_MISALIGNED;
+  return layer_impl(X, signs, n_rht, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
+                    workspace_bytes, stream);
 }
 
 int tq_w4a4_lr_layer_rht(const uint16_t* X, const uint32_t* signs, const uint16_t* L1t,
                          const uint8_t* Wq, const float* s_w, const uint16_t* L2t, int M, int N,
                          int K, int r, int had_block, uint16_t* Y, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  if (!signs) return TQ_ERR_INVALID_VALUE;
-  if (!aligned16(signs)) return TQ_ERR_MISALIGNED;
-  return layer_impl(X, signs, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y, workspace,
-                    workspace_bytes, stream);
+  return tq_w4a4_lr_layer_rhtn(X, signs, 1, L1t, Wq, s_w, L2t, M, N, K, r, had_block, Y,
+                               workspace, workspace_bytes, stream);
 }
 
 int tq_debug_w4a4_lr_layer_decode(const uint16_t* X, const uint16_t* L1t, const uint8_t* Wq,

@@ -79,11 +79,12 @@ struct DecodeParams {
   int8_t* dbg_codes;         // [M][K] activation codes, or null
   float* dbg_sx;             // [M] scales, or null
   int32_t* dbg_acc;          // [M][N] integer sums, or null
-  const uint32_t* signs;     // randomized Hadamard sign mask [K / 32], or null
+  const uint32_t* signs;     // randomized Hadamard sign masks [n_rht][K / 32], or null
   int M, N, K, r, b;
   int C;                     // CTAs per cluster (K / 256)
   int T;                     // 128-channel tiles per CTA
   float scale_mul;           // 1 / (7 sqrt(b))
+  int n_rht;                 // composed randomized Hadamards (masks)
 };
 
 // Shared-memory map (offsets from the 1024-aligned base), for rank R.
@@ -211,7 +212,9 @@ __device__ __forceinline__ void expand16(uint4 w, uint4& lo, uint4& hi) {
   hi = make_uint4(w.x & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u, w.z & 0xF0F0F0F0u, w.w & 0xF0F0F0F0u);
 }
 
-template <int R>
+// kRhtN: composed randomized Hadamards (n_rht > 1 masks); a separate
+// instantiation, so that the single-transform kernels carry none of it.
+template <int R, bool kRhtN>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     w4a4_lr_decode_kernel(const __grid_constant__ CUtensorMap map_w,
                           const __grid_constant__ CUtensorMap map_x,
@@ -414,6 +417,15 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     for (int tt = 0; tt < 2; ++tt) {
       apply_signs<8>(v[tt], p.signs, kbase + 8 * lane);  // x D (randomized Hadamard)
       fwht_warp<8>(v[tt], p.b);
+    }
+    if constexpr (kRhtN) {  // composed randomized Hadamards: D_2 H, D_3 H
+      for (int i = 1; i < p.n_rht; ++i) {
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+          apply_signs<8>(v[tt], p.signs + (size_t)i * (p.K / 32), kbase + 8 * lane);
+          fwht_warp<8>(v[tt], p.b);
+        }
+      }
     }
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
@@ -729,13 +741,14 @@ cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream, int8_t
   p.dbg_sx = dbg_sx;
   p.dbg_acc = dbg_acc;
   p.signs = a.signs;
+  p.n_rht = a.signs ? a.n_rht : 1;
   p.M = a.M;
   p.N = a.N;
   p.K = a.K;
   p.r = a.r;
   p.b = a.had_block;
   p.C = a.K / kSlice;
-  p.scale_mul = (float)(1.0 / (7.0 * sqrt((double)a.had_block)));
+  p.scale_mul = (float)(1.0 / (7.0 * pow(sqrt((double)a.had_block), (double)p.n_rht)));
   // tiles per CTA: spread the channel tiles over the groups the SMs hold,
   // at most kMaxT per CTA
   const int tiles = (a.N + 127) / 128;
@@ -760,12 +773,15 @@ cudaError_t launch_layer_decode2(const LayerArgs& a, cudaStream_t stream, int8_t
     map_l1 = map_x;  // never read
   }
   using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, DecodeParams);
-  const int ri = a.r == 64 ? 3 : a.r / 16;  // 0, 1, 2, 3
-  const KernelFn fns[4] = {w4a4_lr_decode_kernel<0>, w4a4_lr_decode_kernel<16>,
-                           w4a4_lr_decode_kernel<32>, w4a4_lr_decode_kernel<64>};
-  const uint32_t allocs[4] = {Sm<0>::kAlloc, Sm<16>::kAlloc, Sm<32>::kAlloc, Sm<64>::kAlloc};
+  const int ri = (a.r == 64 ? 3 : a.r / 16) + (p.n_rht > 1 ? 4 : 0);
+  const KernelFn fns[8] = {w4a4_lr_decode_kernel<0, false>, w4a4_lr_decode_kernel<16, false>,
+                           w4a4_lr_decode_kernel<32, false>, w4a4_lr_decode_kernel<64, false>,
+                           w4a4_lr_decode_kernel<0, true>,  w4a4_lr_decode_kernel<16, true>,
+                           w4a4_lr_decode_kernel<32, true>, w4a4_lr_decode_kernel<64, true>};
+  const uint32_t allocs[8] = {Sm<0>::kAlloc, Sm<16>::kAlloc, Sm<32>::kAlloc, Sm<64>::kAlloc,
+                              Sm<0>::kAlloc, Sm<16>::kAlloc, Sm<32>::kAlloc, Sm<64>::kAlloc};
   const KernelFn fn = fns[ri];
-  static uint64_t attr_set[4] = {0, 0, 0, 0};
+  static uint64_t attr_set[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(attr_set[ri] >> dev & 1u)) {

@@ -15,21 +15,23 @@ struct Tuning {
 };
 Tuning& tuning();
 
-// `signs`: the randomized Hadamard's sign mask [K / 32] (rotation by D H),
-// or null for the plain Hadamard.
+// `signs`: n_rht randomized Hadamard sign masks [n_rht][K / 32] (rotation
+// by D_1 H ... D_n H, composed transforms), or null for the plain Hadamard.
 cudaError_t launch_pack_weight(const float* Rt, int N, int K, int had_block, uint8_t* Wq,
-                               float* s_w, cudaStream_t stream, const uint32_t* signs = nullptr);
+                               float* s_w, cudaStream_t stream, const uint32_t* signs = nullptr,
+                               int n_rht = 1);
 
 cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
                                 const uint16_t* L1t, int r, uint8_t* Xq, float* s_x,
-                                float* XL1, cudaStream_t stream, const uint32_t* signs = nullptr);
+                                float* XL1, cudaStream_t stream, const uint32_t* signs = nullptr,
+                                int n_rht = 1);
 
 // The butterfly activation kernel writing one code per byte and bf16(X L1)
 // (the int8-code GEMM's operands), with an optional sign mask.
 cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_block,
                                       const uint16_t* L1t, int r, int8_t* Xq8, float* s_x,
                                       uint16_t* XL1b, cudaStream_t stream,
-                                      const uint32_t* signs = nullptr);
+                                      const uint32_t* signs = nullptr, int n_rht = 1);
 
 // Activation stage on tensor cores (many tokens): rotation and X L1 as MMAs.
 // Codes packed (Xq, [M][K/2]) or one int8 per code (Xq8, [M][K]); X L1 as
@@ -109,7 +111,8 @@ cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t stream);
 
 // The whole layer from bf16 X (decode sizes: one fused kernel).
 struct LayerArgs {
-  const uint32_t* signs = nullptr;  // randomized Hadamard sign mask [K / 32], or null
+  const uint32_t* signs = nullptr;  // randomized Hadamard sign masks [n_rht][K / 32], or null
+  int n_rht = 1;
   const uint16_t* X;
   const uint16_t* L1t;
   const uint8_t* Wq;

@@ -49,6 +49,13 @@ _lib.tq_quantize_act_rht.argtypes = [_P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _P]
 _lib.tq_w4a4_lr_layer_rht.restype = _I
 _lib.tq_w4a4_lr_layer_rht.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
                                       ctypes.c_size_t, _P]
+_lib.tq_pack_weight_rhtn.restype = _I
+_lib.tq_pack_weight_rhtn.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _P]
+_lib.tq_quantize_act_rhtn.restype = _I
+_lib.tq_quantize_act_rhtn.argtypes = [_P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P]
+_lib.tq_w4a4_lr_layer_rhtn.restype = _I
+_lib.tq_w4a4_lr_layer_rhtn.argtypes = [_P, _P, _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P,
+                                       ctypes.c_size_t, _P]
 _lib.tq_pack_shared_input.restype = _I
 _lib.tq_pack_shared_input.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P]
 _lib.tq_debug_w4a4_lr_layer_decode.restype = _I
@@ -513,8 +520,13 @@ def tq_w4a4_lr_layer(X, L1t, Wq, s_w, L2t, had_block, Y=None, workspace=None, st
 
 
 def _signs(signs, K):
+    """(pointer, n): a mask [K/32] (one transform) or masks [n][K/32] (n
+    composed transforms, the first applied first), int32 words."""
+    if signs.dim() == 2:
+        _need(signs, torch.int32, (signs.shape[0], K // 32), "signs")
+        return _ptr(signs), int(signs.shape[0])
     _need(signs, torch.int32, (K // 32,), "signs")
-    return _ptr(signs)
+    return _ptr(signs), 1
 
 
 def tq_pack_weight_rht(Rt: torch.Tensor, had_block: int, signs: torch.Tensor, Wq=None, s_w=None,
@@ -525,14 +537,16 @@ def tq_pack_weight_rht(Rt: torch.Tensor, had_block: int, signs: torch.Tensor, Wq
     _need(Rt, torch.float32, (N, K), "Rt")
     Wq = torch.empty(N, K // 2, dtype=torch.uint8, device=Rt.device) if Wq is None else Wq
     s_w = torch.empty(N, dtype=torch.float32, device=Rt.device) if s_w is None else s_w
-    _check(_lib.tq_pack_weight_rht(_ptr(Rt), N, K, int(had_block), _signs(signs, K), _ptr(Wq),
-                                   _ptr(s_w), _stream(stream)), "tq_pack_weight_rht")
+    sp, n = _signs(signs, K)
+    _check(_lib.tq_pack_weight_rhtn(_ptr(Rt), N, K, int(had_block), sp, n, _ptr(Wq),
+                                    _ptr(s_w), _stream(stream)), "tq_pack_weight_rhtn")
     return Wq, s_w
 
 
 def tq_quantize_act_rht(X: torch.Tensor, had_block: int, signs: torch.Tensor, L1t=None,
                         stream=None):
-    """tq_quantize_act with the randomized Hadamard: codes of X D H."""
+    """tq_quantize_act with the randomized Hadamard: codes of X D H (signs
+    [K/32]), or of X D_1 H ... D_n H (signs [n][K/32], composed)."""
     M, K = X.shape
     _need(X, torch.bfloat16, (M, K), "X")
     r = 0 if L1t is None else L1t.shape[0]
@@ -540,10 +554,11 @@ def tq_quantize_act_rht(X: torch.Tensor, had_block: int, signs: torch.Tensor, L1
     Xq = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
     s_x = torch.empty(M, dtype=torch.float32, device=dev)
     XL1 = torch.empty(M, r, dtype=torch.float32, device=dev) if r else None
-    _check(_lib.tq_quantize_act_rht(_ptr(X), M, K, int(had_block), _signs(signs, K),
-                                    _ptr(L1t) if r else None, r, _ptr(Xq), _ptr(s_x),
-                                    _ptr(XL1) if r else None, _stream(stream)),
-           "tq_quantize_act_rht")
+    sp, n = _signs(signs, K)
+    _check(_lib.tq_quantize_act_rhtn(_ptr(X), M, K, int(had_block), sp, n,
+                                     _ptr(L1t) if r else None, r, _ptr(Xq), _ptr(s_x),
+                                     _ptr(XL1) if r else None, _stream(stream)),
+           "tq_quantize_act_rhtn")
     return Xq, s_x, XL1
 
 
@@ -559,10 +574,11 @@ def tq_w4a4_lr_layer_rht(X, signs, L1t, Wq, s_w, L2t, had_block, Y=None, workspa
         workspace = Workspace(X.device)
     ws = workspace.get(tq_layer_workspace_bytes(M, N, K, r)) if isinstance(workspace, Workspace) \
         else workspace
-    _check(_lib.tq_w4a4_lr_layer_rht(_ptr(X), _signs(signs, K), _ptr(L1t) if r else None,
-                                     _ptr(Wq), _ptr(s_w), _ptr(L2t) if r else None, M, N, K, r,
-                                     int(had_block), _ptr(Y), _ptr(ws), ws.numel(),
-                                     _stream(stream)), "tq_w4a4_lr_layer_rht")
+    sp, n = _signs(signs, K)
+    _check(_lib.tq_w4a4_lr_layer_rhtn(_ptr(X), sp, n, _ptr(L1t) if r else None,
+                                      _ptr(Wq), _ptr(s_w), _ptr(L2t) if r else None, M, N, K, r,
+                                      int(had_block), _ptr(Y), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "tq_w4a4_lr_layer_rhtn")
     return Y
 
 

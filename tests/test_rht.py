@@ -283,3 +283,66 @@ def test_composed_eq3_invariance_and_bit_masks():
     X, W = rng.normal(size=(4, K)), rng.normal(size=(6, K))
     lhs = oracle.rotate(X, b, signs=d) @ oracle.rotate(W, b, signs=d).T
     assert np.allclose(lhs, X @ W.T, rtol=0, atol=1e-10)
+
+
+def _dev_masks(n, K, seed):
+    return torch.stack([_dev_signs(K, seed + 101 * i) for i in range(n)]).contiguous()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,b", [(2, 128), (3, 256), (2, 16)])
+def test_composed_weight_and_activation_codes_match_oracle(tq, n, b):
+    K, M = 2048, 200
+    sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=384, r=32, had_block=b)
+    L = synth.make_layer(sh, seed=31)
+    sg = _dev_masks(n, K, 5 * b + n)
+    d = oracle.signs_from_bits(sg.cpu().numpy().view(np.uint32), K)
+    assert d.shape == (n, K)
+    Wq, s_w = tq.tq_pack_weight_rht(L["Rt"].cuda(), b, sg)
+    Xq, s_x, _ = tq.tq_quantize_act_rht(L["X"].cuda(), b, sg)
+    torch.cuda.synchronize()
+    w = oracle.pack_weight(L["Rt"], b, signs=d)
+    check_codes(Wq.cpu().numpy(), w["qw"], w["t_w"], f"composed ({n}) weight codes")
+    check_scales(s_w.cpu().numpy(), w["s_w"], f"composed ({n}) s_w")
+    a = oracle.quantize_act(L["X"], b, signs=d)
+    fx = check_codes(Xq.cpu().numpy(), a["qx"], a["t_x"], f"composed ({n}) activation codes")
+    check_scales(s_x.cpu().numpy(), a["s_x"], f"composed ({n}) s_x")
+    print(f"FLIPS rht{n} act b={b}: x={fx:.3e}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("n,M,K,N,r,b", [(2, 16, 4096, 4096, 32, 128), (3, 1, 2048, 1024, 64, 256),
+                                         (2, 300, 2048, 512, 32, 128), (2, 40, 1024, 264, 16, 64)])
+def test_composed_layer_matches_oracle(tq, n, M, K, N, r, b):
+    # the fused decode kernel (M <= 16), the int8-code path (M > 128) and the
+    # packed path (in between) with n composed transforms on both sides
+    sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=r, had_block=b)
+    L = synth.make_layer(sh, seed=33, device="cuda" if K * N >= 1 << 22 else "cpu")
+    sg = _dev_masks(n, K, M + K + n)
+    d = oracle.signs_from_bits(sg.cpu().numpy().view(np.uint32), K)
+    Wq, s_w = tq.tq_pack_weight_rht(L["Rt"].cuda(), b, sg)
+    Y = tq.tq_w4a4_lr_layer_rht(L["X"].cuda(), sg, L["L1t"].cuda(), Wq, s_w, L["L2t"].cuda(), b)
+    Xq, _, _ = tq.tq_quantize_act_rht(L["X"].cuda(), b, sg)
+    torch.cuda.synchronize()
+    o = oracle.layer(L["X"], L["L1t"], L["L2t"], L["Rt"], b, signs=d)
+    q = oracle.unpack_int4(Xq.cpu().numpy())
+    qw = oracle.unpack_int4(Wq.cpu().numpy())
+    fx = check_codes(q, o["qx"], o["t_x"], "composed codes", packed=False)
+    fw = check_codes(qw, o["qw"], o["t_w"], "composed weight codes", packed=False)
+    fro, mx = check_y(Y.double().cpu().numpy(), y_reference(q, o, fx, qw, fw),
+                      f"composed ({n}) layer M={M} K={K} N={N}")
+    print(f"FLIPS rht{n} layer M={M} path={tq.tq_layer_path(M, N, K, r, b)}: fro={fro:.3e}")
+
+
+def test_composed_entry_argument_checks():
+    import ctypes
+
+    import rank_int4_gemm_b200 as tq
+    lib = tq.tq.raw()
+    P = ctypes.c_void_p
+    F = 0x1000
+    # n_rht outside 1..3
+    for n in (0, 4):
+        assert lib.tq_pack_weight_rhtn(P(F), 8, 256, 128, P(F), n, P(F), P(F), None) == 1
+        assert lib.tq_w4a4_lr_layer_rhtn(P(F), P(F), n, None, P(F), P(F), None, 16, 256, 256, 0,
+                                         128, P(F), P(F), ctypes.c_size_t(1 << 20), None) == 1
