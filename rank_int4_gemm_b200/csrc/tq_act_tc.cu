@@ -394,8 +394,23 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
               cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
             }
           }
+          if (p.Xq8 && !asym) {
+            // one code per byte: staged per warp (the asymmetric min area,
+            // unused here) as [32 rows][64 B], 16-byte chunks swizzled by
+            // row, so that the global stores below cover whole sectors
+            uint32_t w[8];
+#pragma unroll
+            for (int h = 0; h < 8; ++h)
+              w[h] = low_bytes4(cb[4 * h], cb[4 * h + 1], cb[4 * h + 2], cb[4 * h + 3]);
+            const uint32_t sb = base + L.amin + (uint32_t)(warp - kEpiFirstWarp) * 2048u +
+                                (uint32_t)lane * 64u;
+            const uint32_t sw = ((uint32_t)lane >> 1) & 3u;
+            const uint32_t c0 = 2u * (uint32_t)(g - 2 * half);
+            st_shared_v4_tc(sb + ((c0 ^ sw) << 4), make_uint4(w[0], w[1], w[2], w[3]));
+            st_shared_v4_tc(sb + (((c0 + 1u) ^ sw) << 4), make_uint4(w[4], w[5], w[6], w[7]));
+          }
           if (grow < p.M) {
-            if (p.Xq8) {  // one code per byte, in column order
+            if (p.Xq8 && asym) {  // one code per byte, in column order
               uint32_t w[8];
 #pragma unroll
               for (int h = 0; h < 8; ++h)
@@ -418,6 +433,28 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
             }
           }
         }
+      }
+      if (ok && p.Xq8 && !asym) {
+        // the warp's 32 rows x 64 B: lane l writes 16-byte part l % 4 of rows
+        // l / 4 + 8 i, i.e. 8 whole 64-byte row segments per store
+        __syncwarp();
+        const size_t blk = (size_t)(kb0 + i - nb);
+        const uint32_t sbw = base + L.amin + (uint32_t)(warp - kEpiFirstWarp) * 2048u;
+#pragma unroll
+        for (int i4 = 0; i4 < 4; ++i4) {
+          const int rw = (lane >> 2) + 8 * i4, part = lane & 3;
+          const uint32_t src = sbw + (uint32_t)rw * 64u +
+                               ((((uint32_t)part) ^ (((uint32_t)rw >> 1) & 3u)) << 4);
+          uint4 v4;
+          asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                       : "=r"(v4.x), "=r"(v4.y), "=r"(v4.z), "=r"(v4.w)
+                       : "r"(src));
+          const int gr = tile * kTok + q * 32 + rw;
+          if (gr < p.M)
+            *reinterpret_cast<uint4*>(p.Xq8 + (size_t)gr * (size_t)p.K + blk * kBlk + 64 * half +
+                                      16 * part) = v4;
+        }
+        __syncwarp();
       }
       tc_fence_before();
       mbar_arrive(&rot_empty[u]);
