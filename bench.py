@@ -1075,7 +1075,7 @@ def cpu_baseline(M, budget_s=12.0, decode=None, prefill=None):
     * prefill: the first 64 tokens of each prefill layer (weights packed
       beforehand, untimed); the layer time is extrapolated linearly in M.
     Also returns the flip fractions of the timed path's codes against the
-    oracle's on those samples (the benchmark spec's reported fraction)."""
+    oracle's on those samples (the reported fraction of midpoint flips)."""
     import numpy as np
 
     import oracle
