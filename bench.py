@@ -968,8 +968,9 @@ def run_rht(args, rank, world, local_rank, dist):
     """The layer with the randomized Hadamard (a sign mask before the
     Hadamard blocks) against the plain layer: the decode projection (M = 16,
     a stack of 16 layers, the one-kernel path) and the Llama-3-8B gate/up
-    prefill shape (M = 2048: butterfly activation kernel + packed-code GEMM
-    with signs, the int8-code path without)."""
+    prefill shape (M = 2048: the tensor-core activation kernel, which negates
+    the masked columns of each staged X block, then the int8-code GEMM; the
+    plain layer runs the same kernels without the mask)."""
     import torch
 
     import rank_int4_gemm_b200 as tq

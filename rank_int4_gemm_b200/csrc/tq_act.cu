@@ -584,10 +584,12 @@ cudaError_t launch_quantize_act(const uint16_t* X, int M, int K, int had_block,
   prm.signs = signs;
   prm.n_rht = signs ? n_rht : 1;
   prm.scale_mul = scale_after(had_block, prm.n_rht);
-  // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores
-  // (plain Hadamard only; sign masks take the butterfly kernel below).
-  if (!signs && act_tc_supported(M, K, had_block, r))
-    return launch_act_tc(X, M, K, had_block, L1t, r, Xq, nullptr, s_x, XL1, nullptr, stream);
+  // Many tokens: 128-token tiles, rotation and X L1 on the tensor cores, with
+  // at most one sign mask (negated in shared memory before the rotation);
+  // composed transforms take the butterfly kernel below.
+  if ((!signs || prm.n_rht == 1) && act_tc_supported(M, K, had_block, r))
+    return launch_act_tc(X, M, K, had_block, L1t, r, Xq, nullptr, s_x, XL1, nullptr, stream,
+                         nullptr, signs);
   // Few token groups (decode): spread K over up to 16 CTAs of 256 columns.
   const int groups = (M + kActRows - 1) / kActRows;
   if (groups <= 8 && K % 256 == 0 && K / 256 <= 16) return launch_act_e<8>(prm, 16, stream);

@@ -47,6 +47,14 @@ constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
 constexpr int kEpiFirstWarp = 2;
 constexpr int kEpiThreadsTc = 256;
 constexpr int kThreadsTc = 32 * kEpiFirstWarp + kEpiThreadsTc;
+// With a sign mask (randomized Hadamard, x D H): four more warps negate the
+// masked columns of each staged block before its MMAs.
+constexpr int kFlipFirstWarp = kEpiFirstWarp + kEpiThreadsTc / 32;
+constexpr int kFlipThreads = 128;
+template <bool kSigned>
+constexpr int tc_threads() {
+  return kThreadsTc + (kSigned ? kFlipThreads : 0);
+}
 
 struct TcParams {
   uint8_t* Xq;       // [M][K/2] packed codes, or null
@@ -61,13 +69,15 @@ struct TcParams {
   float zmul;         // 1 / sqrt(b): the zero-point of the unnormalised transform
   int kb_total, nb;   // 128-column blocks in K, blocks per CTA
   float scale_mul;    // 1 / (7 sqrt(b)); asymmetric: 1 / (15 sqrt(b))
+  const uint32_t* signs;  // [K / 32] words: bit k % 32 of word k / 32 negates column k, or null
 };
 
 // Shared memory (offsets from the 1024-aligned base).  Atoms are 128-byte
 // swizzled K-major tiles of 64 bf16 columns.  A stage holds one X block and,
 // when X L1 is computed, the matching L1^T block (2 atoms x r rows); an
 // X-L1-only launch has no Hadamard operand.
-constexpr int kNumBarsTc = 2 * kMaxNS + 2 * kRot + 1;  // full, empty; rot_full, rot_empty; xl1_full
+// full, empty; rot_full, rot_empty; xl1_full; flipped (sign mask applied)
+constexpr int kNumBarsTc = 3 * kMaxNS + 2 * kRot + 1;
 struct TcLayout {
   uint32_t h, stage0, stage, amax, amin, bar, misc, bytes;
   int ns;  // stages
@@ -121,9 +131,51 @@ __device__ __forceinline__ uint32_t atom_off(uint32_t row, uint32_t c, uint32_t 
   return (c >> 3) * rows * 128u + row * 128u + (((c & 7u) ^ (row & 7u)) << 4);
 }
 
-__global__ void __launch_bounds__(kThreadsTc, 1)
+// x D on a staged block: negate column k (bit k of the block's 128-bit mask
+// m) in every row of a two-atom tile of `rows` rows (rows % 8 == 0).  Chunk
+// ch of the tile is 16 bytes at tile + 16 ch: atom ch / (8 rows), row
+// (ch / 8) % rows, stored chunk ch % 8, which holds columns 8 (ch % 8 ^ row
+// % 8) .. +7 of the atom.  A sign flip is exact, so (x D) H and (x D)(D L1)
+// = x L1 lose nothing.
+__device__ __forceinline__ uint32_t sign_bits8(uint4 m, uint32_t k0) {
+  const uint32_t w = (k0 & 64u) ? ((k0 & 32u) ? m.w : m.z) : ((k0 & 32u) ? m.y : m.x);
+  return (w >> (k0 & 31u)) & 0xFFu;
+}
+__device__ __forceinline__ void flip_columns(uint32_t tile, uint32_t rows, uint4 m, uint32_t t) {
+  const uint32_t n = 16u * rows;
+  for (uint32_t c0 = t; c0 < n; c0 += 2u * kFlipThreads) {
+    uint4 v[2];
+    uint32_t bits[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t ch = c0 + (uint32_t)u * kFlipThreads;
+      const uint32_t atom = ch >= 8u * rows ? 1u : 0u;
+      const uint32_t k0 = 64u * atom + 8u * ((ch & 7u) ^ ((ch >> 3) & 7u));
+      bits[u] = ch < n ? sign_bits8(m, k0) : 0u;
+      if (ch < n)
+        asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(v[u].x), "=r"(v[u].y), "=r"(v[u].z), "=r"(v[u].w)
+                     : "r"(tile + 16u * ch));
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const uint32_t ch = c0 + (uint32_t)u * kFlipThreads;
+      const uint32_t b = bits[u];
+      // element 2e in the low half of word e, 2e + 1 in the high half
+      v[u].x ^= ((b & 1u) << 15) | ((b & 2u) << 30);
+      v[u].y ^= ((b & 4u) << 13) | ((b & 8u) << 28);
+      v[u].z ^= ((b & 16u) << 11) | ((b & 32u) << 26);
+      v[u].w ^= ((b & 64u) << 9) | ((b & 128u) << 24);
+      if (ch < n) st_shared_v4_tc(tile + 16u * ch, v[u]);
+    }
+  }
+}
+
+template <bool kSigned>
+__global__ void __launch_bounds__(tc_threads<kSigned>(), 1)
     quantize_act_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                            const __grid_constant__ CUtensorMap map_l1, const TcParams p) {
+  constexpr int kThr = tc_threads<kSigned>();
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
@@ -137,6 +189,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   uint64_t* rot_full = bars + 2 * kMaxNS;
   uint64_t* rot_empty = rot_full + kRot;
   uint64_t* xl1_full = rot_full + 2 * kRot;
+  uint64_t* flipped = xl1_full + 1;  // [kMaxNS]: the stage's masked columns negated
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.misc + 4);
 
@@ -185,6 +238,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       mbar_init(&rot_empty[i], kEpiThreadsTc);
     }
     mbar_init(xl1_full, 1);
+    if (kSigned)
+      for (int i = 0; i < kMaxNS; ++i) mbar_init(&flipped[i], kFlipThreads);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&map_x);
@@ -203,7 +258,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
   {
     const int bm = p.b - 1;
     constexpr unsigned long long kParity8 = 0x963C5AF066CCAA00ull;  // byte m: bit e = parity(m & e)
-    for (int ch = threadIdx.x - 32; warp > 0 && ch < (xo ? 0 : kBlk * 16); ch += kThreadsTc - 32) {
+    for (int ch = threadIdx.x - 32; warp > 0 && ch < (xo ? 0 : kBlk * 16); ch += kThr - 32) {
       const int j = ch >> 4, c = ch & 15;
       const int k0 = c * 8;
       uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -271,7 +326,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       const int s = i % L.ns, u = i % kRot;
       const bool second = xo || resident || i >= nb;
       const int j = i < nb ? i : i - nb;
-      if (!mbar_wait(&full[s], (uint32_t)(i / L.ns) & 1u, nullptr, abort_flag)) break;
+      if (!mbar_wait(kSigned ? &flipped[s] : &full[s], (uint32_t)(i / L.ns) & 1u, nullptr,
+                     abort_flag))
+        break;
       if (!xo && !mbar_wait(&rot_empty[u], ((uint32_t)(i / kRot) & 1u) ^ 1u, nullptr, abort_flag))
         break;
       tc_fence_after();
@@ -297,6 +354,31 @@ __global__ void __launch_bounds__(kThreadsTc, 1)
       __syncwarp();
     }
     if (lane == 0 && r > 0) mma_commit(xl1_full);
+    __syncwarp();
+    cluster_wait_acquire();    // B1
+    cluster_arrive_rel();      // B2
+    cluster_wait_acquire();
+    cluster_arrive_rel();      // B3
+    cluster_wait_acquire();
+  } else if (kSigned && warp >= kFlipFirstWarp) {
+    // ==================================================== sign mask (x D)
+    // every staged X block, and in the code pass its L1^T block, before the
+    // MMAs read them (the MMA issuer waits on `flipped` instead of `full`)
+    cluster_wait_acquire();    // B0
+    cluster_arrive_rel();      // B1
+    const uint32_t t = threadIdx.x - kFlipFirstWarp * 32;
+    for (int i = 0; i < n_loads; ++i) {
+      const int s = i % L.ns;
+      const bool second = xo || resident || i >= nb;
+      const int j = i < nb ? i : i - nb;
+      if (!mbar_wait(&full[s], (uint32_t)(i / L.ns) & 1u, nullptr, abort_flag)) break;
+      const uint4 m = __ldg(reinterpret_cast<const uint4*>(p.signs) + (kb0 + j));
+      const uint32_t st = base + L.stage0 + (uint32_t)s * L.stage;
+      flip_columns(st, kTok, m, t);
+      if (second && r > 0) flip_columns(st + 2u * kTok * 128u, (uint32_t)r, m, t);
+      fence_proxy_async_smem();  // generic-proxy writes -> the MMAs' reads
+      mbar_arrive(&flipped[s]);
+    }
     __syncwarp();
     cluster_wait_acquire();    // B1
     cluster_arrive_rel();      // B2
@@ -545,8 +627,13 @@ namespace {
 cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                               int r_total, int r_off, int r, bool xl1_only, uint8_t* Xq,
                               int8_t* Xq8, float* s_x, float* z_x, float* XL1, uint16_t* XL1b,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, const uint32_t* signs) {
   TcParams p{};
+  // X L1 alone needs no mask: (x D)(D L1) = x L1
+  p.signs = xl1_only ? nullptr : signs;
+  const bool sg = p.signs != nullptr;
+  auto* kern = sg ? quantize_act_tc_kernel<true> : quantize_act_tc_kernel<false>;
+  const int threads = sg ? tc_threads<true>() : tc_threads<false>();
   p.Xq = xl1_only ? nullptr : Xq;
   p.Xq8 = xl1_only ? nullptr : Xq8;
   p.s_x = s_x;
@@ -565,18 +652,17 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
   p.zmul = (float)(1.0 / sqrt((double)had_block));
   const int tiles = (M + kTok - 1) / kTok;
   const uint32_t smem_bytes = tc_layout(xl1_only, r).bytes + 1024u;
-  static uint64_t attr_set = 0;
+  static uint64_t attr_set[2] = {0, 0};  // per kernel variant, a bit per device
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(attr_set >> dev & 1u)) {
+  if (!(attr_set[sg] >> dev & 1u)) {
     // every layout is at most kSmemCap (three stages only where they fit)
-    cudaError_t e = cudaFuncSetAttribute(quantize_act_tc_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemCap);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(quantize_act_tc_kernel,
-                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    attr_set |= uint64_t(1) << dev;
+    attr_set[sg] |= uint64_t(1) << dev;
   }
   // a cluster of C CTAs along K per 128-token tile: about one CTA per SM,
   // and no larger than lets every cluster of the grid be resident at once.
@@ -594,7 +680,7 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
     }
     cudaLaunchConfig_t q = {};
     q.gridDim = dim3(Ce, tiles, 1);
-    q.blockDim = dim3(kThreadsTc, 1, 1);
+    q.blockDim = dim3(threads, 1, 1);
     q.dynamicSmemBytes = smem_bytes;
     cudaLaunchAttribute qa[1];
     qa[0].id = cudaLaunchAttributeClusterDimension;
@@ -604,7 +690,7 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
     q.attrs = qa;
     q.numAttrs = 1;
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, quantize_act_tc_kernel, &q) == cudaSuccess &&
+    if (cudaOccupancyMaxActiveClusters(&active, kern, &q) == cudaSuccess &&
         active >= tiles) {
       C = Ce;
       break;
@@ -626,7 +712,7 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(C, tiles, 1);
-  cfg.blockDim = dim3(kThreadsTc, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem_bytes;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -636,7 +722,7 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, quantize_act_tc_kernel, map_x, map_l1, p);
+  return cudaLaunchKernelEx(&cfg, kern, map_x, map_l1, p);
 }
 
 }  // namespace
@@ -647,17 +733,18 @@ cudaError_t launch_act_tc_one(const uint16_t* X, int M, int K, int had_block, co
 // at most kMaxRx columns that skip the rotation.
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                           int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
-                          cudaStream_t stream, float* z_x) {
+                          cudaStream_t stream, float* z_x, const uint32_t* signs) {
+  if (signs && z_x) return cudaErrorInvalidValue;  // the masked codes are symmetric
   if (r <= kMaxRtc)
     return launch_act_tc_one(X, M, K, had_block, L1t, r, 0, r, false, Xq, Xq8, s_x, z_x, XL1,
-                             XL1b, stream);
+                             XL1b, stream, signs);
   if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, nullptr, r, 0, 0, false, Xq, Xq8, s_x,
-                                        z_x, nullptr, nullptr, stream))
+                                        z_x, nullptr, nullptr, stream, signs))
     return e;
   for (int off = 0; off < r; off += kMaxRx) {
     const int w = std::min(kMaxRx, r - off);
     if (cudaError_t e = launch_act_tc_one(X, M, K, had_block, L1t, r, off, w, true, Xq, Xq8, s_x,
-                                          nullptr, XL1, XL1b, stream))
+                                          nullptr, XL1, XL1b, stream, nullptr))
       return e;
   }
   return cudaSuccess;

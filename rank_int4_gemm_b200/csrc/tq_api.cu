@@ -283,13 +283,16 @@ static int layer_impl(const uint16_t* X, const uint32_t* signs, int n_rht, const
     float* s_x8 = reinterpret_cast<float*>(ws + 256 + align256((size_t)M * K));
     uint16_t* XL1b =
         reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(s_x8) + align256((size_t)M * 4));
-    // the tensor-core activation kernel has one Hadamard operand for every
-    // column, so a sign mask takes the butterfly kernel (same int8 outputs)
-    if (cudaError_t e = signs ? tq::launch_quantize_act_bf_i8(X, M, K, had_block, L1t, r, Xq8,
-                                                              s_x8, r > 0 ? XL1b : nullptr, st,
-                                                              signs, n_rht)
-                              : tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8,
-                                                  nullptr, r > 0 ? XL1b : nullptr, st))
+    // the tensor-core activation kernel applies one sign mask (in shared
+    // memory, before its rotation MMA); composed transforms take the
+    // butterfly kernel (same int8 outputs)
+    if (cudaError_t e = (signs && n_rht > 1)
+                            ? tq::launch_quantize_act_bf_i8(X, M, K, had_block, L1t, r, Xq8, s_x8,
+                                                            r > 0 ? XL1b : nullptr, st, signs,
+                                                            n_rht)
+                            : tq::launch_act_tc(X, M, K, had_block, L1t, r, nullptr, Xq8, s_x8,
+                                                nullptr, r > 0 ? XL1b : nullptr, st, nullptr,
+                                                signs))
       return from_cuda(e);
     tq::GemmA8Args a{};
     a.Xq8 = Xq8;

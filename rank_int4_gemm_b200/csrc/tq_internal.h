@@ -38,10 +38,12 @@ cudaError_t launch_quantize_act_bf_i8(const uint16_t* X, int M, int K, int had_b
 // fp32 (XL1) and / or rounded to bf16 (XL1b), either may be null.
 bool act_tc_supported(int M, int K, int had_block, int r);
 // z_x non-null: asymmetric codes (zero-point = row minimum, codes 0..15
-// stored as code - 8), s_x = range / 15
+// stored as code - 8), s_x = range / 15.  signs non-null: one randomized
+// Hadamard mask ([K / 32] words), codes of x D H (symmetric only).
 cudaError_t launch_act_tc(const uint16_t* X, int M, int K, int had_block, const uint16_t* L1t,
                           int r, uint8_t* Xq, int8_t* Xq8, float* s_x, float* XL1, uint16_t* XL1b,
-                          cudaStream_t stream, float* z_x = nullptr);
+                          cudaStream_t stream, float* z_x = nullptr,
+                          const uint32_t* signs = nullptr);
 
 // GEMM with one int8 per activation code (weights expanded into TMEM).
 struct GemmA8Args {

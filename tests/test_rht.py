@@ -135,7 +135,12 @@ def test_signed_weight_pack_matches_oracle(tq, b):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M,b,r", [(1, 128, 32), (16, 256, 16), (200, 128, 64), (70, 256, 0)])
+# M >= 64 with b <= 128 runs the tensor-core activation kernel, which negates
+# the masked columns of each staged X block (and of L1^T) in shared memory;
+# r = 160 adds an X-L1-only launch (unmasked); the rest run the butterflies
+@pytest.mark.parametrize("M,b,r", [(1, 128, 32), (16, 256, 16), (200, 128, 64), (70, 256, 0),
+                                   (300, 64, 16), (1000, 128, 128), (520, 128, 160),
+                                   (130, 32, 0)])
 def test_signed_activation_codes_match_oracle(tq, M, b, r):
     from tests.parity_util import check_xl1
     K = 4096
@@ -180,9 +185,9 @@ def test_signed_layer_matches_oracle(tq, M, K, N, r, b):
 @pytest.mark.parametrize("M,K,N,b", [(300, 1024, 384, 128), (1000, 4096, 1024, 64)])
 def test_signed_layer_int8_path_equals_packed_path_at_rank0(tq, M, K, N, b):
     # above 128 tokens the signed layer writes one code per byte from the
-    # butterfly kernel and runs the int8-code GEMM; at rank 0 its Y equals
-    # the packed codes of the same kernel through the packed-code GEMM bit for
-    # bit (same codes, exact integer sums, the same fp32 epilogue)
+    # tensor-core activation kernel and runs the int8-code GEMM; at rank 0
+    # its Y equals the packed codes of the same kernel through the packed-code
+    # GEMM bit for bit (same codes, exact integer sums, the same fp32 epilogue)
     sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=N, r=0, had_block=b)
     L = synth.make_layer(sh, seed=25, device="cuda")
     sg = _dev_signs(K, M + 7)
@@ -194,6 +199,32 @@ def test_signed_layer_int8_path_equals_packed_path_at_rank0(tq, M, K, N, b):
     Y2 = tq.tq_w4a4_lr_gemm(Xq, s_x, Wq, s_w)
     torch.cuda.synchronize()
     assert torch.equal(Y, Y2)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,r", [(300, 64), (700, 160)])
+def test_masked_tensor_core_kernel_against_the_plain_one(tq, M, r):
+    # the tensor-core activation kernel with a sign mask: an all-zero mask
+    # gives the plain kernel's outputs bit for bit, and with any mask X L1
+    # is unchanged bit for bit ((x D)(D L1) = x L1 with exact sign flips and
+    # the same summation order); the codes of a mask equal those of the plain
+    # kernel on X with its masked columns negated (the same products summed
+    # in the same order)
+    K, b = 2048, 128
+    sh = synth.CONFIGS["decode"].with_(M=M, K=K, N=256, r=r, had_block=b)
+    L = synth.make_layer(sh, seed=26, device="cuda")
+    X, L1t = L["X"].cuda(), L["L1t"].cuda()
+    zero = torch.zeros(K // 32, dtype=torch.int32, device="cuda")
+    sg = _dev_signs(K, M + 3)
+    d = torch.from_numpy(oracle.signs_from_bits(sg.cpu().numpy().view(np.uint32), K)).cuda()
+    plain = tq.tq_quantize_act(X, b, L1t)
+    masked0 = tq.tq_quantize_act_rht(X, b, zero, L1t)
+    masked = tq.tq_quantize_act_rht(X, b, sg, L1t)
+    negated = tq.tq_quantize_act((X.double() * d).to(torch.bfloat16), b, L1t)
+    torch.cuda.synchronize()
+    assert all(torch.equal(u, v) for u, v in zip(plain, masked0))
+    assert torch.equal(masked[2], plain[2])
+    assert torch.equal(masked[0], negated[0]) and torch.equal(masked[1], negated[1])
 
 
 @pytest.mark.gpu
