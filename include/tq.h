@@ -266,16 +266,19 @@ TQ_API int tq_pack_shared_input(int n, const uint8_t* const* Wq, const float* co
  * means d_k = -1.  X L1 reads the unrotated X and is unchanged.
  *
  * tq_pack_weight_rht   -- tq_pack_weight with D H.
- * tq_quantize_act_rht  -- tq_quantize_act with D H: the butterfly kernel
- *                         for every M (the sign flips are exact, in
- *                         registers before the butterflies).
+ * tq_quantize_act_rht  -- tq_quantize_act with D H, on the same kernels:
+ *                         the butterflies (sign flips in registers before
+ *                         them), or for M >= 64 with had_block <= 128 the
+ *                         tensor-core kernel, which negates the masked
+ *                         columns of each staged X block (and of L1^T, so
+ *                         X L1 is unchanged) in shared memory before its
+ *                         MMAs.  Sign flips are exact either way.
  * tq_w4a4_lr_layer_rht -- tq_w4a4_lr_layer with D H (weights from
  *                         tq_pack_weight_rht with the same mask): the
  *                         one-kernel decode layer where it applies; for
- *                         M > 128 with had_block <= 128 the butterfly
- *                         kernel writing one code per byte and bf16(X L1),
- *                         then tq_w4a4_lr_gemm_a8 (the tensor-core
- *                         activation kernel takes no signs); else
+ *                         M > 128 with had_block <= 128 the tensor-core
+ *                         activation kernel writing one code per byte and
+ *                         bf16(X L1), then tq_w4a4_lr_gemm_a8; else
  *                         tq_quantize_act_rht + tq_w4a4_lr_gemm (packed
  *                         codes).  tq_layer_path reports the same choice.
  * Arguments and limits as the plain calls; `signs` 16-byte aligned.
@@ -297,7 +300,9 @@ TQ_API int tq_w4a4_lr_layer_rht(const uint16_t* X, const uint32_t* signs, const 
  * with n = n_rht in 1..3 masks, stored one after another in `signs`
  * ([n_rht][K / 32] words, the first applied first); weights packed by
  * tq_pack_weight_rhtn with the same masks.  The _rht calls above are
- * n_rht = 1.  Same arguments, paths and limits otherwise.
+ * n_rht = 1.  For n_rht > 1 the activations take the butterfly kernel at
+ * every M (above 128 tokens writing one code per byte for the int8-code
+ * GEMM).  Same arguments and limits otherwise.
  */
 TQ_API int tq_pack_weight_rhtn(const float* Rt, int N, int K, int had_block,
                                const uint32_t* signs, int n_rht, uint8_t* Wq, float* s_w,

@@ -22,6 +22,9 @@
 // Warp 0: TMA producer.  Warp 1: TMEM allocation and MMA issue.  Warps 2-9:
 // TMEM readers, two per lane quarter (warp w reads lanes 32*(w%4)..: token
 // rows of the tile; warps 2-5 columns 0-63 of each block, warps 6-9 64-127).
+// With a randomized Hadamard mask (x D H, the TORQUE page's RHT abstract: signs
+// first, then the Hadamard), warps 10-13 negate the masked columns of each
+// staged block in shared memory between the TMA's arrival and the MMAs.
 #include <cuda_bf16.h>
 #include <cudaTypedefs.h>
 
