@@ -108,12 +108,6 @@ __device__ __forceinline__ CodeScale code_scale(float am) {
 __device__ __forceinline__ uint32_t code_bits(float v, float inv) {
   return __float_as_uint(__fadd_rn(__fmul_rn(v, inv), 12582912.f));
 }
-// The same with the clip applied to y (for values that are not the exact
-// registers the absmax was taken over).
-__device__ __forceinline__ uint32_t code_bits_clip(float v, float inv) {
-  const float y = fminf(fmaxf(__fmul_rn(v, inv), -7.f), 7.f);
-  return __float_as_uint(__fadd_rn(y, 12582912.f));
-}
 // Byte j of the result is the low byte of the j-th argument.
 __device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);

@@ -41,7 +41,7 @@ namespace {
 constexpr int kTok = 128;          // tokens per tile (MMA M)
 constexpr int kBlk = 128;          // columns per block (MMA N of the rotation, MMA K)
 constexpr int kMaxNS = 3;          // X / L1^T stages: three where they fit, else two
-constexpr int kRot = 2;            // rotation accumulators in TMEM (128 columns each)
+constexpr int kRot = 3;            // rotation accumulators in TMEM (128 columns each)
 constexpr int kMaxC = 16;          // CTAs per cluster along K (above 8: non-portable size)
 constexpr int kMaxRtc = 128;       // X L1 width computed beside the codes
 constexpr int kMaxRx = 256;        // X L1 columns of one X-L1-only launch
@@ -132,6 +132,16 @@ __device__ __forceinline__ void cluster_arrive_rel() {
 // with `rows` rows per atom.
 __device__ __forceinline__ uint32_t atom_off(uint32_t row, uint32_t c, uint32_t rows) {
   return (c >> 3) * rows * 128u + row * 128u + (((c & 7u) ^ (row & 7u)) << 4);
+}
+
+// Two fp32 products in one packed multiply, each rounded to nearest even as
+// the scalar one.
+__device__ __forceinline__ void mul2_rn(uint32_t& a, uint32_t& b, float s) {
+  uint64_t x, sv;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(a), "r"(b));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sv) : "r"(__float_as_uint(s)));
+  asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(x) : "l"(sv));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(x));
 }
 
 // x D on a staged block: negate column k (bit k of the block's 128-bit mask
@@ -465,18 +475,31 @@ __global__ void __launch_bounds__(tc_threads<kSigned>(), 1)
           tmem_ld32(tmem_rot + (uint32_t)(u * kBlk + 32 * g) + lane_off, v);
           tmem_ld_wait();
           uint32_t cb[32];
+          if (asym) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float f = __uint_as_float(v[e]);
-            if (asym) {
+            for (int e = 0; e < 32; ++e) {
               // RoundClip((x - min) / s) to [0, 15] with ties to even, as
               // code - 8 in the byte (one fp32 subtraction, one product)
+              const float f = __uint_as_float(v[e]);
               float y = (f * cs.pre - mn * cs.pre) * cs.inv;
               y = fminf(fmaxf(y, 0.f), 15.f);
               cb[e] = __float_as_uint(__fadd_rn(y, 12582912.f)) - 8u;
-            } else {
-              if (cs.pre != 1.f) f *= cs.pre;
-              cb[e] = code_bits_clip(f, cs.inv);  // pass 2 recomputes the values
+            }
+          } else {
+            // code_bits of the values pass 1 took the absmax over (the MMA
+            // recomputes them bit for bit, so the clip never acts): the
+            // products two per packed multiply, the rounding adds one by one
+            // (a packed add after a packed multiply was contracted into one
+            // fma, whose single rounding moves exact fp32 ties)
+            if (cs.pre != 1.f) {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * cs.pre);
+            }
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              mul2_rn(v[e], v[e + 1], cs.inv);
+              cb[e] = __float_as_uint(__fadd_rn(__uint_as_float(v[e]), 12582912.f));
+              cb[e + 1] = __float_as_uint(__fadd_rn(__uint_as_float(v[e + 1]), 12582912.f));
             }
           }
           if (p.Xq8 && !asym) {

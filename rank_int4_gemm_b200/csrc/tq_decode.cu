@@ -170,18 +170,18 @@ __device__ __forceinline__ void bar_sync_workers() {
 // A wait of all worker warps: one lane polls the mbarrier (sleeping between
 // polls), the others block on a hardware barrier, so that waiting warps
 // (also those of the next layer's CTA on this SM) take no issue slots.
-// Returns the same outcome to every worker.
+// Returns the same verdict to every worker.
 template <bool kCluster>
 __device__ __forceinline__ bool workers_wait(uint64_t* bar, uint32_t* status,
-                                             volatile int* abort_flag, int* outcome) {
+                                             volatile int* abort_flag, int* verdict) {
   if (threadIdx.x == 0) {
     const bool ok = kCluster ? mbar_wait_cluster(bar, 0u, status, abort_flag)
                              : mbar_wait(bar, 0u, status, abort_flag);
-    *outcome = ok ? 1 : 0;
+    *verdict = ok ? 1 : 0;
   }
   bar_sync_workers();
-  const bool ok = *reinterpret_cast<volatile int*>(outcome) != 0;
-  bar_sync_workers();  // the outcome slot may be reused by the next wait
+  const bool ok = *reinterpret_cast<volatile int*>(verdict) != 0;
+  bar_sync_workers();  // the verdict slot may be reused by the next wait
   return ok;
 }
 __device__ __forceinline__ uint4 ldg_nc_v4(const void* ptr) {
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
   uint64_t* acc_full = bars + 8;     // [kMaxT]: tile j's MMAs done (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kMisc + 4);
-  int* outcome = reinterpret_cast<int*>(smem + S::kMisc + 8);
+  int* verdict = reinterpret_cast<int*>(smem + S::kMisc + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     const int row = 32 * q + lane;  // channel within a tile = TMEM lane
 
     // ---- 1. weights int4 -> int8 (16 * code): tiles h and h + 2
-    bool ok = workers_wait<false>(w_full, p.status, abort_flag, outcome);
+    bool ok = workers_wait<false>(w_full, p.status, abort_flag, verdict);
     uint4 t3[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) t3[c] = make_uint4(0u, 0u, 0u, 0u);
@@ -398,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     tmem_st_wait();
 
     // ---- 2. rotation of tokens warp and warp + 8, partial absmax
-    ok = workers_wait<false>(x_full, p.status, abort_flag, outcome) && ok;
+    ok = workers_wait<false>(x_full, p.status, abort_flag, verdict) && ok;
     float v[2][8];
     float am_part[2] = {0.f, 0.f};
 #pragma unroll
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     }
 
     // ---- 3. codes with the cluster-wide absmax -> the MMAs may start
-    ok = workers_wait<true>(amax_bar, p.status, abort_flag, outcome) && ok;
+    ok = workers_wait<true>(amax_bar, p.status, abort_flag, verdict) && ok;
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       const int t = warp + 8 * tt;
@@ -493,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
       constexpr int kKP = 8 / kNt;           // k-parts: 4, 2 or 1
       constexpr int kSteps = (kSlice / 16) / kKP;
       constexpr int kGrp = kSteps < 8 ? kSteps : 8;  // operands held at once
-      const bool l1_ok = workers_wait<false>(l1_full, p.status, abort_flag, outcome);
+      const bool l1_ok = workers_wait<false>(l1_full, p.status, abort_flag, verdict);
       ok = ok && l1_ok;
       const int nt = warp % kNt, kp = warp / kNt;
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -553,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
       // ---- 4b. owned tokens: X L1 = sum of the C partials (cluster order),
       //          bf16, to every CTA
       if (own_tok > 0) {
-        const bool got = workers_wait<true>(xl1p_bar, p.status, abort_flag, outcome);
+        const bool got = workers_wait<true>(xl1p_bar, p.status, abort_flag, verdict);
         constexpr int kR8 = R / 8;
         if (tid < own_tok * kR8) {
           const int li = tid / kR8, c8 = tid - li * kR8;
@@ -608,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     for (int jj = 0; jj < 2; ++jj) {
       const int j = h + 2 * jj;
       if (j >= p.T) continue;  // warp-uniform
-      // one lane of each warp polls; its warp-mates take its outcome
+      // one lane of each warp polls; its warp-mates take its verdict
       bool got = true;
       if (lane == 0) got = mbar_wait(&acc_full[j], 0u, p.status, abort_flag);
       got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
@@ -642,8 +642,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm<R>)
     // ---- 6. owner epilogue: Y[t][n] for the owned channels, four tokens
     //         per item (the waits' named barriers also make s_x of every
     //         token, written in step 3 by other threads, visible here)
-    ok = workers_wait<true>(part_bar, p.status, abort_flag, outcome) && ok;
-    if (R > 0) ok = workers_wait<true>(xl1b_bar, p.status, abort_flag, outcome) && ok;
+    ok = workers_wait<true>(part_bar, p.status, abort_flag, verdict) && ok;
+    if (R > 0) ok = workers_wait<true>(xl1b_bar, p.status, abort_flag, verdict) && ok;
     if (ok) {
       const int items = per * 4;
       for (int it = tid; it < items; it += kWorkers) {
